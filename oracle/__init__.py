@@ -1,0 +1,191 @@
+"""Float64 CPU oracle for learnable-sink attention (ctypes shim).
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package.  The CUDA library and
+its Python binding never do; the two implementations share no code.
+
+The arithmetic lives in ``sinkattn_oracle.c`` (plain C, float64, OpenMP over
+rows), which follows the page "Attention Sink, Learnable Sink and dsink"
+(notes.kuangjux.top): the forward of section 4 with the sink as an explicit
+extra softmax column, the backward as the explicit Jacobian of that augmented
+softmax (sections 7-8), the visible set of section 2, and the StreamingLLM
+ring-buffer KV set (sink segment + sliding window).
+
+Every function takes and returns numpy arrays; floating-point inputs are
+converted to float64 here (the caller passes the same rounded values the GPU
+sees).  The mask is given as plain keyword arguments:
+``causal, n_sink, window, cu_seqlens, block_indices, block_q, block_k``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sinkattn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libsinkattn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_d = ctypes.POINTER(ctypes.c_double)
+_i32 = ctypes.POINTER(ctypes.c_int32)
+_u8 = ctypes.POINTER(ctypes.c_uint8)
+_PROBLEM = [ctypes.c_int] * 4 + [ctypes.c_double] + [ctypes.c_int] * 3 + [
+    _i32, ctypes.c_int, ctypes.c_int, _i32, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
+                               "-std=c11", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            lib.oracle_fwd.argtypes = _PROBLEM + [_d, _d, _d, _d, _d, _d, _d]
+            lib.oracle_fwd_rows.argtypes = _PROBLEM + [
+                _d, _d, _d, _d, ctypes.c_int, _i32, _d, _d, _d]
+            lib.oracle_bwd.argtypes = _PROBLEM + [_d, _d, _d, _d, _d, _d, _d, _d, _d]
+            lib.oracle_decode.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [
+                _d, _d, _d, _i32, ctypes.c_int, ctypes.c_int, _d, _d, _d, _d]
+            lib.oracle_visible_dense.argtypes = _PROBLEM + [ctypes.c_int, _u8]
+            lib.oracle_tile_states.argtypes = _PROBLEM + [
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, _u8]
+            lib.oracle_num_threads.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i32arr(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _p(a, typ):
+    return None if a is None else a.ctypes.data_as(typ)
+
+
+class _Problem:
+    """Shapes and mask fields in the order the C functions take them."""
+
+    def __init__(self, T_tot, Hq, Hkv, D, scale, causal=True, n_sink=0, window=0,
+                 cu_seqlens=None, block_indices=None, block_q=64, block_k=64):
+        self.cu = _i32arr(cu_seqlens)
+        if self.cu is None:
+            self.cu = np.array([0, T_tot], dtype=np.int32)
+        self.n_seq = len(self.cu) - 1
+        self.bi = _i32arr(block_indices)
+        self.max_blocks = 0 if self.bi is None else int(self.bi.shape[-1])
+        self.args = (int(T_tot), int(Hq), int(Hkv), int(D), float(scale),
+                     int(bool(causal)), int(n_sink), int(window),
+                     _p(self.cu, _i32), self.n_seq, 0, _p(self.bi, _i32),
+                     int(block_q), int(block_k), self.max_blocks)
+
+
+def _shapes(q, k):
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    return T, Hq, Hkv, D
+
+
+def fwd(q, k, v, sink, scale, **mask):
+    """Returns (out [T,Hq,D], lse_new [T,Hq], sink_s [T,Hq]) in float64."""
+    q, k, v, sink = _f64(q), _f64(k), _f64(v), _f64(sink)
+    T, Hq, Hkv, D = _shapes(q, k)
+    pr = _Problem(T, Hq, Hkv, D, scale, **mask)
+    out = np.zeros((T, Hq, D)); lse = np.zeros((T, Hq)); ss = np.zeros((T, Hq))
+    _load().oracle_fwd(*pr.args, _p(q, _d), _p(k, _d), _p(v, _d), _p(sink, _d),
+                       _p(out, _d), _p(lse, _d), _p(ss, _d))
+    return out, lse, ss
+
+
+def fwd_rows(q, k, v, sink, scale, rows, **mask):
+    """Forward of selected (token, head) rows: rows int array [n, 2].
+    Returns (out [n,D], lse [n], sink_s [n])."""
+    q, k, v, sink = _f64(q), _f64(k), _f64(v), _f64(sink)
+    T, Hq, Hkv, D = _shapes(q, k)
+    rows = _i32arr(rows).reshape(-1, 2)
+    n = rows.shape[0]
+    pr = _Problem(T, Hq, Hkv, D, scale, **mask)
+    out = np.zeros((n, D)); lse = np.zeros(n); ss = np.zeros(n)
+    _load().oracle_fwd_rows(*pr.args, _p(q, _d), _p(k, _d), _p(v, _d), _p(sink, _d),
+                            n, _p(rows, _i32), _p(out, _d), _p(lse, _d), _p(ss, _d))
+    return out, lse, ss
+
+
+def bwd(q, k, v, sink, dout, scale, **mask):
+    """Returns (dq, dk, dv, dsink) in float64; dsink is None without a sink."""
+    q, k, v, sink, dout = _f64(q), _f64(k), _f64(v), _f64(sink), _f64(dout)
+    T, Hq, Hkv, D = _shapes(q, k)
+    pr = _Problem(T, Hq, Hkv, D, scale, **mask)
+    dq = np.zeros((T, Hq, D)); dk = np.zeros((T, Hkv, D)); dv = np.zeros((T, Hkv, D))
+    dsink = np.zeros(Hq) if sink is not None else None
+    rc = _load().oracle_bwd(*pr.args, _p(q, _d), _p(k, _d), _p(v, _d), _p(sink, _d),
+                            _p(dout, _d), _p(dq, _d), _p(dk, _d), _p(dv, _d),
+                            _p(dsink, _d))
+    if rc != 0:
+        raise MemoryError("oracle_bwd: allocation failed")
+    return dq, dk, dv, dsink
+
+
+def decode(q, k_cache, v_cache, cache_seqlens, n_sink, window, sink, scale):
+    """Ring-buffer decode. q [B,Hq,D], caches [B,S,Hkv,D] (S = n_sink+window).
+    Returns (out [B,Hq,D], lse_new [B,Hq], sink_s [B,Hq])."""
+    q, kc, vc, sink = _f64(q), _f64(k_cache), _f64(v_cache), _f64(sink)
+    cs = _i32arr(cache_seqlens)
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    out = np.zeros((B, Hq, D)); lse = np.zeros((B, Hq)); ss = np.zeros((B, Hq))
+    _load().oracle_decode(B, Hq, Hkv, D, float(scale), _p(q, _d), _p(kc, _d),
+                          _p(vc, _d), _p(cs, _i32), int(n_sink), int(window),
+                          _p(sink, _d), _p(out, _d), _p(lse, _d), _p(ss, _d))
+    return out, lse, ss
+
+
+def visible_dense(T_tot, Hq, Hkv, g, **mask):
+    """Dense visibility matrix [T, T] (uint8) of KV head g."""
+    pr = _Problem(T_tot, Hq, Hkv, 1, 1.0, **mask)
+    vis = np.zeros((T_tot, T_tot), dtype=np.uint8)
+    _load().oracle_visible_dense(*pr.args, int(g), _p(vis, _u8))
+    return vis
+
+
+def tile_states(T_tot, Hq, Hkv, tile_q, tile_k, **mask):
+    """Brute-force tile classification: uint8 [Hkv, n_qtiles, max_ktiles]
+    with 0 = no visible pair, 1 = partly visible, 2 = fully visible."""
+    pr = _Problem(T_tot, Hq, Hkv, 1, 1.0, **mask)
+    lens = np.diff(pr.cu)
+    nqt = int(sum((int(l) + tile_q - 1) // tile_q for l in lens))
+    max_kt = int((int(lens.max()) + tile_k - 1) // tile_k) if len(lens) else 0
+    st = np.zeros((Hkv, max(nqt, 1), max(max_kt, 1)), dtype=np.uint8)
+    _load().oracle_tile_states(*pr.args, int(tile_q), int(tile_k), max(max_kt, 1),
+                               _p(st, _u8))
+    return st[:, :nqt, :max_kt]
