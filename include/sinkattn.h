@@ -1,0 +1,227 @@
+/*
+ * sinkattn.h -- C ABI of libsinkattn.so: grouped-query attention whose softmax
+ * denominator carries a per-head learnable sink logit, for B200 (sm_100a).
+ *
+ * The operation (page "Attention Sink, Learnable Sink and dsink",
+ * notes.kuangjux.top; section 1 for the scores and GQA head map, section 4
+ * for the sink, sections 7-8 for the gradients):
+ *
+ *   x_ijh   = scale * <Q_ih, K_j,g(h)>,   g(h) = h / (Hq / Hkv)
+ *   Z_ih    = sum_{j visible} e^{x_ijh},  L_orig = log Z
+ *   L_new   = log(Z + e^{a_h})            (the sink logit a_h is NOT scaled)
+ *   sink_s  = Z / (Z + e^{a_h}) = sigma(L_orig - a_h)   (mass on real tokens)
+ *   O_ih    = sink_s * sum_j (e^{x_ijh} / Z) V_j,g(h)   (= O_orig scaled by s)
+ *   dsink_h = -sum_i Delta_ih * p_sink_ih,  Delta_ih = <dO_ih, O_ih>,
+ *             p_sink = e^{a_h - L_new}    (section 7 boxed result; section 10
+ *             recommends exp(a - LSE_total) over 1 - sink_s)
+ *   dQ/dK/dV: the usual softmax gradients with P = e^{x - L_new} and Delta
+ *             computed from the sink-scaled O (section 8).
+ *
+ * learnable_sink == NULL disables the sink (page 1 section 4: "None"); a sink
+ * of 0 still adds e^0 = 1 to the denominator.
+ *
+ * Visible set (page 1 section 2: block selection, window, causality and
+ * sample boundaries all restrict it).  With sequence-local positions qi, kj
+ * of the same packed sequence:
+ *   causal                 => kj <= qi
+ *   window > 0             => kj < n_sink  or  qi - kj < window   (StreamingLLM
+ *                             KV set: initial sink tokens plus a recent window)
+ *   block_indices != NULL  => kj / block_k is listed for (KV head g(h),
+ *                             query block qi / block_q).
+ *
+ * Layouts (token-major, packed varlen; page 1 sections 1 and 7: out [T, Hq, D],
+ * delta [T, Hq], dsink [Hq]):
+ *   Q, O, dQ, dO : [T_tot, Hq, D]     K, V, dK, dV : [T_tot, Hkv, D]
+ *   LSE_new, sink_s : [T_tot, Hq] float32     learnable_sink, dsink : [Hq] float32
+ *   All tensors contiguous, row-major as written.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer is DEVICE memory owned by the caller (except the
+ *     sinkattn_mask struct itself, which is read on the host during the call).
+ *     The library never allocates device memory; scratch comes from the
+ *     caller's workspace, sized by the *_bytes queries.
+ *   - Work is enqueued asynchronously on `stream`; a return of SINKATTN_OK
+ *     means arguments were valid and kernels were launched.  Errors detected
+ *     on the device (a bounded wait that ran out, an out-of-range block index)
+ *     are recorded in a per-device status word read by sinkattn_get_status().
+ *   - Arguments are validated on the host first; on any invalid argument
+ *     nothing is launched and SINKATTN_ERR_INVALID_ARG is returned.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Nothing is written to the inputs (q, k, v, learnable_sink, masks).
+ */
+#ifndef SINKATTN_H_
+#define SINKATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *sinkattn_stream_t;
+
+/* Return codes. */
+#define SINKATTN_OK 0
+#define SINKATTN_ERR_INVALID_ARG 1 /* bad pointer, shape, alignment or mask   */
+#define SINKATTN_ERR_UNSUPPORTED 2 /* device is not sm_100, or dtype/D combo  */
+#define SINKATTN_ERR_CUDA 3        /* a CUDA runtime/driver call failed        */
+#define SINKATTN_ERR_WORKSPACE 4   /* workspace/plan buffer too small          */
+#define SINKATTN_ERR_TIMEOUT 5     /* device: a bounded barrier wait ran out   */
+#define SINKATTN_ERR_BOUNDS 6      /* device: block index out of range         */
+#define SINKATTN_ERR_PLAN 7        /* plan built for a different problem       */
+
+/* Element type of Q/K/V/O/dO/dQ/dK/dV.  LSE, sink_s, sinks and dsink are
+ * always float32 (page 1 section 9: sink_s is kept in FP32). */
+typedef enum {
+    SINKATTN_BF16 = 0, /* tensor-core path (tcgen05), fp32 accumulation   */
+    SINKATTN_FP32 = 2  /* exact-fp32 CUDA-core path                        */
+} sinkattn_dtype;
+
+/* Mask descriptor (read on the host during the call; the arrays it points to
+ * are device memory).
+ *   causal        1: key kj visible only if kj <= qi (sequence-local).
+ *   n_sink        with window > 0: keys [0, n_sink) of each sequence stay
+ *                 visible (StreamingLLM keeps 4).
+ *   window        > 0: also visible if qi - kj < window (requires causal);
+ *                 0: no window restriction.
+ *   cu_seqlens    device int32 [n_seq + 1], cu_seqlens[0] = 0,
+ *                 cu_seqlens[n_seq] = T_tot, non-decreasing.  Sequences never
+ *                 attend across their boundary.  Required.
+ *   n_seq         number of packed sequences (>= 1).
+ *   max_seqlen    an upper bound on every sequence length (used for sizing).
+ *   block_indices NULL, or device int32 [Hkv, n_qblk, max_blocks]: for each
+ *                 KV head and each sequence-local query block (numbered
+ *                 globally in sequence order: sum over sequences of
+ *                 ceil(len / block_q) rows), the sequence-local key blocks it
+ *                 may see; -1 entries are padding, duplicates are ignored.
+ *                 The diagonal block is NOT added implicitly.  An index
+ *                 >= ceil(len / block_k) or < -1 sets SINKATTN_ERR_BOUNDS in
+ *                 the status word and is skipped.
+ *   n_qblk        rows of block_indices per KV head (ignored when NULL).
+ *   block_q, block_k  block sizes; with block_indices both must be equal and
+ *                 64 or 128.  Ignored when block_indices is NULL.
+ *   max_blocks    entries per row, 1..32 (ignored when NULL). */
+typedef struct {
+    int32_t causal;
+    int32_t n_sink;
+    int32_t window;
+    const int32_t *cu_seqlens;
+    int32_t n_seq;
+    int32_t max_seqlen;
+    const int32_t *block_indices;
+    int32_t n_qblk;
+    int32_t block_q;
+    int32_t block_k;
+    int32_t max_blocks;
+} sinkattn_mask;
+
+/* ---- tile schedule ("plan") ---------------------------------------------
+ * The mask is turned into a tile schedule once and reused by forward and
+ * backward (and by every layer that shares the mask).  For each query tile
+ * and KV head it lists the key tiles holding at least one visible pair, each
+ * flagged full (no element mask needed) or partial; for each key tile the
+ * reverse list of query tiles (reverse CSR, used by the backward).  Fully
+ * masked tiles are never visited.  Query tiles are 128 tokens (block_q with
+ * block_indices), key tiles 128 keys (block_k with block_indices); tiles are
+ * sequence-local (a tile never spans two sequences).
+ *
+ * sinkattn_plan_bytes returns the plan buffer size needed for this shape and
+ * mask (an upper bound; depends on T_tot, Hkv, n_seq, max_seqlen and the
+ * block sizes only, not on the contents of cu_seqlens/block_indices), or 0 if
+ * the arguments are invalid.  sinkattn_plan fills `plan` (device memory,
+ * 16-byte aligned, caller-owned) on `stream`; forward and backward calls
+ * later in stream order may read it.  The plan stays valid as long as the
+ * mask arrays' contents do not change. */
+size_t sinkattn_plan_bytes(int T_tot, int Hq, int Hkv, const sinkattn_mask *mask);
+int sinkattn_plan(int T_tot, int Hq, int Hkv, const sinkattn_mask *mask,
+                  void *plan, size_t plan_bytes, sinkattn_stream_t stream);
+
+/* ---- forward --------------------------------------------------------------
+ * Computes O, LSE_new and sink_s (page 1 section 4; page 4 section 5's gate
+ * G = sigma(LSE - sink) equals sink_s).
+ *   dt        SINKATTN_BF16 (D = 64 or 128) or SINKATTN_FP32 (D = 64 or 128).
+ *   T_tot     total packed tokens (>= 1).   Hq % Hkv == 0.
+ *   scale     softmax scale alpha (typically 1/sqrt(D)).
+ *   q, k, v   inputs of type dt, layouts above.
+ *   learnable_sink  float32 [Hq] or NULL.
+ *   mask      the mask the plan was built from.
+ *   plan      built by sinkattn_plan for the same T_tot/Hq/Hkv/mask.
+ *   out       [T_tot, Hq, D] of type dt (written).
+ *   lse_new   float32 [T_tot, Hq] (written; natural log, includes the sink;
+ *             -inf for a row that sees no key and has no sink).
+ *   sink_s    float32 [T_tot, Hq] or NULL (written if non-NULL; 0 for a row
+ *             that sees no key).
+ * A row that sees no key gets O = 0 (and LSE = a_h, sink_s = 0 with a sink). */
+int sinkattn_fwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                 const void *q, const void *k, const void *v,
+                 const float *learnable_sink, const sinkattn_mask *mask,
+                 const void *plan, size_t plan_bytes,
+                 void *out, float *lse_new, float *sink_s,
+                 sinkattn_stream_t stream);
+
+/* ---- backward -------------------------------------------------------------
+ * Computes dQ, dK, dV and dsink (page 1 sections 7-8).
+ *   out, lse_new  the forward's O and LSE_new (sink-inclusive).
+ *   dout          upstream gradient dL/dO, [T_tot, Hq, D] of type dt.
+ *   learnable_sink  float32 [Hq] or NULL (then dsink is not written).
+ *   dq, dk, dv    outputs of type dt (overwritten, not accumulated).
+ *   dsink         float32 [Hq] (overwritten; summed over every query of every
+ *                 sequence, no division by the token count, section 7).
+ *   workspace     device scratch of at least sinkattn_bwd_workspace_bytes().
+ * dK/dV sum over the Hq/Hkv query heads of each KV head.  dsink is computed
+ * once per query (section 10's double-counting warning) in the Delta
+ * preprocess and reduced deterministically. */
+size_t sinkattn_bwd_workspace_bytes(sinkattn_dtype dt, int T_tot, int Hq, int Hkv,
+                                    int D, const sinkattn_mask *mask);
+int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                 const void *q, const void *k, const void *v, const void *out,
+                 const void *dout, const float *lse_new,
+                 const float *learnable_sink, const sinkattn_mask *mask,
+                 const void *plan, size_t plan_bytes,
+                 void *dq, void *dk, void *dv, float *dsink,
+                 void *workspace, size_t workspace_bytes, sinkattn_stream_t stream);
+
+/* ---- ring-buffer decode ---------------------------------------------------
+ * One query token per sequence attends over a StreamingLLM KV cache: n_sink
+ * fixed slots holding the first tokens plus a circular window of `window`
+ * slots holding the most recent ones (page 3: a fixed sink segment plus a
+ * sliding window; the oldest non-sink entry is overwritten).
+ *   q              [B, Hq, D] of type dt.
+ *   k_cache, v_cache  [B, S, Hkv, D], S = n_sink + window.  Token at absolute
+ *                  position p lives in slot p if p < n_sink, else in slot
+ *                  n_sink + (p - n_sink) % window.
+ *   cache_seqlens  device int32 [B]: tokens ever appended to sequence b,
+ *                  the current token included (>= 0).  Slots
+ *                  [0, min(cache_seqlens[b], S)) hold valid tokens.
+ *   learnable_sink float32 [Hq] or NULL.
+ *   out [B, Hq, D] (type dt), lse_new / sink_s float32 [B, Hq] (sink_s may be
+ *   NULL).
+ *   num_splits     key splits per (sequence, KV head); 0 picks one.
+ *   workspace      at least sinkattn_decode_workspace_bytes(B, Hq, D, splits).
+ * Since no positional encoding is applied inside, the result depends only on
+ * which tokens are in the cache, not on where the ring head is. */
+size_t sinkattn_decode_workspace_bytes(int B, int Hq, int D, int num_splits);
+int sinkattn_decode_num_splits(int B, int Hq, int Hkv, int D, int n_sink, int window);
+int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scale,
+                    const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *cache_seqlens, int n_sink, int window,
+                    const float *learnable_sink, void *out, float *lse_new,
+                    float *sink_s, int num_splits, void *workspace,
+                    size_t workspace_bytes, sinkattn_stream_t stream);
+
+/* ---- status ---------------------------------------------------------------
+ * sinkattn_get_status synchronises `stream`, then returns the first error code
+ * any kernel of this library recorded on the current device since the last
+ * sinkattn_clear_status (SINKATTN_OK if none), or SINKATTN_ERR_CUDA if the
+ * synchronisation itself failed. */
+int sinkattn_get_status(sinkattn_stream_t stream);
+int sinkattn_clear_status(sinkattn_stream_t stream);
+const char *sinkattn_error_string(int code);
+int sinkattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SINKATTN_H_ */

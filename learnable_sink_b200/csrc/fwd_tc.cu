@@ -1,0 +1,475 @@
+// Forward pass on the 5th-generation tensor cores (tcgen05) for bf16 inputs.
+//
+// Page "Attention Sink, Learnable Sink and dsink": scores and GQA map
+// (section 1), the sink logit folded into the softmax denominator with a zero
+// value (section 4), LSE_new and the gate sink_s (sections 4 and 9); page
+// "Attention Sink Forges Native MoE" (section 5) reads the same gate as
+// G = sigma(LSE - sink).
+//
+// One CTA = NQT query tiles of 128 rows that share a token range and a KV
+// head (a tile is 128 tokens of one head, or 64 tokens x 2 heads), and one
+// list of key tiles from the plan.  Warp roles:
+//   warps [0, 4 NQT)  softmax: warpgroup t owns query tile t, one thread per
+//                     row (TMEM lane = row); online softmax in registers,
+//                     lazy rescaling of the TMEM O accumulator, epilogue.
+//   warp 4 NQT        TMA producer: Q once, then K and V tiles through an
+//                     NS-stage mbarrier ring.
+//   warp 4 NQT + 1    MMA issuer (one thread): S_t = Q_t K^T (SS, smem
+//                     operands) and O_t += P_t V (TS, P read from TMEM where
+//                     softmax wrote it over S_t).
+// Tensor memory: S_t at columns [t TK, (t+1) TK), O_t after all S tiles.
+// The two query tiles ping-pong: while warpgroup 0 exponentiates S_0 the
+// tensor core runs tile 1's MMAs and vice versa.
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+
+namespace sk {
+
+namespace {
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
+
+template <int D_, int TQ_, int TK_, int NQT_>
+struct FwdCfg {
+  static constexpr int D = D_, TQ = TQ_, TK = TK_, NQT = NQT_;
+  static constexpr int HPT = 128 / TQ;           // heads per query tile
+  static constexpr int DH = D / 64;              // 64-column halves of a row
+  static constexpr int Q_BYTES = 128 * D * 2;    // one query tile
+  static constexpr int KV_BYTES = TK * D * 2;    // one K (or V) tile
+  static constexpr int SMEM_BUDGET = 200 * 1024;
+  static constexpr int NS_RAW = (SMEM_BUDGET - NQT * Q_BYTES) / (2 * KV_BYTES);
+  static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
+  static_assert(NS >= 2, "not enough shared memory for a two-stage ring");
+  static constexpr int THREADS = (4 * NQT + 2) * 32;
+  static constexpr int PRODUCER_WARP = 4 * NQT;
+  static constexpr int MMA_WARP = 4 * NQT + 1;
+  static constexpr int S_COL = 0;                // S_t at t * TK
+  static constexpr int O_COL = NQT * TK;         // O_t at O_COL + t * D
+  static constexpr int TMEM_NEED = NQT * (TK + D);
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
+                                 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
+  static_assert(TMEM_NEED <= 512, "tensor memory budget");
+  // shared memory layout (offsets from a 1024-aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQT * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
+  static constexpr int N_BARS = 1 + 4 * NS + 3 * NQT + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  static constexpr int MIN_BLOCKS = (TK == 64 && D == 64) ? 2 : 1;
+};
+
+struct FwdParams {
+  const int* plan;
+  const float* sink;
+  __nv_bfloat16* out;
+  float* lse;
+  float* sink_s;
+  int* status;
+  int Hq, Hkv, G, causal, n_sink, window;
+  int per_item, chunks;  // CTAs per plan item, head chunks per KV head
+  float scale_log2;
+};
+
+__device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitBudgetCycles) return false;
+  return true;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                  const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
+  constexpr int D = C::D, TK = C::TK, NQT = C::NQT, HPT = C::HPT, NS = C::NS, DH = C::DH;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kf = bars + 1;
+  uint64_t* bar_ke = bar_kf + NS;
+  uint64_t* bar_vf = bar_ke + NS;
+  uint64_t* bar_ve = bar_vf + NS;
+  uint64_t* bar_s = bar_ve + NS;
+  uint64_t* bar_p = bar_s + NQT;
+  uint64_t* bar_o = bar_p + NQT;
+  uint64_t* bar_fin = bar_o + NQT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const PlanHdr* hdr = reinterpret_cast<const PlanHdr*>(p.plan);
+  const int rank = blockIdx.x / p.per_item;
+  if (rank >= hdr->n_fwd_items) return;
+  const int rem = blockIdx.x % p.per_item;
+  const int idx = p.plan[hdr->off_fwd_order + rank];
+  const TileItem it = reinterpret_cast<const TileItem*>(p.plan + hdr->off_fwd_items)[idx];
+  const int kvh = it.kvh >= 0 ? it.kvh : rem / p.chunks;
+  const int chunk = rem % p.chunks;
+  const int head0 = kvh * p.G + chunk * NQT * HPT;
+  const int* ent = p.plan + hdr->off_fwd_entries + it.entry_off;
+  const int n = it.entry_len;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_kf + s, 1);
+      mbar_init(bar_ke + s, 1);
+      mbar_init(bar_vf + s, 1);
+      mbar_init(bar_ve + s, 1);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(bar_s + t, 1);
+      mbar_init(bar_p + t, 128);
+      mbar_init(bar_o + t, 1);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n > 0) {
+      const int tok0 = it.seq_start + it.tile_start;
+      mbar_expect_tx(bar_q, NQT * C::Q_BYTES);
+      for (int t = 0; t < NQT; ++t)
+        for (int h = 0; h < DH; ++h)
+          tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_q, bar_q,
+                      h * 64, head0 + t * HPT, tok0);
+      int last_k[NS], last_v[NS];
+      for (int s = 0; s < NS; ++s) last_k[s] = last_v[s] = -1;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int s = j % NS;
+        const uint32_t par = ((j / NS) & 1) ^ 1;
+        const int krow = it.seq_start + (__ldg(ent + j) >> 1) * TK;
+        ok = mbar_wait(bar_ke + s, par, abort_flag, p.status);
+        if (!ok) break;
+        mbar_expect_tx(bar_kf + s, C::KV_BYTES);
+        for (int h = 0; h < DH; ++h)
+          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + h * (C::KV_BYTES / DH), &tmap_k,
+                      bar_kf + s, h * 64, kvh, krow);
+        last_k[s] = j;
+        ok = mbar_wait(bar_ve + s, par, abort_flag, p.status);
+        if (!ok) break;
+        mbar_expect_tx(bar_vf + s, C::KV_BYTES);
+        for (int h = 0; h < DH; ++h)
+          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + h * (C::KV_BYTES / DH), &tmap_v,
+                      bar_vf + s, h * 64, kvh, krow);
+        last_v[s] = j;
+      }
+      if (!ok) {  // let copies already in flight land before the CTA exits
+        wait_noabort(bar_q, 0);
+        for (int s = 0; s < NS; ++s) {
+          if (last_k[s] >= 0) wait_noabort(bar_kf + s, (last_k[s] / NS) & 1);
+          if (last_v[s] >= 0) wait_noabort(bar_vf + s, (last_v[s] / NS) & 1);
+        }
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, TK, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t sq = smem_u32(smem + C::OFF_Q), sk = smem_u32(smem + C::OFF_K),
+                     sv = smem_u32(smem + C::OFF_V);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status);
+      for (int j = 0; j <= n && ok; ++j) {
+        if (j < n) ok = mbar_wait(bar_kf + j % NS, (j / NS) & 1, abort_flag, p.status);
+        if (ok && j > 0) ok = mbar_wait(bar_vf + (j - 1) % NS, ((j - 1) / NS) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (j > 0) {
+            ok = mbar_wait(bar_p + t, (j - 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t vbase = sv + ((j - 1) % NS) * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < TK / 16; ++kk) {
+              // B = V tile, MN-major: 64-column atoms TK*128 B apart, 8-row groups 1 KB apart
+              const uint64_t bdesc = sdesc_sw128(vbase + kk * 16 * 128, TK * 128, 1024);
+              mma_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * TK + kk * 8, bdesc, idesc_pv,
+                     (j > 1 || kk > 0) ? 1u : 0u);
+            }
+          }
+          if (j < n) {
+            const uint32_t qbase = sq + t * C::Q_BYTES;
+            const uint32_t kbase = sk + (j % NS) * C::KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B inside the 128-B row
+              const uint64_t adesc = sdesc_sw128(qbase + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024);
+              const uint64_t bdesc = sdesc_sw128(kbase + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024);
+              mma_ss(tmem + C::S_COL + t * TK, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_s + t);
+          }
+        }
+        if (!ok) break;
+        if (j > 0) mma_commit(bar_ve + (j - 1) % NS);
+        if (j < n) mma_commit(bar_ke + j % NS);
+      }
+      if (ok)
+        for (int t = 0; t < NQT; ++t) mma_commit(bar_o + t);
+      // drain: every MMA issued by this thread has completed once bar_fin fires
+      mma_commit(bar_fin);
+      wait_noabort(bar_fin, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp / 4;                     // query tile of this warpgroup
+    const int wq = warp % 4;                    // TMEM lane quadrant
+    const int r = wq * 32 + lane;               // row of the tile
+    const int tok = r / HPT, hh = r % HPT;
+    const int head = head0 + t * HPT + hh;
+    const int qi = it.tile_start + tok;         // sequence-local query position
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + C::S_COL + t * TK;
+    const uint32_t o_addr = tmem + lane_off + C::O_COL + t * D;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int e = __ldg(ent + j);
+      const int k0 = (e >> 1) * TK;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s + t, j & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      float x[TK];
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(s_addr + c * 32, rr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(rr[i]) * p.scale_log2;
+      }
+      if (e & 1) {  // partial tile: element mask
+#pragma unroll
+        for (int c = 0; c < TK; ++c)
+          if (!visible_elem(qi, k0 + c, it.seq_len, p.causal, p.n_sink, p.window)) x[c] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < TK; ++c) mx = fmaxf(mx, x[c]);
+      // Lazy rescale: the running reference max m only moves when the tile
+      // max exceeds it by more than 2^8.  Per-row decision, but the TMEM
+      // load/store are warp-collective, so the warp rescales together and
+      // rows that need nothing multiply by 1.
+      const bool need = mx > m + kRescaleThreshold;  // true on the first visible tile
+      float corr = 1.f;
+      if (need) {
+        corr = exp2f(m - mx);  // 0 when m = -inf
+        l *= corr;
+      }
+      const bool touch_o = need && j > 0 && m != -INFINITY;
+      if (__any_sync(0xffffffffu, touch_o)) {
+        // O_t row *= corr.  Safe: PV_t(j-1) completed before S_t(j) was
+        // signalled (tcgen05 operations complete in issue order).
+        const float f = touch_o ? corr : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(o_addr + c * 32, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
+          tmem_st32(o_addr + c * 32, rr);
+        }
+      }
+      if (need) m = mx;
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < TK / 64; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = fast_exp2(x[c * 64 + 2 * i] - mu);
+          const float p1 = fast_exp2(x[c * 64 + 2 * i + 1] - mu);
+          rs += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_addr + c * 32, pk);  // P over the first TK/2 columns of S_t
+      }
+      l += rs;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p + t);
+    }
+    // epilogue: fold the sink into the denominator (log2 domain) and stream
+    // O out of tensor memory 32 columns at a time
+    const bool have_o =
+        __all_sync(0xffffffffu, n > 0 && ok && mbar_wait(bar_o + t, 0, abort_flag, p.status));
+    if (n > 0 && !have_o) ok = false;
+    if (ok && tok < it.tile_len) {
+      const float a2 = p.sink ? __ldg(p.sink + head) * kLog2e : -INFINITY;
+      const float mt = fmaxf(m, a2);
+      float o_scale = 0.f, lse_v = -INFINITY, ss = 0.f;
+      if (mt != -INFINITY) {
+        const float fr = (m == -INFINITY) ? 0.f : exp2f(m - mt);
+        const float lr = l * fr;
+        const float den = lr + (p.sink ? exp2f(a2 - mt) : 0.f);
+        o_scale = fr / den;
+        lse_v = (mt + log2f(den)) * kLn2;
+        ss = lr / den;
+      }
+      const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
+      p.lse[row] = lse_v;
+      if (p.sink_s) p.sink_s[row] = ss;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * D);
+      if (!have_o) {
+        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = z;
+      }
+    }
+    if (have_o) {
+      // all 32 lanes of the warp take part in the tcgen05.ld
+      tc_fence_after();
+      const bool store = ok && tok < it.tile_len;
+      float o_scale = 0.f;
+      if (store) {
+        const float a2 = p.sink ? __ldg(p.sink + head) * kLog2e : -INFINITY;
+        const float mt = fmaxf(m, a2);
+        if (mt != -INFINITY) {
+          const float fr = (m == -INFINITY) ? 0.f : exp2f(m - mt);
+          const float den = l * fr + (p.sink ? exp2f(a2 - mt) : 0.f);
+          o_scale = fr / den;
+        }
+      }
+      const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(o_addr + c * 32, rr);
+        tmem_ld_wait();
+        if (store) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * o_scale, __uint_as_float(rr[8 * v + 1]) * o_scale);
+            u.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * o_scale, __uint_as_float(rr[8 * v + 3]) * o_scale);
+            u.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * o_scale, __uint_as_float(rr[8 * v + 5]) * o_scale);
+            u.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * o_scale, __uint_as_float(rr[8 * v + 7]) * o_scale);
+            dst[c * 4 + v] = u;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// 3-D bf16 tensor map over [T, H, D] (D contiguous), box {64, box_h, box_t},
+// 128-byte swizzle.  Out-of-range rows read as zero.
+bool make_tmap_3d(CUtensorMap* map, const void* base, int T, int H, int D, int box_h, int box_t) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_t};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+template <int D, int TQ, int TK, int NQT>
+int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
+  using C = FwdCfg<D, TQ, TK, NQT>;
+  CUtensorMap mq, mk, mv;
+  if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, TQ) ||
+      !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, TK) ||
+      !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, TK))
+    return SINKATTN_ERR_CUDA;
+  FwdParams fp{};
+  fp.plan = p.plan;
+  fp.sink = p.sink;
+  fp.out = static_cast<__nv_bfloat16*>(out);
+  fp.lse = lse;
+  fp.sink_s = sink_s;
+  fp.status = p.status;
+  fp.Hq = p.Hq;
+  fp.Hkv = p.Hkv;
+  fp.G = p.Hq / p.Hkv;
+  fp.causal = p.causal;
+  fp.n_sink = p.n_sink;
+  fp.window = p.window;
+  fp.chunks = fp.G / (NQT * C::HPT);
+  fp.per_item = (p.ps.kh_slots == 1 ? p.Hkv : 1) * fp.chunks;
+  fp.scale_log2 = p.scale * kLog2e;
+  const long long grid = (long long)p.ps.cap_items * fp.per_item;
+  if (grid < 1 || grid > 0x7fffffffLL) return SINKATTN_ERR_INVALID_ARG;
+  auto kern = fwd_tc_kernel<C>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return SINKATTN_ERR_CUDA;
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, fp);
+  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_fwd_tc(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
+  const int G = p.Hq / p.Hkv;
+  const int tile = p.ps.tile;  // 128 (dense masks) or the block size (64/128)
+  // a query tile is 128 rows: 128 tokens x 1 head, or 64 tokens x 2 heads
+  if (tile == 128) {
+    const bool two = (G % 2 == 0);
+    if (p.D == 128) return two ? launch_cfg<128, 128, 128, 2>(p, out, lse, sink_s, stream)
+                               : launch_cfg<128, 128, 128, 1>(p, out, lse, sink_s, stream);
+    return two ? launch_cfg<64, 128, 128, 2>(p, out, lse, sink_s, stream)
+               : launch_cfg<64, 128, 128, 1>(p, out, lse, sink_s, stream);
+  }
+  // 64-token tiles need two heads per query tile
+  if (G % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;
+  const bool two = (G % 4 == 0);
+  if (p.D == 128) return two ? launch_cfg<128, 64, 64, 2>(p, out, lse, sink_s, stream)
+                             : launch_cfg<128, 64, 64, 1>(p, out, lse, sink_s, stream);
+  return two ? launch_cfg<64, 64, 64, 2>(p, out, lse, sink_s, stream)
+             : launch_cfg<64, 64, 64, 1>(p, out, lse, sink_s, stream);
+}
+
+}  // namespace sk

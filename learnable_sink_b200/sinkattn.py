@@ -1,0 +1,246 @@
+"""Thin Python binding of libsinkattn.so (ctypes; argument marshalling only).
+
+Every computation runs in the CUDA library; this module only checks tensor
+metadata, allocates outputs with torch, and passes raw device pointers and
+the current CUDA stream through the C ABI declared in ``include/sinkattn.h``.
+There is no fallback: if the library is missing or the device is not a B200
+(sm_100a), calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsinkattn.so")
+
+BF16, FP32 = 0, 2
+OK = 0
+ERR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "TIMEOUT",
+             6: "BOUNDS", 7: "PLAN"}
+
+_c = ctypes
+_vp = _c.c_void_p
+_i = _c.c_int
+_sz = _c.c_size_t
+
+
+class CMask(_c.Structure):
+    """Mirror of ``sinkattn_mask``."""
+    _fields_ = [("causal", _c.c_int32), ("n_sink", _c.c_int32), ("window", _c.c_int32),
+                ("cu_seqlens", _vp), ("n_seq", _c.c_int32), ("max_seqlen", _c.c_int32),
+                ("block_indices", _vp), ("n_qblk", _c.c_int32), ("block_q", _c.c_int32),
+                ("block_k", _c.c_int32), ("max_blocks", _c.c_int32)]
+
+
+class SinkAttnError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {ERR_NAMES.get(code, code)} ({error_string(code)})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libsinkattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m learnable_sink_b200.build` (nvcc, sm_100a)")
+        L = _c.CDLL(LIB_PATH)
+        M = _c.POINTER(CMask)
+        L.sinkattn_plan_bytes.restype = _sz
+        L.sinkattn_plan_bytes.argtypes = [_i, _i, _i, M]
+        L.sinkattn_plan.argtypes = [_i, _i, _i, M, _vp, _sz, _vp]
+        L.sinkattn_fwd.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, M, _vp, _sz,
+                                   _vp, _vp, _vp, _vp]
+        L.sinkattn_bwd_workspace_bytes.restype = _sz
+        L.sinkattn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, M]
+        L.sinkattn_bwd.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, M, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.sinkattn_decode_workspace_bytes.restype = _sz
+        L.sinkattn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
+        L.sinkattn_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
+        L.sinkattn_decode.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _i, _i,
+                                      _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
+        L.sinkattn_get_status.argtypes = [_vp]
+        L.sinkattn_clear_status.argtypes = [_vp]
+        L.sinkattn_error_string.restype = _c.c_char_p
+        L.sinkattn_error_string.argtypes = [_i]
+        L.sinkattn_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return lib().sinkattn_error_string(code).decode()
+
+
+def _check(fn, code):
+    if code != OK:
+        raise SinkAttnError(fn, code)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else _vp(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return _vp(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+@dataclass
+class Mask:
+    """Mask descriptor.  ``cu_seqlens`` / ``block_indices`` are int32 CUDA
+    tensors; ``max_seqlen`` must bound every sequence length."""
+    cu_seqlens: torch.Tensor
+    max_seqlen: int
+    causal: bool = True
+    n_sink: int = 0
+    window: int = 0
+    block_indices: Optional[torch.Tensor] = None
+    block_q: int = 64
+    block_k: int = 64
+
+    def c(self) -> CMask:
+        bi = self.block_indices
+        return CMask(int(bool(self.causal)), int(self.n_sink), int(self.window),
+                     self.cu_seqlens.data_ptr(), int(self.cu_seqlens.numel() - 1),
+                     int(self.max_seqlen), None if bi is None else bi.data_ptr(),
+                     0 if bi is None else int(bi.shape[1]), int(self.block_q), int(self.block_k),
+                     0 if bi is None else int(bi.shape[2]))
+
+    @staticmethod
+    def from_spec(spec, device="cuda") -> "Mask":
+        """From :class:`learnable_sink_b200.workloads.MaskSpec` (CPU tensors)."""
+        bi = spec.block_indices
+        return Mask(cu_seqlens=spec.cu_seqlens.to(device=device, dtype=torch.int32).contiguous(),
+                    max_seqlen=max(1, spec.max_seqlen), causal=spec.causal, n_sink=spec.n_sink,
+                    window=spec.window,
+                    block_indices=None if bi is None else bi.to(device=device, dtype=torch.int32).contiguous(),
+                    block_q=spec.block_q, block_k=spec.block_k)
+
+
+class Plan:
+    """Tile schedule built on the device from a mask (reusable by fwd/bwd)."""
+
+    def __init__(self, T_tot: int, Hq: int, Hkv: int, mask: Mask, stream=None):
+        self.T_tot, self.Hq, self.Hkv, self.mask = T_tot, Hq, Hkv, mask
+        self._cm = mask.c()
+        nbytes = lib().sinkattn_plan_bytes(T_tot, Hq, Hkv, _c.byref(self._cm))
+        if nbytes == 0:
+            raise SinkAttnError("sinkattn_plan_bytes", 1)
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=mask.cu_seqlens.device)
+        _check("sinkattn_plan", lib().sinkattn_plan(T_tot, Hq, Hkv, _c.byref(self._cm),
+                                                    _ptr(self.buf), nbytes, _stream(stream)))
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def fwd(q, k, v, sink, mask: Mask, plan: Plan, scale: Optional[float] = None, stream=None,
+        out=None, lse=None, sink_s=None):
+    """Forward.  Returns (out [T,Hq,D], lse_new [T,Hq] fp32, sink_s [T,Hq] fp32)."""
+    _contig(q, k, v, sink)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=q.device) if lse is None else lse
+    sink_s = torch.empty(T, Hq, dtype=torch.float32, device=q.device) if sink_s is None else sink_s
+    cm = mask.c()
+    _check("sinkattn_fwd", lib().sinkattn_fwd(
+        _dt(q), T, Hq, Hkv, D, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(sink), _c.byref(cm),
+        _ptr(plan.buf), plan.nbytes, _ptr(out), _ptr(lse), _ptr(sink_s), _stream(stream)))
+    return out, lse, sink_s
+
+
+def bwd_workspace_bytes(q, k, mask: Mask) -> int:
+    T, Hq, D = q.shape
+    cm = mask.c()
+    return int(lib().sinkattn_bwd_workspace_bytes(_dt(q), T, Hq, k.shape[1], D, _c.byref(cm)))
+
+
+def bwd(q, k, v, out, dout, lse, sink, mask: Mask, plan: Plan, scale: Optional[float] = None,
+        stream=None, workspace=None, dq=None, dk=None, dv=None, dsink=None):
+    """Backward.  Returns (dq, dk, dv, dsink or None)."""
+    _contig(q, k, v, out, dout, lse, sink)
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    cm = mask.c()
+    nws = lib().sinkattn_bwd_workspace_bytes(_dt(q), T, Hq, Hkv, D, _c.byref(cm))
+    if workspace is None:
+        workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if dsink is None and sink is not None:
+        dsink = torch.empty(Hq, dtype=torch.float32, device=q.device)
+    _check("sinkattn_bwd", lib().sinkattn_bwd(
+        _dt(q), T, Hq, Hkv, D, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+        _ptr(sink), _c.byref(cm), _ptr(plan.buf), plan.nbytes, _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(dsink), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv, dsink
+
+
+def decode_num_splits(B, Hq, Hkv, D, n_sink, window) -> int:
+    return int(lib().sinkattn_decode_num_splits(B, Hq, Hkv, D, n_sink, window))
+
+
+def decode_workspace_bytes(B, Hq, D, num_splits) -> int:
+    return int(lib().sinkattn_decode_workspace_bytes(B, Hq, D, num_splits))
+
+
+def decode(q, k_cache, v_cache, cache_seqlens, n_sink: int, window: int, sink,
+           scale: Optional[float] = None, num_splits: int = 0, stream=None, workspace=None,
+           out=None, lse=None, sink_s=None):
+    """Ring-buffer decode.  Returns (out [B,Hq,D], lse_new [B,Hq], sink_s [B,Hq])."""
+    _contig(q, k_cache, v_cache, cache_seqlens, sink)
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if num_splits <= 0:
+        num_splits = decode_num_splits(B, Hq, Hkv, D, n_sink, window)
+    nws = decode_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if lse is None else lse
+    sink_s = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if sink_s is None else sink_s
+    _check("sinkattn_decode", lib().sinkattn_decode(
+        _dt(q), B, Hq, Hkv, D, scale, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens),
+        int(n_sink), int(window), _ptr(sink), _ptr(out), _ptr(lse), _ptr(sink_s), int(num_splits),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse, sink_s
+
+
+def get_status(stream=None) -> int:
+    return int(lib().sinkattn_get_status(_stream(stream)))
+
+
+def clear_status(stream=None) -> None:
+    _check("sinkattn_clear_status", lib().sinkattn_clear_status(_stream(stream)))

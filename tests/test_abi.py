@@ -1,0 +1,72 @@
+"""The C-ABI library loads and exports every symbol include/sinkattn.h
+declares; host-only queries behave (no GPU needed, no kernel launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from learnable_sink_b200 import sinkattn as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sinkattn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sinkattn_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(S.LIB_PATH):
+        import learnable_sink_b200.build as B
+        B.build()
+    return S.lib()
+
+
+def test_header_declares_the_three_entry_points():
+    fns = declared_functions()
+    for name in ("sinkattn_fwd", "sinkattn_bwd", "sinkattn_decode", "sinkattn_plan"):
+        assert name in fns
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [f for f in declared_functions() if not hasattr(lib, f)]
+    assert not missing, missing
+
+
+def test_error_strings_and_version(lib):
+    assert S.error_string(0) == "ok"
+    for code in range(1, 8):
+        assert S.error_string(code) != "unknown error"
+    assert lib.sinkattn_version() >= 100
+
+
+def _mask(**kw):
+    m = S.CMask(1, 0, 0, 16, 1, 128, None, 0, 64, 64, 0)  # fake aligned device pointer
+    for k, v in kw.items():
+        setattr(m, k, v)
+    return m
+
+
+def test_plan_bytes_validates_masks(lib):
+    ok = _mask()
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(ok)) > 0
+    assert lib.sinkattn_plan_bytes(128, 3, 2, ctypes.byref(ok)) == 0         # Hq % Hkv
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(_mask(causal=0, window=8))) == 0
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(_mask(cu_seqlens=None))) == 0
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(_mask(cu_seqlens=8))) == 0  # misaligned
+    bs = _mask(block_indices=32, n_qblk=2, max_blocks=17)
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(bs)) > 0
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(_mask(block_indices=32, n_qblk=2, max_blocks=33))) == 0
+    assert lib.sinkattn_plan_bytes(128, 4, 2, ctypes.byref(_mask(block_indices=32, n_qblk=2, max_blocks=4, block_q=32, block_k=32))) == 0
+
+
+def test_workspace_queries(lib):
+    m = _mask()
+    assert lib.sinkattn_bwd_workspace_bytes(0, 128, 4, 2, 64, ctypes.byref(m)) >= 128 * 4 * 4
+    assert lib.sinkattn_bwd_workspace_bytes(0, 128, 4, 2, 96, ctypes.byref(m)) == 0
+    assert lib.sinkattn_decode_workspace_bytes(32, 32, 128, 4) >= 32 * 32 * 4 * 130 * 4
+    assert lib.sinkattn_decode_workspace_bytes(32, 32, 80, 4) == 0

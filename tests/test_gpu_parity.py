@@ -1,0 +1,271 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle
+on the same seeded inputs, plus bit-exact checks of the tile schedule."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from learnable_sink_b200 import sinkattn as S
+from learnable_sink_b200 import workloads as W
+
+from gpu_util import (TOL, check_lse, check_status, dev, max_abs, np64, read_plan, rel_err,
+                      run_bwd, run_fwd)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    S.clear_status()
+    yield
+    check_status()
+
+
+def spec(cu, causal=True, n_sink=0, window=0, bi=None, block=64):
+    return W.MaskSpec(causal=causal, n_sink=n_sink, window=window,
+                      cu_seqlens=torch.tensor(cu, dtype=torch.int32), block_indices=bi,
+                      block_q=block, block_k=block)
+
+
+# ------------------------------------------------------------ tile schedule
+
+def expected_lists(ms, T, Hq, Hkv, tile):
+    st = oracle.tile_states(T, Hq, Hkv, tile, tile, **ms.oracle_kwargs())
+    lens = np.diff(ms.cu_seqlens.numpy())
+    base = np.concatenate([[0], np.cumsum([(int(l) + tile - 1) // tile for l in lens])])
+    fwd, bwd = {}, {}
+    for g in range(Hkv):
+        for s, l in enumerate(lens):
+            nt = (int(l) + tile - 1) // tile
+            for qt in range(nt):
+                ents = [(kt << 1) | int(st[g, base[s] + qt, kt] == 1)
+                        for kt in range(nt) if st[g, base[s] + qt, kt] > 0]
+                fwd[(g, int(base[s] + qt))] = ents
+            for kt in range(nt):
+                ents = [(qt << 1) | int(st[g, base[s] + qt, kt] == 1)
+                        for qt in range(nt) if st[g, base[s] + qt, kt] > 0]
+                bwd[(g, int(base[s] + kt))] = ents
+    return fwd, bwd
+
+
+def _with_dups(bi, seed):
+    """Shuffle rows, insert duplicate ids and -1 padding in the middle."""
+    rng = np.random.default_rng(seed)
+    b = bi.numpy().copy()
+    for g in range(b.shape[0]):
+        for r in range(b.shape[1]):
+            row = b[g, r]
+            valid = row[row >= 0]
+            if len(valid) >= 2 and len(valid) < b.shape[2]:
+                valid = np.concatenate([valid, valid[:1]])  # duplicate
+            pad = np.full(b.shape[2] - len(valid), -1, dtype=np.int32)
+            b[g, r] = rng.permutation(np.concatenate([valid, pad]))
+    return torch.from_numpy(b)
+
+
+PLAN_CASES = {
+    "causal_ragged": (spec([0, 300, 600]), 600, 8, 2),
+    "band": (spec([0, 1000], n_sink=4, window=200), 1000, 4, 2),
+    "varlen_empty_seq": (spec([0, 1, 130, 130, 700, 1000]), 1000, 4, 4),
+    "non_causal": (spec([0, 200, 333], causal=False), 333, 2, 1),
+    "band_varlen": (spec([0, 77, 600, 1000], n_sink=3, window=129), 1000, 4, 1),
+}
+
+
+def _block_case(block, seed, dups):
+    cu = W.random_cu_seqlens(1500, 100, 700, seed)
+    bi = W.random_block_indices(cu, 2, block, block, 5, seed + 7)
+    if dups:
+        bi = _with_dups(bi, seed)
+    return spec(cu.tolist(), bi=bi, block=block), int(cu[-1]), 4, 2
+
+
+PLAN_CASES["block64"] = _block_case(64, 3, False)
+PLAN_CASES["block64_dups"] = _block_case(64, 4, True)
+PLAN_CASES["block128"] = _block_case(128, 5, True)
+
+
+@pytest.mark.parametrize("name", list(PLAN_CASES))
+def test_plan_matches_bruteforce_tiles(name):
+    ms, T, Hq, Hkv = PLAN_CASES[name]
+    m = S.Mask.from_spec(ms)
+    plan = S.Plan(T, Hq, Hkv, m)
+    torch.cuda.synchronize()
+    hdr, fwd, bwd, fwd_lens, bwd_lens = read_plan(plan)
+    tile = hdr["tile"]
+    assert tile == (ms.block_q if ms.block_indices is not None else 128)
+    exp_fwd, exp_bwd = expected_lists(ms, T, Hq, Hkv, tile)
+    for (g, tg), ents in exp_fwd.items():
+        key = (g, tg) if ms.block_indices is not None else (-1, tg)
+        assert key in fwd, (g, tg)
+        assert fwd[key]["entries"] == ents, (g, tg, fwd[key]["entries"], ents)
+    for (g, tg), ents in exp_bwd.items():
+        key = (g, tg) if ms.block_indices is not None else (-1, tg)
+        assert bwd[key]["entries"] == ents, (g, tg)
+    n_slots = Hkv if ms.block_indices is not None else 1
+    assert hdr["n_fwd"] == len(exp_fwd) // (Hkv // n_slots)
+    assert all(a >= b for a, b in zip(fwd_lens, fwd_lens[1:])), "not longest-first"
+    assert all(a >= b for a, b in zip(bwd_lens, bwd_lens[1:]))
+
+
+# ------------------------------------------------------------ fp32 path
+
+def _compare_fwd(inp, out, lse, ss, tol=None):
+    tol = tol or TOL[inp.q.dtype]
+    ro, rl, rs = oracle.fwd(inp.q, inp.k, inp.v, inp.sink, inp.scale, **inp.mask.oracle_kwargs())
+    eo = max_abs(np64(out), ro)
+    assert eo <= tol["o"], f"O max abs {eo:.3e}"
+    el = check_lse(np64(lse), rl, tol["lse"])
+    es = max_abs(np64(ss), rs)
+    assert es <= tol["ss"], f"sink_s max abs {es:.3e}"
+    return eo, el, es
+
+
+def _compare_bwd(inp, grads, tol=None):
+    tol = tol or TOL[inp.q.dtype]
+    dq, dk, dv, dsink = grads
+    r = oracle.bwd(inp.q, inp.k, inp.v, inp.sink, inp.dout, inp.scale, **inp.mask.oracle_kwargs())
+    for name, got, ref in (("dq", dq, r[0]), ("dk", dk, r[1]), ("dv", dv, r[2])):
+        e = rel_err(np64(got), ref)
+        assert e <= tol["grad"], f"{name} rel {e:.3e}"
+    if inp.sink is not None:
+        e = rel_err(np64(dsink), r[3])
+        assert e <= tol["grad"], f"dsink rel {e:.3e}"
+
+
+def test_tiny_fp32_forward_backward():
+    inp = W.tiny()
+    out, lse, ss, m, plan = run_fwd(inp)
+    _compare_fwd(inp, out, lse, ss)
+    _compare_bwd(inp, run_bwd(inp, out, lse, m, plan))
+
+
+FP32_CASES = {
+    "no_sink": dict(sink_std=None),
+    "zero_sink": dict(sink_values=[0.0] * 4),
+    "extreme_sinks": dict(sink_values=[-80.0, -20.0, 20.0, 80.0]),
+    "band": dict(mask=spec([0, 300], n_sink=4, window=37)),
+    "varlen_empty": dict(mask=spec([0, 5, 5, 140, 300])),
+}
+
+
+@pytest.mark.parametrize("name", list(FP32_CASES))
+def test_fp32_variants(name):
+    kw = dict(FP32_CASES[name])
+    mask = kw.pop("mask", spec([0, 300]))
+    T = int(mask.cu_seqlens[-1])
+    inp = W.make_attn(name, T_tot=T, Hq=4, Hkv=2, D=64, dtype=torch.float32, mask=mask,
+                      seed=123, **kw)
+    out, lse, ss, m, plan = run_fwd(inp)
+    _compare_fwd(inp, out, lse, ss)
+    _compare_bwd(inp, run_bwd(inp, out, lse, m, plan))
+
+
+def test_fp32_block_sparse_with_empty_rows():
+    cu = torch.tensor([0, 200, 450], dtype=torch.int32)
+    bi = W.random_block_indices(cu, 2, 64, 64, 2, 9)
+    bi[:, 1, :] = -1          # query block 1 of sequence 0 sees nothing
+    bi[1, 5, :] = -1
+    mask = W.MaskSpec(causal=True, cu_seqlens=cu, block_indices=bi, block_q=64, block_k=64)
+    for sink_std in (1.0, None):
+        inp = W.make_attn("bs_empty", T_tot=450, Hq=4, Hkv=2, D=128, dtype=torch.float32,
+                          mask=mask, seed=5, sink_std=sink_std)
+        out, lse, ss, m, plan = run_fwd(inp)
+        _compare_fwd(inp, out, lse, ss)
+        _compare_bwd(inp, run_bwd(inp, out, lse, m, plan))
+
+
+# ------------------------------------------------------------ bf16 tensor-core forward
+
+BF16_FWD = {
+    "causal_ragged_D128_G4": dict(cu=[0, 300, 555], Hq=8, Hkv=2, D=128),
+    "causal_D64_G4": dict(cu=[0, 384], Hq=8, Hkv=2, D=64),
+    "causal_D128_G1": dict(cu=[0, 200, 457], Hq=2, Hkv=2, D=128),
+    "band_D128": dict(cu=[0, 900], Hq=4, Hkv=2, D=128, n_sink=4, window=200),
+    "band_varlen_D64_G2": dict(cu=[0, 50, 700], Hq=4, Hkv=2, D=64, n_sink=4, window=130),
+    "no_sink_D128": dict(cu=[0, 260], Hq=4, Hkv=1, D=128, sink_std=None),
+    "extreme_sinks": dict(cu=[0, 260], Hq=4, Hkv=1, D=128, sink_values=[-80.0, -20.0, 20.0, 80.0]),
+    "non_causal": dict(cu=[0, 100, 300], Hq=4, Hkv=2, D=128, causal=False),
+}
+
+
+def _bf16_inputs(name, cfg, seed=7):
+    cfg = dict(cfg)
+    cu = cfg.pop("cu")
+    mask = spec(cu, causal=cfg.pop("causal", True), n_sink=cfg.pop("n_sink", 0),
+                window=cfg.pop("window", 0))
+    return W.make_attn(name, T_tot=cu[-1], dtype=torch.bfloat16, mask=mask, seed=seed, **cfg)
+
+
+@pytest.mark.parametrize("name", list(BF16_FWD))
+def test_bf16_forward(name):
+    inp = _bf16_inputs(name, BF16_FWD[name])
+    out, lse, ss, m, plan = run_fwd(inp)
+    _compare_fwd(inp, out, lse, ss)
+
+
+@pytest.mark.parametrize("G,D,block", [(8, 64, 64), (2, 64, 64), (4, 128, 64), (4, 128, 128)])
+def test_bf16_forward_block_sparse(G, D, block):
+    cu = W.random_cu_seqlens(1400, 100, 600, 11)
+    bi = W.random_block_indices(cu, 2, block, block, 4, 12, shuffle=True)
+    mask = W.MaskSpec(causal=True, cu_seqlens=cu, block_indices=bi, block_q=block, block_k=block)
+    inp = W.make_attn("bs", T_tot=int(cu[-1]), Hq=2 * G, Hkv=2, D=D, dtype=torch.bfloat16,
+                      mask=mask, seed=13)
+    out, lse, ss, m, plan = run_fwd(inp)
+    _compare_fwd(inp, out, lse, ss)
+
+
+# ------------------------------------------------------------ decode
+
+def _compare_decode(d, out, lse, ss, tol):
+    ro, rl, rs = oracle.decode(d.q, d.k_cache, d.v_cache, d.cache_seqlens, d.n_sink, d.window,
+                               d.sink, d.scale)
+    eo = max_abs(np64(out), ro)
+    assert eo <= tol["o"], f"O {eo:.3e}"
+    check_lse(np64(lse), rl, tol["lse"])
+    es = max_abs(np64(ss), rs)
+    assert es <= tol["ss"], f"sink_s {es:.3e}"
+
+
+def _run_decode(d, num_splits=0):
+    out, lse, ss = S.decode(dev(d.q), dev(d.k_cache), dev(d.v_cache), dev(d.cache_seqlens),
+                            d.n_sink, d.window, dev(d.sink), scale=d.scale, num_splits=num_splits)
+    torch.cuda.synchronize()
+    return out, lse, ss
+
+
+def test_decode_streamingllm_config():
+    d = W.decode()
+    _compare_decode(d, *_run_decode(d), TOL[torch.bfloat16])
+
+
+@pytest.mark.parametrize("splits", [1, 3, 16])
+def test_decode_partial_fill_and_splits(splits):
+    d = W.decode(B=6, n_sink=4, window=60, Hq=8, Hkv=2, D=64, seqlen_range=(0, 70))
+    d.cache_seqlens = torch.tensor([0, 1, 3, 4, 37, 64], dtype=torch.int32)
+    _compare_decode(d, *_run_decode(d, splits), TOL[torch.bfloat16])
+
+
+def test_decode_fp32_no_sink():
+    d = W.decode(B=4, n_sink=2, window=40, Hq=4, Hkv=4, D=128, dtype=torch.float32,
+                 seqlen_range=(1, 100), sink_std=None)
+    _compare_decode(d, *_run_decode(d), TOL[torch.float32])
+
+
+def test_decode_rotation_invariance():
+    d = W.decode(B=1, n_sink=4, window=64, Hq=8, Hkv=2, D=128, seqlen_range=(500, 500))
+    o0, l0, s0 = _run_decode(d)
+    r = 17
+    kc, vc = d.k_cache.clone(), d.v_cache.clone()
+    kc[:, 4:] = torch.roll(d.k_cache[:, 4:], r, dims=1)
+    vc[:, 4:] = torch.roll(d.v_cache[:, 4:], r, dims=1)
+    d.k_cache, d.v_cache = kc, vc
+    d.cache_seqlens = d.cache_seqlens + r
+    o1, l1, s1 = _run_decode(d)
+    # same set of tokens: equal up to summation order
+    assert max_abs(np64(o0), np64(o1)) <= 1e-2
+    assert max_abs(np64(l0), np64(l1)) <= 1e-5
