@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the learnable-sink attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass over every hot-path stage on synthetic inputs:
+  * training prefill (B=4 x T=4096 packed, Hq=32, Hkv=8, D=128, bf16, causal):
+    tile schedule from the mask, forward (O, LSE_new, sink_s), backward
+    (Delta/dsink preprocess, dK/dV/dQ kernel, dQ conversion) -- and, with N > 1
+    ranks, the all-reduce of dsink (the sink is a parameter shared by every
+    rank's queries);
+  * StreamingLLM decode (32 sequences x 1 query, ring cache of 4 sink + 1020
+    window slots, Hq=32, Hkv=8, D=128, bf16), after an L2 flush.
+The headline value is the prefill fwd+bwd algorithmic throughput (visible
+(query, key, head) triples x (4 + 10) x D flop) over all ranks; decode GB/s is
+reported beside it.  Each rank processes its own batch (weak scaling).  Times
+are CUDA events on the launching stream, max over ranks.
+
+``--impl reference`` times the float64 CPU oracle (the correctness reference of
+this repository) on the host cores on a bounded slice of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from learnable_sink_b200 import workloads as W  # noqa: E402
+
+METRIC = "sink-attn fwd+bwd TFLOP/s & decode KV GB/s on 1 B200, % of roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def file_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_traffic(kernel):
+    """ncu-measured DRAM bytes per launch (profiles/traffic.json), valid only
+    while the kernel's source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f).get(kernel)
+    if not t:
+        return None
+    src = os.path.join(ROOT, t["source"])
+    if not os.path.exists(src) or file_hash(src) != t["source_sha256_16"]:
+        return None
+    return float(t["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.lines = index, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(inp, n_tok, n_groups):
+    """Time the float64 oracle on sequence 0's first n_tok tokens and the
+    first n_groups KV heads (with their query heads).  Returns (seconds,
+    flop, description)."""
+    import numpy as np
+    import oracle
+    T, Hq, Hkv, D = inp.shape
+    G = Hq // Hkv
+    sl = slice(0, n_tok)
+    hq = slice(0, G * n_groups)
+    hk = slice(0, n_groups)
+    q, k, v = inp.q[sl, hq], inp.k[sl, hk], inp.v[sl, hk]
+    do, a = inp.dout[sl, hq], inp.sink[hq]
+    cu = np.array([0, n_tok], dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.fwd(q, k, v, a, inp.scale, causal=True, cu_seqlens=cu)
+    oracle.bwd(q, k, v, a, do, inp.scale, causal=True, cu_seqlens=cu)
+    dt = time.perf_counter() - t0
+    pairs = n_tok * (n_tok + 1) // 2 * G * n_groups
+    desc = (f"oracle fwd+bwd on sequence 0 tokens [0,{n_tok}) x {n_groups} KV head(s) "
+            f"({G * n_groups} query heads) of the prefill workload, float64, "
+            f"{oracle.num_threads()} OpenMP threads")
+    return dt, pairs * 14 * D, desc, oracle.num_threads()
+
+
+def run_reference(args, world, rank):
+    base = {"metric": METRIC, "unit": "TFLOP/s", "higher_is_better": True, "impl": "reference"}
+    if rank != 0:
+        return
+    inp = W.prefill()
+    n_tok, n_groups = 2048, 1
+    for _ in range(args.warmup):
+        cpu_oracle_sample(inp, n_tok, n_groups)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl, desc, cores = cpu_oracle_sample(inp, n_tok, n_groups)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = dict(base, value=value, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=tot_t / args.steps * 1e3, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic",
+                config={"workload": "training prefill B4 T4096 Hq32 Hkv8 D128 causal fwd+bwd",
+                        "sample": desc},
+                cpu_baseline={"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                              "sample": desc},
+                e2e={"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                     "d2h_bytes_per_step": 0})
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    from learnable_sink_b200 import sinkattn as S
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---- prefill inputs (per rank: its own batch)
+    inp = W.prefill(seed_offset=1000 * rank)
+    T, Hq, Hkv, D = inp.shape
+    pairs = W.visible_pairs(inp.mask, Hq, Hkv)
+    flop_fwd, flop_bwd = 4 * D * pairs, 10 * D * pairs
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    sink, dout = inp.sink.to(dev), inp.dout.to(dev)
+    mask = S.Mask.from_spec(inp.mask, dev)
+    plan = S.Plan(T, Hq, Hkv, mask)
+    out = torch.empty_like(q)
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    sink_s = torch.empty_like(lse)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dsink = torch.empty(Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(S.bwd_workspace_bytes(q, k, mask), dtype=torch.uint8, device=dev)
+
+    # ---- decode inputs
+    dec = W.decode(seed_offset=1000 * rank)
+    dq_in = dec.q.to(dev)
+    kc, vc = dec.k_cache.to(dev), dec.v_cache.to(dev)
+    cs, dsk = dec.cache_seqlens.to(dev), dec.sink.to(dev)
+    B, dHq, dD = dec.q.shape
+    dHkv = dec.k_cache.shape[2]
+    n_splits = S.decode_num_splits(B, dHq, dHkv, dD, dec.n_sink, dec.window)
+    dws = torch.empty(S.decode_workspace_bytes(B, dHq, dD, n_splits), dtype=torch.uint8, device=dev)
+    dout_dec = torch.empty_like(dq_in)
+    dlse = torch.empty(B, dHq, dtype=torch.float32, device=dev)
+    dss = torch.empty_like(dlse)
+    valid = torch.clamp(dec.cache_seqlens, max=dec.n_sink + dec.window).sum().item()
+    dec_bytes = 2 * valid * dHkv * dD * 2 + 2 * B * dHq * dD * 2 + 2 * B * dHq * 4 + B * 4
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def prefill_step():
+        plan.rebuild()
+        S.fwd(q, k, v, sink, mask, plan, scale=inp.scale, out=out, lse=lse, sink_s=sink_s)
+        S.bwd(q, k, v, out, dout, lse, sink, mask, plan, scale=inp.scale, workspace=ws,
+              dq=dq, dk=dk, dv=dv, dsink=dsink)
+        if world > 1:
+            torch.distributed.all_reduce(dsink)
+
+    def decode_step():
+        S.decode(dq_in, kc, vc, cs, dec.n_sink, dec.window, dsk, scale=dec.scale,
+                 num_splits=n_splits, workspace=dws, out=dout_dec, lse=dlse, sink_s=dss)
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+    # warm-up (also creates every event handle)
+    for _ in range(args.warmup):
+        prefill_step()
+        flush.zero_()
+        decode_step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = {n: [ev() for _ in range(K)] for n in
+           ("p0", "p1", "d0", "d1", "kf0", "kf1", "kb0", "kb1", "kd0", "kd1")}
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        r0 = ev()
+        for i in range(K):
+            S.set_kernel_events(S.KERNEL_FWD, evs["kf0"][i], evs["kf1"][i])
+            S.set_kernel_events(S.KERNEL_BWD, evs["kb0"][i], evs["kb1"][i])
+            S.set_kernel_events(S.KERNEL_DECODE, evs["kd0"][i], evs["kd1"][i])
+            evs["p0"][i].record()
+            prefill_step()
+            evs["p1"][i].record()
+            flush.zero_()  # decode's working set is about L2-sized: start it cold
+            evs["d0"][i].record()
+            decode_step()
+            evs["d1"][i].record()
+        r1 = ev()
+        torch.cuda.synchronize()
+    for w in (S.KERNEL_FWD, S.KERNEL_BWD, S.KERNEL_DECODE):
+        S.set_kernel_events(w, None, None)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    code = S.get_status()
+    if code != 0:
+        raise RuntimeError(f"device status {S.ERR_NAMES.get(code, code)}")
+
+    def total(a, b):
+        return sum(x.elapsed_time(y) for x, y in zip(evs[a], evs[b]))
+
+    region_ms = max_over_ranks(r0.elapsed_time(r1), world)
+    prefill_ms = max_over_ranks(total("p0", "p1"), world)
+    decode_ms = max_over_ranks(total("d0", "d1"), world)
+    kf_ms = total("kf0", "kf1") / K
+    kb_ms = total("kb0", "kb1") / K
+    kd_ms = total("kd0", "kd1") / K
+    value = world * K * (flop_fwd + flop_bwd) / (prefill_ms * 1e-3) / 1e12
+    dec_gbs = world * K * dec_bytes / (decode_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    pin = {n: t.cpu().pin_memory() for n, t in (("q", inp.q), ("k", inp.k), ("v", inp.v),
+                                                 ("dout", inp.dout), ("sink", inp.sink))}
+    h_dsink = torch.empty(Hq, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = h_dsink.numel() * 4
+
+    def e2e_step():
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        dout.copy_(pin["dout"], non_blocking=True)
+        sink.copy_(pin["sink"], non_blocking=True)
+        prefill_step()
+        h_dsink.copy_(dsink, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = ev()
+    K2 = max(3, K // 2)
+    for _ in range(K2):
+        e2e_step()
+    e1 = ev()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * K2 * (flop_fwd + flop_bwd) / (e2e_ms * 1e-3) / 1e12
+
+    if rank != 0:
+        return
+    clocks = clk.summary()
+    peak_tf = peaks["bf16_tflops_sustained"]
+    bwd_ach = flop_bwd / (kb_ms * 1e-3) / 1e12
+    fwd_ach = flop_fwd / (kf_ms * 1e-3) / 1e12
+    dec_kernel_bytes = 2 * valid * dHkv * dD * 2
+    dec_ach = dec_kernel_bytes / (kd_ms * 1e-3) / 1e9
+    traffic = load_traffic("bwd_tc_kernel")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": region_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": "training prefill B4 T4096 Hq32 Hkv8 D128 bf16 causal, plan+fwd+bwd "
+                        "(+ StreamingLLM decode B32 cache 4+1020 Hq32 Hkv8 D128 per step)",
+            "global_batch": 4 * world, "seq_len": 4096, "parallelism": f"dp{world}",
+            "visible_pairs_per_rank": pairs,
+            "l2": "prefill inputs larger than L2; L2 flushed (256 MB write) before each decode",
+        },
+        "decode": {"value": dec_gbs, "unit": "GB/s", "ms_per_call": decode_ms / K,
+                   "bytes_per_call": dec_bytes, "num_splits": n_splits},
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": K2,
+                "what": "pinned-host q,k,v,dO,sink -> device, plan+fwd+bwd, dsink -> host"},
+        "gpu_launches": K * (9 + 1 + 4 + 2),
+        "roofline": {"kernel": "bwd_tc_kernel (dK/dV/dQ)", "bound": "tensor",
+                     "achieved": bwd_ach, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": bwd_ach / peak_tf, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "algorithmic": "10*D flop per visible pair x visible pairs per launch"},
+        "kernels": {
+            "fwd_tc_kernel": {"ms": kf_ms, "achieved_tflops": fwd_ach,
+                              "frac_of_sustained": fwd_ach / peak_tf},
+            "bwd_tc_kernel": {"ms": kb_ms, "achieved_tflops": bwd_ach,
+                              "frac_of_sustained": bwd_ach / peak_tf},
+            "decode_split_kernel": {"ms": kd_ms, "achieved_gbs": dec_ach,
+                                    "frac_of_hbm": dec_ach / peaks["hbm_gbs"]},
+        },
+    }
+    if world == 1:
+        dt, fl, desc, cores = cpu_oracle_sample(inp, 4096, 2)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "sample": desc, "seconds": dt}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    world, rank, local = init_dist() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if args.impl == "ours" and world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -211,6 +211,22 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
                     float *sink_s, int num_splits, void *workspace,
                     size_t workspace_bytes, sinkattn_stream_t stream);
 
+/* ---- profiling hook ---------------------------------------------------------
+ * Records CUDA events around the main kernel of later calls, on the stream
+ * that kernel is launched on, so a caller can time that kernel alone (the
+ * other launches of the call stay outside the events).
+ *   which   SINKATTN_KERNEL_FWD (the attention forward kernel),
+ *           SINKATTN_KERNEL_BWD (the dK/dV/dQ kernel of sinkattn_bwd),
+ *           SINKATTN_KERNEL_DECODE (the split-KV streaming kernel).
+ *   start, stop  cudaEvent_t handles created by the caller, or both NULL to
+ *           stop recording.  They are recorded by every later call of that
+ *           kind on the calling host thread's current device until changed.
+ * Returns SINKATTN_ERR_INVALID_ARG for an unknown `which`. */
+#define SINKATTN_KERNEL_FWD 0
+#define SINKATTN_KERNEL_BWD 1
+#define SINKATTN_KERNEL_DECODE 2
+int sinkattn_set_kernel_events(int which, void *start, void *stop);
+
 /* ---- status ---------------------------------------------------------------
  * sinkattn_get_status synchronises `stream`, then returns the first error code
  * any kernel of this library recorded on the current device since the last

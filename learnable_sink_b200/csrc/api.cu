@@ -47,6 +47,8 @@ bool device_is_sm100() {
   return g_is_sm100[dev] == 1;
 }
 
+thread_local KernelEvents g_events[3];
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool mask_ok(int T_tot, int Hq, int Hkv, const sinkattn_mask* m) {
@@ -93,12 +95,13 @@ constexpr size_t kAlign = 256;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct BwdLayout {
-  size_t delta, part, dq_accum, total;
+  size_t delta, lse2, part, dq_accum, total;
 };
 BwdLayout bwd_layout(int dt, int T_tot, int Hq, int D) {
   BwdLayout L{};
   size_t off = 0;
   L.delta = off; off += round_up(sizeof(float) * (size_t)T_tot * Hq);
+  L.lse2 = off; off += round_up(sizeof(float) * (size_t)T_tot * Hq);
   L.part = off; off += round_up(sizeof(float) * (size_t)preprocess_blocks(T_tot) * Hq);
   L.dq_accum = off;
   if (dt == SINKATTN_BF16) off += round_up(bwd_tc_workspace_bytes(T_tot, Hq, D));
@@ -107,6 +110,11 @@ BwdLayout bwd_layout(int dt, int T_tot, int Hq, int D) {
 }
 
 }  // namespace
+
+KernelEvents kernel_events(int which) {
+  return (which >= 0 && which < 3) ? g_events[which] : KernelEvents{};
+}
+
 }  // namespace sk
 
 using namespace sk;
@@ -227,6 +235,7 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
   b.dv = dv;
   b.dsink = learnable_sink ? dsink : nullptr;
   b.delta = reinterpret_cast<float*>(ws + L.delta);
+  b.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   b.dsink_part = reinterpret_cast<float*>(ws + L.part);
   b.dq_accum = reinterpret_cast<float*>(ws + L.dq_accum);
   b.n_part_blocks = preprocess_blocks(T_tot);
@@ -300,6 +309,14 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
   p.part = static_cast<float*>(workspace);
   p.status = status_word();
   return launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sinkattn_set_kernel_events(int which, void* start, void* stop) {
+  if (which < 0 || which > 2 || ((start == nullptr) != (stop == nullptr)))
+    return SINKATTN_ERR_INVALID_ARG;
+  g_events[which].start = static_cast<cudaEvent_t>(start);
+  g_events[which].stop = static_cast<cudaEvent_t>(stop);
+  return SINKATTN_OK;
 }
 
 int sinkattn_get_status(sinkattn_stream_t stream) {

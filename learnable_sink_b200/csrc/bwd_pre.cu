@@ -3,6 +3,10 @@
 //   Delta_ih = sum_d dO_ihd * O_ihd                 (fp32, from the sink-scaled O)
 //   p_sink   = exp(a_h - L_new,ih)                  (section 10: avoids 1 - sink_s)
 //   dsink_h  = -sum_i Delta_ih * p_sink,ih          (every query counted once)
+// Delta and LSE_new * log2(e) are written head-major ([Hq][T_tot]) so the
+// backward kernels read a query tile's values with coalesced loads; a row
+// with LSE = -inf (it sees no key and has no sink) gets +inf there, which
+// makes every recomputed probability of the row exactly 0.
 // Each CTA owns a fixed range of tokens and writes one partial per head; a
 // second kernel sums the partials in a fixed order, so dsink is bitwise
 // deterministic.  HBM-bound: it streams O and dO once.
@@ -57,7 +61,7 @@ __device__ __forceinline__ float row_dot(const T* a, const T* b, int lane) {
 template <typename T, int D>
 __global__ void __launch_bounds__(kPreThreads) preprocess_kernel(
     const T* out, const T* dout, const float* lse, const float* sink, float* delta,
-    float* part, int T_tot, int Hq) {
+    float* lse2, float* part, int T_tot, int Hq) {
   __shared__ float wpart[kPreThreads / 32][kMaxHeads];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NW = kPreThreads / 32;
@@ -71,9 +75,12 @@ __global__ void __launch_bounds__(kPreThreads) preprocess_kernel(
   for (long long r = r0 + warp; r < r1; r += NW) {
     const float d = row_dot<T, D>(out + r * D, dout + r * D, lane);
     if (lane == 0) {
-      delta[r] = d;
+      const int h = (int)(r % Hq);
+      const long long t = r / Hq;
+      const float l = lse[r];
+      delta[(long long)h * T_tot + t] = d;
+      lse2[(long long)h * T_tot + t] = (l == -INFINITY) ? INFINITY : l * kLog2e;
       if (sink) {
-        const int h = (int)(r % Hq);
         const float ps = __expf(sink[h] - lse[r]);
         wpart[warp][h] -= d * ps;
       }
@@ -109,16 +116,16 @@ int launch_bwd_preprocess(const AttnProblem& p, const BwdBuffers& b, cudaStream_
     const auto* o = static_cast<const __nv_bfloat16*>(b.out);
     const auto* d = static_cast<const __nv_bfloat16*>(b.dout);
     if (p.D == 64)
-      preprocess_kernel<__nv_bfloat16, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<__nv_bfloat16, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
     else
-      preprocess_kernel<__nv_bfloat16, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<__nv_bfloat16, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   } else {
     const auto* o = static_cast<const float*>(b.out);
     const auto* d = static_cast<const float*>(b.dout);
     if (p.D == 64)
-      preprocess_kernel<float, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<float, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
     else
-      preprocess_kernel<float, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<float, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   }
   if (p.sink && b.dsink)
     dsink_reduce_kernel<<<(p.Hq + 127) / 128, 128, 0, stream>>>(b.dsink_part, nb, p.Hq, b.dsink);

@@ -1,14 +1,496 @@
-// Backward on the tensor cores (placeholder until the tcgen05 kernels land).
+// Backward pass on the tensor cores (tcgen05) for bf16 inputs.
+//
+// Page "Attention Sink, Learnable Sink and dsink", section 8: with the
+// probabilities rebuilt from the sink-inclusive LSE, P = exp(x - L_new), and
+// Delta taken from the sink-scaled output, the ordinary softmax gradients
+//   dS = P * (dP - Delta),  dP = dO V^T
+//   dV = P^T dO,  dK = alpha dS^T Q,  dQ = alpha dS K
+// already carry the sink's effect; dsink comes from the preprocess
+// (section 7) and is not touched here.  Section 10 describes a backward split
+// by KV block over reverse lists; this kernel is that split.
+//
+// One CTA = one 128-key tile of one KV head (the plan's reverse list gives
+// the query tiles that see it); it loops over (query tile, query head) pairs.
+// Tensor memory (512 columns):
+//   S^T  [keys x 128 query rows] fp32, overwritten in place by P^T (bf16,
+//        packed two per column at the front of each warpgroup's slice)
+//   dP^T [keys x 128] fp32, overwritten by dS^T (bf16, same packing); then reused for the
+//        dQ tile [128 query rows x D] once dK has consumed dS^T
+//   dK, dV [keys x D] fp32 accumulators for the whole CTA
+// MMAs per (query tile, head), issued by one thread in this order:
+//   S^T = K Q^T (SS) | dP^T = V dO^T (SS) | dV += P^T dO (TS) |
+//   dK += dS^T Q (TS) | dQ = dS K (SS; dS^T also staged in shared memory)
+// Warps 0-7 compute (warpgroup c owns query columns [64c, 64c + 64), thread =
+// key row), warp 8 is the TMA producer, warp 9 issues MMAs.  The compute
+// warps also move each dQ tile out of tensor memory into an fp32 buffer with
+// vector reductions (a query row gets one contribution per visible key
+// tile); a small kernel converts it to bf16.
 #include "internal.h"
 
 namespace sk {
+
+namespace {
+
+template <int D_>
+struct BwdCfg {
+  static constexpr int D = D_, KT = 128, TQ = 128, HPT = 1;
+  static constexpr int DH = D / 64;
+  static constexpr int Q_BYTES = 128 * D * 2;   // Q or dO tile (128 rows)
+  static constexpr int KV_BYTES = KT * D * 2;   // K or V tile
+  static constexpr int DS_BYTES = KT * 128 * 2; // dS^T tile
+  static constexpr int SMEM_LIMIT = 227 * 1024;
+  static constexpr int FIXED = 2 * KV_BYTES + DS_BYTES + 1024 /*lse, delta*/ + 512 /*bars*/ + 1024;
+  static constexpr int NS_RAW = (SMEM_LIMIT - FIXED) / (2 * Q_BYTES);
+  static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
+  static_assert(NS >= 2, "shared memory");
+  static constexpr int THREADS = 10 * 32;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  static constexpr int S_COL = 0, DP_COL = 128, DK_COL = 256, DV_COL = 256 + D;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_DS = OFF_V + KV_BYTES;
+  static constexpr int OFF_Q = OFF_DS + DS_BYTES;
+  static constexpr int OFF_DO = OFF_Q + NS * Q_BYTES;
+  static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[128]
+  static constexpr int OFF_DL = OFF_LSE + 512;            // float[128]
+  static constexpr int OFF_BAR = OFF_DL + 512;
+  static constexpr int N_BARS = 1 + 2 * NS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+};
+
+struct BwdParams {
+  const int* plan;
+  const float* lse2;   // [Hq, T] head-major, log2 domain
+  const float* delta;  // [Hq, T]
+  float* dq_accum;     // [T, Hq, D] fp32
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int* status;
+  int T_tot, Hq, Hkv, G, causal, n_sink, window, per_item;
+  float scale_log2, alpha;
+};
+
+__device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitBudgetCycles) return false;
+  return true;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+// Packed bf16 P^T / dS^T columns: warpgroup c writes its 64 query columns
+// as 32 packed words at the front of its own fp32 slice [64c, 64c + 64), so
+// it never overwrites fp32 values the other warpgroup has yet to read.  K step
+// kk (16 query columns) of the TS-MMA A operand therefore starts at:
+__device__ __forceinline__ constexpr uint32_t a_col(int kk) { return (kk / 4) * 64 + (kk % 4) * 8; }
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                  const __grid_constant__ CUtensorMap tmap_do,
+                  const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const BwdParams p) {
+  constexpr int D = C::D, KT = C::KT, TQ = C::TQ, HPT = C::HPT, NS = C::NS, DH = C::DH;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_kv = bars;
+  uint64_t* bar_qf = bars + 1;
+  uint64_t* bar_qe = bar_qf + NS;
+  uint64_t* bar_s = bar_qe + NS;
+  uint64_t* bar_dp = bar_s + 1;
+  uint64_t* bar_p = bar_dp + 1;
+  uint64_t* bar_ds = bar_p + 1;
+  uint64_t* bar_dq = bar_ds + 1;
+  uint64_t* bar_dqf = bar_dq + 1;
+  uint64_t* bar_fin = bar_dqf + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
+  float* s_dl = reinterpret_cast<float*>(smem + C::OFF_DL);
+
+  const PlanHdr* hdr = reinterpret_cast<const PlanHdr*>(p.plan);
+  const int rank = blockIdx.x / p.per_item;
+  if (rank >= hdr->n_bwd_items) return;
+  const int rem = blockIdx.x % p.per_item;
+  const int idx = p.plan[hdr->off_bwd_order + rank];
+  const TileItem it = reinterpret_cast<const TileItem*>(p.plan + hdr->off_bwd_items)[idx];
+  const int kvh = it.kvh >= 0 ? it.kvh : rem;
+  const int* ent = p.plan + hdr->off_bwd_entries + it.entry_off;
+  const int GH = p.G / HPT;             // query-head groups per key tile
+  const int n_it = it.entry_len * GH;   // (query tile, head group) iterations
+  const int k0 = it.tile_start;         // sequence-local first key
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_qf + s, 1);
+      mbar_init(bar_qe + s, 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
+    mbar_init(bar_dq, 1);
+    mbar_init(bar_dqf, 256);
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_do);
+    prefetch_tensormap(&tmap_k);
+    prefetch_tensormap(&tmap_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_it > 0) {
+      const int krow = it.seq_start + k0;
+      mbar_expect_tx(bar_kv, 2 * C::KV_BYTES);
+      for (int h = 0; h < DH; ++h) {
+        tma_load_3d(smem + C::OFF_K + h * (C::KV_BYTES / DH), &tmap_k, bar_kv, h * 64, kvh, krow);
+        tma_load_3d(smem + C::OFF_V + h * (C::KV_BYTES / DH), &tmap_v, bar_kv, h * 64, kvh, krow);
+      }
+      int last[NS];
+      for (int s = 0; s < NS; ++s) last[s] = -1;
+      bool ok = true;
+      for (int i = 0; i < n_it && ok; ++i) {
+        const int s = i % NS;
+        const int e = __ldg(ent + i / GH);
+        const int q_tok = it.seq_start + (e >> 1) * TQ;
+        const int h0 = kvh * p.G + (i % GH) * HPT;
+        ok = mbar_wait(bar_qe + s, ((i / NS) & 1) ^ 1, abort_flag, p.status);
+        if (!ok) break;
+        mbar_expect_tx(bar_qf + s, 2 * C::Q_BYTES);
+        for (int h = 0; h < DH; ++h) {
+          tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_q,
+                      bar_qf + s, h * 64, h0, q_tok);
+          tma_load_3d(smem + C::OFF_DO + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_do,
+                      bar_qf + s, h * 64, h0, q_tok);
+        }
+        last[s] = i;
+      }
+      if (!ok) {
+        wait_noabort(bar_kv, 0);
+        for (int s = 0; s < NS; ++s)
+          if (last[s] >= 0) wait_noabort(bar_qf + s, (last[s] / NS) & 1);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_it > 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(KT, 128, 0, 0);   // S^T, dP^T
+      constexpr uint32_t id_kv = idesc_bf16_f32(KT, D, 0, 1);    // dV, dK (B MN-major)
+      constexpr uint32_t id_q = idesc_bf16_f32(128, D, 1, 1);    // dQ (A, B MN-major)
+      const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V),
+                     sDS = smem_u32(smem + C::OFF_DS), sQ = smem_u32(smem + C::OFF_Q),
+                     sDO = smem_u32(smem + C::OFF_DO);
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status);
+      for (int i = 0; i < n_it && ok; ++i) {
+        const int s = i % NS;
+        ok = mbar_wait(bar_qf + s, (i / NS) & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t q_s = sQ + s * C::Q_BYTES, do_s = sDO + s * C::Q_BYTES;
+        // S^T = K Q^T (both K-major)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          mma_ss(tmem + C::S_COL,
+                 sdesc_sw128(sK + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
+                 sdesc_sw128(q_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_s);
+        // dP^T = V dO^T, into the columns the previous dQ tile occupied
+        if (i > 0) {
+          ok = mbar_wait(bar_dqf, (i - 1) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          mma_ss(tmem + C::DP_COL,
+                 sdesc_sw128(sV + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
+                 sdesc_sw128(do_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_dp);
+        // dV += P^T dO  (P^T bf16 in tensor memory over S^T; dO MN-major)
+        ok = mbar_wait(bar_p, i & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + C::DV_COL, tmem + C::S_COL + a_col(kk),
+                 sdesc_sw128(do_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q  (dS^T bf16 in tensor memory over dP^T)
+        ok = mbar_wait(bar_ds, i & 1, abort_flag, p.status);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + C::DK_COL, tmem + C::DP_COL + a_col(kk),
+                 sdesc_sw128(q_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        // dQ = dS K  (A = dS from the staged dS^T tile, both MN-major)
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk)
+          mma_ss(tmem + C::DP_COL, sdesc_sw128(sDS + kk * 2048, KT * 128, 1024),
+                 sdesc_sw128(sK + kk * 2048, C::KV_BYTES / DH, 1024), id_q, kk > 0 ? 1u : 0u);
+        mma_commit(bar_dq);
+        mma_commit(bar_qe + s);
+      }
+      mma_commit(bar_fin);
+      wait_noabort(bar_fin, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ compute
+    const int cw = warp / 4;          // query-column half
+    const int wq = warp % 4;          // TMEM lane quadrant
+    const int tw = wq * 32 + lane;    // 0..127 within the warpgroup
+    const int r = tw;                 // key row (= TMEM lane)
+    const int kj = k0 + r;            // sequence-local key
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const float* lse_s = s_lse + 64 * cw;
+    const float* dl_s = s_dl + 64 * cw;
+    bool ok = true;
+    for (int i = 0; i < n_it; ++i) {
+      const int e = __ldg(ent + i / GH);
+      const int q0 = (e >> 1) * TQ;
+      const bool partial = (e & 1) != 0;
+      const int h0 = kvh * p.G + (i % GH) * HPT;
+      const int q_len = min(TQ, it.seq_len - q0);
+      // this warpgroup's 64 query columns: log2-domain LSE and Delta
+      named_bar_sync(1 + cw, 128);
+      if (tw < 64) {
+        const int col = 64 * cw + tw;
+        const int tok = col / HPT, hh = col % HPT;
+        const bool valid = tok < q_len;
+        const long long gi = (long long)(h0 + hh) * p.T_tot + it.seq_start + q0 + tok;
+        s_lse[col] = valid ? __ldg(p.lse2 + gi) : INFINITY;
+        s_dl[col] = valid ? __ldg(p.delta + gi) : 0.f;
+      }
+      named_bar_sync(1 + cw, 128);
+      // P^T = exp2(S^T * alpha * log2e - LSE2)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s, i & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      float P[64];
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(tmem + lane_off + C::S_COL + 64 * cw, a);
+        tmem_ld32(tmem + lane_off + C::S_COL + 64 * cw + 32, b);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          P[c] = fast_exp2(__uint_as_float(a[c]) * p.scale_log2 - lse_s[c]);
+          P[c + 32] = fast_exp2(__uint_as_float(b[c]) * p.scale_log2 - lse_s[c + 32]);
+        }
+      }
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int tok = (64 * cw + c) / HPT;
+          if (!visible_elem(q0 + tok, kj, it.seq_len, p.causal, p.n_sink, p.window)) P[c] = 0.f;
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(P[2 * c], P[2 * c + 1]);
+        tmem_st32(tmem + lane_off + C::S_COL + 64 * cw, pk);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(bar_p);
+      // dS^T = P^T * (dP^T - Delta)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, i & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t ds[32];
+      {
+        uint32_t a[32], b[32];
+        tmem_ld32(tmem + lane_off + C::DP_COL + 64 * cw, a);
+        tmem_ld32(tmem + lane_off + C::DP_COL + 64 * cw + 32, b);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          ds[c] = pack_bf16x2(P[2 * c] * (__uint_as_float(a[2 * c]) - dl_s[2 * c]),
+                              P[2 * c + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[2 * c + 1]));
+          ds[c + 16] = pack_bf16x2(P[32 + 2 * c] * (__uint_as_float(b[2 * c]) - dl_s[32 + 2 * c]),
+                                   P[33 + 2 * c] * (__uint_as_float(b[2 * c + 1]) - dl_s[33 + 2 * c]));
+        }
+      }
+      tmem_st32(tmem + lane_off + C::DP_COL + 64 * cw, ds);
+      // the previous dQ MMA must be done reading the staged dS tile
+      if (i > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (i - 1) & 1, abort_flag, p.status));
+        if (!ok) break;
+      }
+      {
+        // row r of the [keys][64 queries] half-tile, 128-byte swizzle
+        uint8_t* row = smem + C::OFF_DS + cw * (KT * 128) + r * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) * 16)) =
+              make_uint4(ds[4 * j], ds[4 * j + 1], ds[4 * j + 2], ds[4 * j + 3]);
+      }
+      fence_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+      // dQ tile: lanes are query rows; this warpgroup takes D/2 columns
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dq[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + C::DP_COL + (D / 2) * cw + 32 * c, a);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) dq[32 * c + x] = a[x];
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dqf);
+      {
+        const int qrow = tw;  // query row of the tile held by this lane
+        const int tok = qrow / HPT, hh = qrow % HPT;
+        if (tok < q_len) {
+          float* dst = p.dq_accum +
+                       ((long long)(it.seq_start + q0 + tok) * p.Hq + h0 + hh) * D + (D / 2) * cw;
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c)
+            red_add_v4(dst + 4 * c, __uint_as_float(dq[4 * c]), __uint_as_float(dq[4 * c + 1]),
+                       __uint_as_float(dq[4 * c + 2]), __uint_as_float(dq[4 * c + 3]));
+        }
+      }
+    }
+    // dK (warpgroup 0) and dV (warpgroup 1) rows of this key tile
+    const bool have = n_it > 0 && ok &&
+                      __all_sync(0xffffffffu, mbar_wait(bar_fin, 0, abort_flag, p.status));
+    const bool store = (n_it == 0 || have) && kj < it.seq_len;
+    __nv_bfloat16* dst_base = (cw == 0 ? p.dk : p.dv);
+    uint4* dst = reinterpret_cast<uint4*>(dst_base + ((long long)(it.seq_start + kj) * p.Hkv + kvh) * D);
+    const float f = cw == 0 ? p.alpha : 1.f;
+    if (have) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + (cw == 0 ? C::DK_COL : C::DV_COL) + 32 * c, a);
+        tmem_ld_wait();
+        if (store) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[4 * c + v] = make_uint4(
+                pack_bf16x2(__uint_as_float(a[8 * v]) * f, __uint_as_float(a[8 * v + 1]) * f),
+                pack_bf16x2(__uint_as_float(a[8 * v + 2]) * f, __uint_as_float(a[8 * v + 3]) * f),
+                pack_bf16x2(__uint_as_float(a[8 * v + 4]) * f, __uint_as_float(a[8 * v + 5]) * f),
+                pack_bf16x2(__uint_as_float(a[8 * v + 6]) * f, __uint_as_float(a[8 * v + 7]) * f));
+        }
+      }
+    } else if (store) {
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// dQ = alpha * accumulated fp32, rounded to bf16.
+__global__ void dq_convert_kernel(const float4* acc, uint2* dq, long long n4, float alpha) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = acc[i];
+  dq[i] = make_uint2(pack_bf16x2(v.x * alpha, v.y * alpha), pack_bf16x2(v.z * alpha, v.w * alpha));
+}
+
+template <int D>
+int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  CUtensorMap mq, mdo, mk, mv;
+  if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
+      !make_tmap_3d(&mdo, b.dout, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
+      !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::KT) ||
+      !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::KT))
+    return SINKATTN_ERR_CUDA;
+  BwdParams bp{};
+  bp.plan = p.plan;
+  bp.lse2 = b.lse2;
+  bp.delta = b.delta;
+  bp.dq_accum = b.dq_accum;
+  bp.dk = static_cast<__nv_bfloat16*>(b.dk);
+  bp.dv = static_cast<__nv_bfloat16*>(b.dv);
+  bp.status = p.status;
+  bp.T_tot = p.T_tot;
+  bp.Hq = p.Hq;
+  bp.Hkv = p.Hkv;
+  bp.G = p.Hq / p.Hkv;
+  bp.causal = p.causal;
+  bp.n_sink = p.n_sink;
+  bp.window = p.window;
+  bp.per_item = p.ps.kh_slots == 1 ? p.Hkv : 1;
+  bp.scale_log2 = p.scale * kLog2e;
+  bp.alpha = p.scale;
+  const size_t acc_bytes = sizeof(float) * (size_t)p.T_tot * p.Hq * D;
+  if (cudaMemsetAsync(b.dq_accum, 0, acc_bytes, stream) != cudaSuccess) return SINKATTN_ERR_CUDA;
+  const long long grid = (long long)p.ps.cap_items * bp.per_item;
+  if (grid < 1 || grid > 0x7fffffffLL) return SINKATTN_ERR_INVALID_ARG;
+  auto kern = bwd_tc_kernel<C>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+      cudaSuccess)
+    return SINKATTN_ERR_CUDA;
+  record_start(SINKATTN_KERNEL_BWD, stream);
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, bp);
+  record_stop(SINKATTN_KERNEL_BWD, stream);
+  const long long n4 = (long long)p.T_tot * p.Hq * D / 4;
+  dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const float4*>(b.dq_accum), reinterpret_cast<uint2*>(b.dq), n4, p.scale);
+  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+}  // namespace
 
 size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int D) {
   return sizeof(float) * (size_t)T_tot * Hq * D;
 }
 
-int launch_bwd_tc(const AttnProblem&, const BwdBuffers&, cudaStream_t) {
-  return SINKATTN_ERR_UNSUPPORTED;
+int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
+  if (p.ps.tile != 128) return SINKATTN_ERR_UNSUPPORTED;  // 64-key block tiles: not yet
+  return p.D == 128 ? launch_cfg<128>(p, b, stream) : launch_cfg<64>(p, b, stream);
 }
 
 }  // namespace sk

@@ -216,7 +216,9 @@ int launch_split(const DecodeProblem& p, int chunk, cudaStream_t stream) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SINKATTN_ERR_CUDA;
   dim3 grid(p.num_splits, p.Hkv, p.B);
+  record_start(SINKATTN_KERNEL_DECODE, stream);
   kern<<<grid, kDecThreads, smem, stream>>>(p, chunk);
+  record_stop(SINKATTN_KERNEL_DECODE, stream);
   dim3 g2(p.Hq, p.B);
   decode_combine_kernel<T, D><<<g2, D, 0, stream>>>(p, p.num_splits);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;

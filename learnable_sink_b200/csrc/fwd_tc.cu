@@ -446,7 +446,9 @@ int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaS
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
+  record_start(SINKATTN_KERNEL_FWD, stream);
   kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, fp);
+  record_stop(SINKATTN_KERNEL_FWD, stream);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

@@ -10,6 +10,20 @@
 
 namespace sk {
 
+// Events recorded around a main kernel (profiling hook; both null = off).
+struct KernelEvents {
+  cudaEvent_t start = nullptr, stop = nullptr;
+};
+KernelEvents kernel_events(int which);
+inline void record_start(int which, cudaStream_t s) {
+  const KernelEvents e = kernel_events(which);
+  if (e.start) cudaEventRecord(e.start, s);
+}
+inline void record_stop(int which, cudaStream_t s) {
+  const KernelEvents e = kernel_events(which);
+  if (e.stop) cudaEventRecord(e.stop, s);
+}
+
 struct PlanLaunch {
   void* plan;
   PlanSizes sizes;
@@ -52,7 +66,8 @@ struct BwdBuffers {
   void* dk;
   void* dv;
   float* dsink;
-  float* delta;         // [T_tot, Hq] workspace
+  float* delta;         // [Hq, T_tot] workspace (head-major)
+  float* lse2;          // [Hq, T_tot] workspace: LSE_new * log2(e), -inf -> +inf
   float* dsink_part;    // [n_part_blocks, Hq] workspace
   float* dq_accum;      // [T_tot, Hq, D] fp32 workspace (tensor path)
   int n_part_blocks;

@@ -25,7 +25,7 @@ struct SimtArgs {
   const float* v;
   const float* sink;
   const int* plan;
-  int Hq, Hkv, causal, n_sink, window, tile;
+  int Hq, Hkv, causal, n_sink, window, tile, T_tot;
   float scale_log2;  // alpha * log2(e)
   int* status;
 };
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kWarps * 32) dq_simt_kernel(SimtArgs a, const 
     const int qi = it.tile_start + r;
     const long long row = (long long)(it.seq_start + qi) * a.Hq + head;
     const float lse2 = lse[row] * kLog2e;
-    const float dl = delta[row];
+    const float dl = delta[(long long)head * a.T_tot + it.seq_start + qi];
     float qv[E], dov[E], acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kWarps * 32) dkdv_simt_kernel(SimtArgs a, cons
           s = warp_sum(s) * a.scale_log2;
           dp = warp_sum(dp);
           const float p = exp2f(s - lse[row] * kLog2e);
-          const float ds = p * (dp - delta[row]);
+          const float ds = p * (dp - delta[(long long)head * a.T_tot + it.seq_start + qi]);
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             dka[e] += ds * a.q[row * D + lane + 32 * e];
@@ -230,6 +230,7 @@ SimtArgs make_args(const AttnProblem& p) {
   a.n_sink = p.n_sink;
   a.window = p.window;
   a.tile = p.ps.tile;
+  a.T_tot = p.T_tot;
   a.scale_log2 = p.scale * kLog2e;
   a.status = p.status;
   return a;

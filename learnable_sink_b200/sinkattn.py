@@ -70,6 +70,7 @@ def lib():
         L.sinkattn_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
         L.sinkattn_decode.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _i, _i,
                                       _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
+        L.sinkattn_set_kernel_events.argtypes = [_i, _vp, _vp]
         L.sinkattn_get_status.argtypes = [_vp]
         L.sinkattn_clear_status.argtypes = [_vp]
         L.sinkattn_error_string.restype = _c.c_char_p
@@ -147,8 +148,13 @@ class Plan:
         if nbytes == 0:
             raise SinkAttnError("sinkattn_plan_bytes", 1)
         self.buf = torch.empty(nbytes, dtype=torch.uint8, device=mask.cu_seqlens.device)
-        _check("sinkattn_plan", lib().sinkattn_plan(T_tot, Hq, Hkv, _c.byref(self._cm),
-                                                    _ptr(self.buf), nbytes, _stream(stream)))
+        self.rebuild(stream)
+
+    def rebuild(self, stream=None) -> None:
+        """Rebuild the schedule in place (e.g. after the mask arrays changed)."""
+        _check("sinkattn_plan", lib().sinkattn_plan(self.T_tot, self.Hq, self.Hkv,
+                                                    _c.byref(self._cm), _ptr(self.buf),
+                                                    self.buf.numel(), _stream(stream)))
 
     @property
     def nbytes(self) -> int:
@@ -236,6 +242,18 @@ def decode(q, k_cache, v_cache, cache_seqlens, n_sink: int, window: int, sink,
         int(n_sink), int(window), _ptr(sink), _ptr(out), _ptr(lse), _ptr(sink_s), int(num_splits),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return out, lse, sink_s
+
+
+KERNEL_FWD, KERNEL_BWD, KERNEL_DECODE = 0, 1, 2
+
+
+def set_kernel_events(which: int, start=None, stop=None) -> None:
+    """Have later calls record torch.cuda.Event ``start``/``stop`` around their
+    main kernel (events must already have been recorded once, so that torch
+    has created them).  Pass None, None to stop."""
+    sp = None if start is None else _vp(start.cuda_event)
+    ep = None if stop is None else _vp(stop.cuda_event)
+    _check("sinkattn_set_kernel_events", lib().sinkattn_set_kernel_events(int(which), sp, ep))
 
 
 def get_status(stream=None) -> int:

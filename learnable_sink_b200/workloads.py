@@ -219,3 +219,50 @@ def decode(B: int = 32, n_sink: int = 4, window: int = 1020, Hq: int = 32,
     sink = None if sink_std is None else _normal(gen, (Hq,), torch.float32, sink_std)
     return DecodeInputs(f"StreamingLLM decode B{B} cache {n_sink}+{window} Hq{Hq} Hkv{Hkv} D{D}",
                         q, kc, vc, cs, n_sink, window, sink, 1.0 / math.sqrt(D))
+
+
+def visible_pairs(spec: MaskSpec, Hq: int, Hkv: int) -> int:
+    """Number of visible (query, key, query-head) triples of a mask: the unit
+    of algorithmic work (forward 4*D flop each, backward 10*D).  Counted from
+    closed forms per sequence (causal / StreamingLLM band) or per selected
+    block; bookkeeping only."""
+    lens = (spec.cu_seqlens[1:] - spec.cu_seqlens[:-1]).tolist()
+    G = Hq // Hkv
+    if spec.block_indices is None:
+        total = 0
+        for L in lens:
+            i = np.arange(L, dtype=np.int64)
+            if not spec.causal:
+                total += L * L
+            elif spec.window <= 0:
+                total += L * (L + 1) // 2
+            else:
+                win = np.minimum(i + 1, spec.window)
+                sink = np.minimum(spec.n_sink, np.maximum(0, i + 1 - spec.window))
+                total += int((win + sink).sum())
+        return int(total) * Hq
+    bq, bk = spec.block_q, spec.block_k
+    bi = spec.block_indices.numpy()
+    total = 0
+    for g in range(Hkv):
+        r = 0
+        for L in lens:
+            nqb = (L + bq - 1) // bq
+            for qb in range(nqb):
+                blocks = set(int(b) for b in bi[g, r] if b >= 0)
+                qi = np.arange(qb * bq, min(qb * bq + bq, L))
+                for b in blocks:
+                    kj = np.arange(b * bk, min(b * bk + bk, L))
+                    if spec.causal and spec.window <= 0:
+                        # count kj <= qi in closed form per row
+                        total += int(np.clip(qi[:, None] - kj[None, :] >= 0, 0, 1).sum()) \
+                            if b == qb else (len(qi) * len(kj) if b < qb else 0)
+                    else:
+                        vis = np.ones((len(qi), len(kj)), dtype=bool)
+                        if spec.causal:
+                            vis &= kj[None, :] <= qi[:, None]
+                        if spec.window > 0:
+                            vis &= (kj[None, :] < spec.n_sink) | (qi[:, None] - kj[None, :] < spec.window)
+                        total += int(vis.sum())
+                r += 1
+    return int(total) * G

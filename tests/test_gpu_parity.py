@@ -269,3 +269,24 @@ def test_decode_rotation_invariance():
     # same set of tokens: equal up to summation order
     assert max_abs(np64(o0), np64(o1)) <= 1e-2
     assert max_abs(np64(l0), np64(l1)) <= 1e-5
+
+
+# ------------------------------------------------------------ bf16 tensor-core backward
+
+BF16_BWD = {
+    "causal_ragged_D128_G4": dict(cu=[0, 300, 555], Hq=8, Hkv=2, D=128),
+    "causal_D64_G4": dict(cu=[0, 384], Hq=8, Hkv=2, D=64),
+    "causal_D128_G1": dict(cu=[0, 200, 457], Hq=2, Hkv=2, D=128),
+    "band_D128": dict(cu=[0, 900], Hq=4, Hkv=2, D=128, n_sink=4, window=200),
+    "band_varlen_D64_G2": dict(cu=[0, 50, 700], Hq=4, Hkv=2, D=64, n_sink=4, window=130),
+    "no_sink_D128": dict(cu=[0, 260], Hq=4, Hkv=1, D=128, sink_std=None),
+    "extreme_sinks": dict(cu=[0, 260], Hq=4, Hkv=1, D=128, sink_values=[-80.0, -20.0, 20.0, 80.0]),
+    "non_causal": dict(cu=[0, 100, 300], Hq=4, Hkv=2, D=128, causal=False),
+}
+
+
+@pytest.mark.parametrize("name", list(BF16_BWD))
+def test_bf16_backward(name):
+    inp = _bf16_inputs(name, BF16_BWD[name], seed=21)
+    out, lse, ss, m, plan = run_fwd(inp)
+    _compare_bwd(inp, run_bwd(inp, out, lse, m, plan))
