@@ -211,6 +211,34 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
                     float *sink_s, int num_splits, void *workspace,
                     size_t workspace_bytes, sinkattn_stream_t stream);
 
+/* ---- ring-buffer decode without caller scratch ------------------------------
+ * No counterpart on the pages: this is a service for callers of this library.
+ * Same computation, arguments and results as sinkattn_decode, minus the
+ * workspace.  It is for callers that cannot hand out scratch memory -- e.g. a
+ * serving loop that reserves all device memory before requests arrive and may
+ * not allocate while they are in flight (cudaMalloc can block on the device and
+ * can fail under memory pressure), or a plain C program that owns only its
+ * input and output buffers.  The per-split partials go to a fixed 4 MiB array
+ * in the library's device image (every GPU that loads the library keeps it
+ * until the process exits); nothing is allocated.
+ *   - Limit: B * Hq * num_splits * (D + 2) * 4 bytes must fit in 4 MiB.  With
+ *     num_splits = 0 the automatic split count is lowered until it fits;
+ *     a problem that does not fit even with one split, or an explicit
+ *     num_splits that does not fit, returns SINKATTN_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array and leaves its contents behind; each
+ *     call writes every partial it reads, so nothing needs clearing, but calls
+ *     that overlap on the GPU (different streams, or concurrent host threads)
+ *     race on the array and must be serialised by the caller. */
+int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scale,
+                            const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *cache_seqlens, int n_sink, int window,
+                            const float *learnable_sink, void *out, float *lse_new,
+                            float *sink_s, int num_splits, sinkattn_stream_t stream);
+
 /* ---- profiling hook ---------------------------------------------------------
  * Records CUDA events around the main kernel of later calls, on the stream
  * that kernel is launched on, so a caller can time that kernel alone (the
