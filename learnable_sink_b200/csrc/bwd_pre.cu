@@ -17,92 +17,103 @@ namespace sk {
 namespace {
 
 constexpr int kPreThreads = 256;
-constexpr int kPreTokens = 64;  // tokens per CTA
+constexpr int kPreTokens = 16;   // tokens per CTA
+constexpr int kRows = 8;         // rows in flight per warp
 constexpr int kMaxHeads = 256;
 
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
+// D/32 elements of one row held by a lane, converted to fp32.
 template <typename T, int D>
-__device__ __forceinline__ float row_dot(const T* a, const T* b, int lane) {
-  float s = 0.f;
-  if constexpr (sizeof(T) == 2) {
-    // D/32 bf16 per lane, loaded as one 4- or 8-byte vector
-    constexpr int E = D / 32;
-    const __nv_bfloat16* pa = reinterpret_cast<const __nv_bfloat16*>(a) + lane * E;
-    const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(b) + lane * E;
-    if constexpr (E == 4) {
-      const uint2 ua = *reinterpret_cast<const uint2*>(pa);
-      const uint2 ub = *reinterpret_cast<const uint2*>(pb);
-      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&ua);
-      const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&ub);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float2 fx = __bfloat1622float2(x[e]), fy = __bfloat1622float2(y[e]);
-        s += fx.x * fy.x + fx.y * fy.y;
+struct RowFrag {
+  static constexpr int E = D / 32;
+  float v[E];
+  __device__ __forceinline__ void load(const T* row, int lane) {
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(row) + lane * E;
+      if constexpr (E == 4) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+      } else {
+        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(p));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        v[0] = a.x; v[1] = a.y;
       }
     } else {
-      const uint32_t ua = *reinterpret_cast<const uint32_t*>(pa);
-      const uint32_t ub = *reinterpret_cast<const uint32_t*>(pb);
-      const float2 fx = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ua));
-      const float2 fy = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ub));
-      s = fx.x * fy.x + fx.y * fy.y;
-    }
-  } else {
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) s += a[lane + 32 * e] * b[lane + 32 * e];
+      for (int e = 0; e < E; ++e) v[e] = __ldg(row + lane * E + e);
+    }
   }
-  return warp_sum(s);
-}
+};
 
+// One warp owns one head of the CTA's tokens, kRows rows at a time: all loads
+// of a group are issued before any reduction, so each lane keeps 2 kRows loads
+// in flight.  Delta and LSE2 of consecutive tokens land in consecutive words
+// of the head-major arrays; the warp also writes the CTA's dsink partial for
+// its head (fixed order, so dsink is bitwise deterministic).
 template <typename T, int D>
 __global__ void __launch_bounds__(kPreThreads) preprocess_kernel(
     const T* out, const T* dout, const float* lse, const float* sink, float* delta,
     float* lse2, float* part, int T_tot, int Hq) {
-  __shared__ float wpart[kPreThreads / 32][kMaxHeads];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NW = kPreThreads / 32;
-  for (int hh = threadIdx.x; hh < NW * kMaxHeads; hh += kPreThreads)
-    (&wpart[0][0])[hh] = 0.f;
-  __syncthreads();
   const int t0 = blockIdx.x * kPreTokens;
-  const int t1 = min(t0 + kPreTokens, T_tot);
-  const long long r0 = (long long)t0 * Hq, r1 = (long long)t1 * Hq;
-  // warp w handles rows r0 + w, r0 + w + NW, ... in order (deterministic)
-  for (long long r = r0 + warp; r < r1; r += NW) {
-    const float d = row_dot<T, D>(out + r * D, dout + r * D, lane);
-    if (lane == 0) {
-      const int h = (int)(r % Hq);
-      const long long t = r / Hq;
-      const float l = lse[r];
-      delta[(long long)h * T_tot + t] = d;
-      lse2[(long long)h * T_tot + t] = (l == -INFINITY) ? INFINITY : l * kLog2e;
-      if (sink) {
-        const float ps = __expf(sink[h] - lse[r]);
-        wpart[warp][h] -= d * ps;
-      }
-    }
-  }
-  __syncthreads();
-  if (sink) {
-    for (int h = threadIdx.x; h < Hq; h += kPreThreads) {
-      float s = 0.f;
+  for (int h = warp; h < Hq; h += kPreThreads / 32) {
+    const float a = sink ? __ldg(sink + h) : 0.f;
+    float dsum = 0.f;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) s += wpart[w][h];
-      part[(long long)blockIdx.x * Hq + h] = s;
+    for (int g = 0; g < kPreTokens; g += kRows) {
+      RowFrag<T, D> o[kRows], d[kRows];
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        const int t = min(t0 + g + r, T_tot - 1);
+        const long long row = ((long long)t * Hq + h) * D;
+        o[r].load(out + row, lane);
+        d[r].load(dout + row, lane);
+      }
+      float acc[kRows];
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        acc[r] = 0.f;
+#pragma unroll
+        for (int e = 0; e < RowFrag<T, D>::E; ++e) acc[r] += o[r].v[e] * d[r].v[e];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
+      // lane r (< kRows) writes token t0 + g + r
+      float mine = 0.f;
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) mine = (lane == r) ? acc[r] : mine;
+      const int t = t0 + g + lane;
+      float contrib = 0.f;
+      if (lane < kRows && t < T_tot) {
+        const float l = __ldg(lse + (long long)t * Hq + h);
+        delta[(long long)h * T_tot + t] = mine;
+        lse2[(long long)h * T_tot + t] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+        if (sink) contrib = -mine * __expf(a - l);  // -Delta * p_sink
+      }
+      dsum += contrib;
+    }
+    if (sink) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+      if (lane == 0) part[(long long)blockIdx.x * Hq + h] = dsum;
     }
   }
 }
 
+// dsink[h] = sum of the per-CTA partials: one warp per head, lanes stride
+// over the partials in a fixed order, then a fixed butterfly.
 __global__ void dsink_reduce_kernel(const float* part, int n_blocks, int Hq, float* dsink) {
-  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  const int h = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (h >= Hq) return;
   float s = 0.f;
-  for (int b = 0; b < n_blocks; ++b) s += part[(long long)b * Hq + h];
-  dsink[h] = s;
+  for (int b = lane; b < n_blocks; b += 32) s += part[(long long)b * Hq + h];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) dsink[h] = s;
 }
 
 }  // namespace
@@ -128,7 +139,7 @@ int launch_bwd_preprocess(const AttnProblem& p, const BwdBuffers& b, cudaStream_
       preprocess_kernel<float, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   }
   if (p.sink && b.dsink)
-    dsink_reduce_kernel<<<(p.Hq + 127) / 128, 128, 0, stream>>>(b.dsink_part, nb, p.Hq, b.dsink);
+    dsink_reduce_kernel<<<(p.Hq + 3) / 4, 128, 0, stream>>>(b.dsink_part, nb, p.Hq, b.dsink);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

@@ -31,9 +31,13 @@ namespace sk {
 
 namespace {
 
-template <int D_>
+// KT = 128: 128-key tiles, query tiles of 128 tokens x 1 head.
+// KT = 64 (64-key block selection): M = 64 for the key-side MMAs (tensor-memory
+// rows m at lanes m % 16 + 32 (m / 16)), query tiles of 64 tokens x 2 heads so
+// the dQ MMA keeps M = 128.
+template <int D_, int KT_>
 struct BwdCfg {
-  static constexpr int D = D_, KT = 128, TQ = 128, HPT = 1;
+  static constexpr int D = D_, KT = KT_, TQ = KT_, HPT = 128 / KT_;
   static constexpr int DH = D / 64;
   static constexpr int Q_BYTES = 128 * D * 2;   // Q or dO tile (128 rows)
   static constexpr int KV_BYTES = KT * D * 2;   // K or V tile
@@ -80,17 +84,26 @@ __device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
 // Packed bf16 P^T / dS^T columns: warpgroup c writes its 64 query columns
 // as 32 packed words at the front of its own fp32 slice [64c, 64c + 64), so
 // it never overwrites fp32 values the other warpgroup has yet to read.  K step
 // kk (16 query columns) of the TS-MMA A operand therefore starts at:
 __device__ __forceinline__ constexpr uint32_t a_col(int kk) { return (kk / 4) * 64 + (kk % 4) * 8; }
+
+// fp32 add of a shared-memory box into global memory through the tensor map
+// (bulk reduction; rows past the tensor's extent are skipped by the hardware)
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src,
+                                                  int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -101,7 +114,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                   const __grid_constant__ CUtensorMap tmap_do,
                   const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmap_v,
+                  const __grid_constant__ CUtensorMap tmap_dq, const BwdParams p) {
   constexpr int D = C::D, KT = C::KT, TQ = C::TQ, HPT = C::HPT, NS = C::NS, DH = C::DH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,7 +152,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(bar_kv, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_qf + s, 1);
-      mbar_init(bar_qe + s, 1);
+      mbar_init(bar_qe + s, 2);  // released by the two compute warpgroups
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
@@ -159,6 +173,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     prefetch_tensormap(&tmap_do);
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
+    prefetch_tensormap(&tmap_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -263,8 +278,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int kk = 0; kk < KT / 16; ++kk)
           mma_ss(tmem + C::DP_COL, sdesc_sw128(sDS + kk * 2048, KT * 128, 1024),
                  sdesc_sw128(sK + kk * 2048, C::KV_BYTES / DH, 1024), id_q, kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq);
-        mma_commit(bar_qe + s);
+        mma_commit(bar_dq);  // the compute warps release stage s after flushing dQ
       }
       mma_commit(bar_fin);
       wait_noabort(bar_fin, 0);
@@ -274,44 +288,63 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int cw = warp / 4;          // query-column half
     const int wq = warp % 4;          // TMEM lane quadrant
     const int tw = wq * 32 + lane;    // 0..127 within the warpgroup
-    const int r = tw;                 // key row (= TMEM lane)
+    // key row held by this thread's TMEM lane (with KT = 64 only lanes 0-15
+    // of each quadrant carry rows; the others join the collective loads)
+    const int r = KT == 128 ? tw : wq * 16 + (lane & 15);
+    const bool row_ok = KT == 128 || lane < 16;
     const int kj = k0 + r;            // sequence-local key
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const float* lse_s = s_lse + 64 * cw;
     const float* dl_s = s_dl + 64 * cw;
+    // The next iteration's entry and (for 64 of the threads) its LSE2 / Delta
+    // values are loaded one iteration ahead, so global-load latency stays off
+    // the critical path.
+    auto fetch = [&](int i, int& e, float& l2, float& dl) {
+      e = __ldg(ent + i / GH);
+      l2 = INFINITY;
+      dl = 0.f;
+      if (tw < 64) {
+        const int q0 = (e >> 1) * TQ;
+        const int col = 64 * cw + tw;
+        const int tok = col / HPT, hh = col % HPT;
+        const int h0 = kvh * p.G + (i % GH) * HPT;
+        if (tok < it.seq_len - q0) {
+          const long long gi = (long long)(h0 + hh) * p.T_tot + it.seq_start + q0 + tok;
+          l2 = __ldg(p.lse2 + gi);
+          dl = __ldg(p.delta + gi);
+        }
+      }
+    };
+    int e_nx = 0;
+    float l2_nx = INFINITY, dl_nx = 0.f;
+    if (n_it > 0) fetch(0, e_nx, l2_nx, dl_nx);
     bool ok = true;
     for (int i = 0; i < n_it; ++i) {
-      const int e = __ldg(ent + i / GH);
+      const int e = e_nx;
       const int q0 = (e >> 1) * TQ;
       const bool partial = (e & 1) != 0;
       const int h0 = kvh * p.G + (i % GH) * HPT;
       const int q_len = min(TQ, it.seq_len - q0);
-      // this warpgroup's 64 query columns: log2-domain LSE and Delta
-      named_bar_sync(1 + cw, 128);
+      named_bar_sync(1 + cw, 128);  // previous iteration's smem reads are done
       if (tw < 64) {
-        const int col = 64 * cw + tw;
-        const int tok = col / HPT, hh = col % HPT;
-        const bool valid = tok < q_len;
-        const long long gi = (long long)(h0 + hh) * p.T_tot + it.seq_start + q0 + tok;
-        s_lse[col] = valid ? __ldg(p.lse2 + gi) : INFINITY;
-        s_dl[col] = valid ? __ldg(p.delta + gi) : 0.f;
+        s_lse[64 * cw + tw] = l2_nx;
+        s_dl[64 * cw + tw] = dl_nx;
       }
       named_bar_sync(1 + cw, 128);
-      // P^T = exp2(S^T * alpha * log2e - LSE2)
+      if (i + 1 < n_it) fetch(i + 1, e_nx, l2_nx, dl_nx);
+      // P^T = exp2(S^T * alpha * log2e - LSE2), 32 columns at a time
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s, i & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
       float P[64];
-      {
-        uint32_t a[32], b[32];
-        tmem_ld32(tmem + lane_off + C::S_COL + 64 * cw, a);
-        tmem_ld32(tmem + lane_off + C::S_COL + 64 * cw + 32, b);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + C::S_COL + 64 * cw + 32 * h2, a);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          P[c] = fast_exp2(__uint_as_float(a[c]) * p.scale_log2 - lse_s[c]);
-          P[c + 32] = fast_exp2(__uint_as_float(b[c]) * p.scale_log2 - lse_s[c + 32]);
-        }
+        for (int c = 0; c < 32; ++c)
+          P[32 * h2 + c] = fast_exp2(__uint_as_float(a[c]) * p.scale_log2 - lse_s[32 * h2 + c]);
       }
       if (partial) {
 #pragma unroll
@@ -334,17 +367,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t ds[32];
-      {
-        uint32_t a[32], b[32];
-        tmem_ld32(tmem + lane_off + C::DP_COL + 64 * cw, a);
-        tmem_ld32(tmem + lane_off + C::DP_COL + 64 * cw + 32, b);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + C::DP_COL + 64 * cw + 32 * h2, a);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          ds[c] = pack_bf16x2(P[2 * c] * (__uint_as_float(a[2 * c]) - dl_s[2 * c]),
-                              P[2 * c + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[2 * c + 1]));
-          ds[c + 16] = pack_bf16x2(P[32 + 2 * c] * (__uint_as_float(b[2 * c]) - dl_s[32 + 2 * c]),
-                                   P[33 + 2 * c] * (__uint_as_float(b[2 * c + 1]) - dl_s[33 + 2 * c]));
+          const int x = 32 * h2 + 2 * c;
+          ds[16 * h2 + c] = pack_bf16x2(P[x] * (__uint_as_float(a[2 * c]) - dl_s[x]),
+                                        P[x + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[x + 1]));
         }
       }
       tmem_st32(tmem + lane_off + C::DP_COL + 64 * cw, ds);
@@ -353,7 +385,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (i - 1) & 1, abort_flag, p.status));
         if (!ok) break;
       }
-      {
+      if (row_ok) {
         // row r of the [keys][64 queries] half-tile, 128-byte swizzle
         uint8_t* row = smem + C::OFF_DS + cw * (KT * 128) + r * 128;
 #pragma unroll
@@ -365,38 +397,52 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_ds);
-      // dQ tile: lanes are query rows; this warpgroup takes D/2 columns
+      // dQ tile: lanes are query rows; this warpgroup takes D/2 columns, 32
+      // at a time.  All MMAs of this iteration are complete, so the stage's
+      // Q (warpgroup 0) or dO (warpgroup 1) buffer takes the fp32 values
+      // (128-byte swizzle), and one thread adds them into the fp32 dQ buffer
+      // with bulk tensor reductions.  Query rows past the sequence end carry
+      // exact zeros (their P is 0), so adding them is harmless.
       ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t dq[D / 2];
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t a[32];
-        tmem_ld32(tmem + lane_off + C::DP_COL + (D / 2) * cw + 32 * c, a);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) dq[32 * c + x] = a[x];
-      }
-      tc_fence_before();
-      mbar_arrive(bar_dqf);
       {
-        const int qrow = tw;  // query row of the tile held by this lane
-        const int tok = qrow / HPT, hh = qrow % HPT;
-        if (tok < q_len) {
-          float* dst = p.dq_accum +
-                       ((long long)(it.seq_start + q0 + tok) * p.Hq + h0 + hh) * D + (D / 2) * cw;
+        const int s = i % NS;
+        uint8_t* stage = smem + (cw == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
+        const int qrow = tw;
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c)
-            red_add_v4(dst + 4 * c, __uint_as_float(dq[4 * c]), __uint_as_float(dq[4 * c + 1]),
-                       __uint_as_float(dq[4 * c + 2]), __uint_as_float(dq[4 * c + 3]));
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::DP_COL + (D / 2) * cw + 32 * c, a);
+          tmem_ld_wait();
+          if (c == D / 64 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar_dqf);  // the dP region may be overwritten
+          }
+          uint8_t* row = stage + c * (128 * 128) + qrow * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
+                make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+        }
+        fence_async_smem();
+        named_bar_sync(1 + cw, 128);
+        if (tw == 0) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_reduce_add_3d(&tmap_dq, stage + c * (128 * 128), (D / 2) * cw + 32 * c, h0,
+                              it.seq_start + q0);
+          bulk_commit();
+          bulk_wait_read0();      // the stage buffer has been read
+          mbar_arrive(bar_qe + s);
         }
       }
     }
+    if (tw == 0) bulk_wait0();    // reductions complete before the CTA exits
     // dK (warpgroup 0) and dV (warpgroup 1) rows of this key tile
     const bool have = n_it > 0 && ok &&
                       __all_sync(0xffffffffu, mbar_wait(bar_fin, 0, abort_flag, p.status));
-    const bool store = (n_it == 0 || have) && kj < it.seq_len;
+    const bool store = (n_it == 0 || have) && row_ok && kj < it.seq_len;
     __nv_bfloat16* dst_base = (cw == 0 ? p.dk : p.dv);
     uint4* dst = reinterpret_cast<uint4*>(dst_base + ((long long)(it.seq_start + kj) * p.Hkv + kvh) * D);
     const float f = cw == 0 ? p.alpha : 1.f;
@@ -438,14 +484,15 @@ __global__ void dq_convert_kernel(const float4* acc, uint2* dq, long long n4, fl
   dq[i] = make_uint2(pack_bf16x2(v.x * alpha, v.y * alpha), pack_bf16x2(v.z * alpha, v.w * alpha));
 }
 
-template <int D>
+template <int D, int KT>
 int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
-  using C = BwdCfg<D>;
-  CUtensorMap mq, mdo, mk, mv;
+  using C = BwdCfg<D, KT>;
+  CUtensorMap mq, mdo, mk, mv, mdq;
   if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
       !make_tmap_3d(&mdo, b.dout, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
       !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::KT) ||
-      !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::KT))
+      !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::KT) ||
+      !make_tmap_3d_f32(&mdq, b.dq_accum, p.T_tot, p.Hq, D, C::HPT, C::TQ))
     return SINKATTN_ERR_CUDA;
   BwdParams bp{};
   bp.plan = p.plan;
@@ -474,7 +521,7 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
   record_start(SINKATTN_KERNEL_BWD, stream);
-  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, bp);
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, mdq, bp);
   record_stop(SINKATTN_KERNEL_BWD, stream);
   const long long n4 = (long long)p.T_tot * p.Hq * D / 4;
   dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(
@@ -489,8 +536,10 @@ size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int D) {
 }
 
 int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
-  if (p.ps.tile != 128) return SINKATTN_ERR_UNSUPPORTED;  // 64-key block tiles: not yet
-  return p.D == 128 ? launch_cfg<128>(p, b, stream) : launch_cfg<64>(p, b, stream);
+  if (p.ps.tile == 128)
+    return p.D == 128 ? launch_cfg<128, 128>(p, b, stream) : launch_cfg<64, 128>(p, b, stream);
+  if ((p.Hq / p.Hkv) % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;  // 64-token tiles pair heads
+  return p.D == 128 ? launch_cfg<128, 64>(p, b, stream) : launch_cfg<64, 64>(p, b, stream);
 }
 
 }  // namespace sk

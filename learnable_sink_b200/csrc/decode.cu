@@ -176,6 +176,162 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeProblem
   }
 }
 
+// bf16 variant of the split kernel: the split's K and V rows are fetched
+// into shared memory by TMA bulk tensor copies (every byte requested at once,
+// no per-thread load latency), then scored and accumulated from shared memory
+// exactly as above.  A split longer than kChunkRows is processed in pieces
+// with an online rescale.
+constexpr int kChunkRows = 128;
+
+template <int D, int G>
+struct TmaDecGeom {
+  static constexpr int DH = D / 64;
+  static constexpr int ROWS_BYTES = kChunkRows * 128;         // one 64-column half
+  static constexpr int KV_BYTES = DH * ROWS_BYTES;            // K (or V) piece
+  static constexpr int OFF_K = 0, OFF_V = KV_BYTES, OFF_SC = 2 * KV_BYTES;
+  static constexpr int OFF_RED = OFF_SC + G * kChunkRows * 4;
+  static constexpr int LPR = D / 8, NGRP = kDecThreads / LPR;
+  static constexpr int OFF_BAR = OFF_RED + NGRP * G * D * 4;
+  static constexpr int SMEM = OFF_BAR + 64 + 128;
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecThreads) decode_tma_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+    DecodeProblem p, int chunk) {
+  using Geo = TmaDecGeom<D, G>;
+  constexpr int LPR = Geo::LPR, NGRP = Geo::NGRP, DH = Geo::DH;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+  float* sc = reinterpret_cast<float*>(sm + Geo::OFF_SC);    // [G][kChunkRows]
+  float* red = reinterpret_cast<float*>(sm + Geo::OFF_RED);  // [NGRP][G][D]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR);
+  __shared__ float m_s[G], l_s[G], f_s[G];
+  __shared__ int abort_s;
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int S = p.n_sink + p.window;
+  const int n_valid = min(max(p.cache_seqlens[b], 0), S);
+  const int s0 = split * chunk;
+  const int n = max(min(s0 + chunk, n_valid) - s0, 0);
+  const int tid = threadIdx.x, grp = tid / LPR, gl = tid % LPR;
+  const int c0 = gl * 8, hf = c0 / 64, cin = c0 % 64;
+  const int warp = tid >> 5, lane = tid & 31;
+  const float scale_log2 = p.scale * kLog2e;
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (tid < G) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
+  __syncthreads();
+
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.Hq + kvh * G) * D;
+  float qv[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    load8<__nv_bfloat16>(qb + h * D + c0, qv[h]);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) qv[h][c] *= scale_log2;
+  }
+  float acc[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
+
+  const int n_pieces = (n + kChunkRows - 1) / kChunkRows;
+  for (int pc = 0; pc < n_pieces; ++pc) {
+    const int base = pc * kChunkRows;
+    const int rows = min(kChunkRows, n - base);
+    if (tid == 0) {
+      mbar_expect_tx(bar, 2 * Geo::KV_BYTES);
+      const int row0 = b * S + s0 + base;  // rows past the split are read but unused
+      for (int h = 0; h < DH; ++h) {
+        tma_load_3d(sm + Geo::OFF_K + h * Geo::ROWS_BYTES, &tmap_k, bar, h * 64, kvh, row0);
+        tma_load_3d(sm + Geo::OFF_V + h * Geo::ROWS_BYTES, &tmap_v, bar, h * 64, kvh, row0);
+      }
+    }
+    if (!mbar_wait(bar, pc & 1, &abort_s, p.status)) break;
+    // scores of this piece
+    for (int r = grp; r < kChunkRows; r += NGRP) {
+      float kf[8];
+      const uint4 u = *reinterpret_cast<const uint4*>(sm + Geo::OFF_K + hf * Geo::ROWS_BYTES + r * 128 + cin * 2);
+      bf16x8_to_f32(u, kf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) s += qv[h][c] * kf[c];
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (gl == 0 && r < rows) sc[h * kChunkRows + r] = s;
+      }
+    }
+    __syncthreads();
+    // running max / sum per head (warp h handles head h)
+    for (int h = warp; h < G; h += kDecThreads / 32) {
+      float m = -INFINITY;
+      for (int i = lane; i < rows; i += 32) m = fmaxf(m, sc[h * kChunkRows + i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const float mo = m_s[h];
+      const float mn = fmaxf(mo, m);
+      float l = 0.f;
+      for (int i = lane; i < rows; i += 32) {
+        const float e = exp2f(sc[h * kChunkRows + i] - mn);
+        sc[h * kChunkRows + i] = e;
+        l += e;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (lane == 0) {
+        const float f = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+        f_s[h] = f;
+        l_s[h] = l_s[h] * f + l;
+        m_s[h] = mn;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float f = f_s[h];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[h][c] *= f;
+    }
+    for (int r = grp; r < rows; r += NGRP) {
+      float vf[8];
+      const uint4 u = *reinterpret_cast<const uint4*>(sm + Geo::OFF_V + hf * Geo::ROWS_BYTES + r * 128 + cin * 2);
+      bf16x8_to_f32(u, vf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float pr = sc[h * kChunkRows + r];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[h][c] += pr * vf[c];
+      }
+    }
+    __syncthreads();  // the piece's buffers may be refilled
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) red[((long long)grp * G + h) * D + c0 + c] = acc[h][c];
+  __syncthreads();
+  float* part = p.part + (((long long)b * p.Hq + kvh * G) * gridDim.x + split) * (D + 2);
+  for (int i = tid; i < G * D; i += kDecThreads) {
+    const int h = i / D, d = i % D;
+    float s = 0.f;
+    for (int g = 0; g < NGRP; ++g) s += red[((long long)g * G + h) * D + d];
+    part[(long long)h * gridDim.x * (D + 2) + d] = s;
+  }
+  if (tid < G) {
+    float* ph = part + (long long)tid * gridDim.x * (D + 2);
+    ph[D] = n > 0 ? m_s[tid] : -INFINITY;
+    ph[D + 1] = n > 0 ? l_s[tid] : 0.f;
+  }
+}
+
 // Merge splits + sink.  One CTA per (head, sequence), D threads.
 template <typename T, int D>
 __global__ void decode_combine_kernel(DecodeProblem p, int n_splits) {
@@ -207,8 +363,30 @@ __global__ void decode_combine_kernel(DecodeProblem p, int n_splits) {
   }
 }
 
+template <int D, int G>
+int launch_tma(const DecodeProblem& p, int chunk, cudaStream_t stream) {
+  using Geo = TmaDecGeom<D, G>;
+  const int S = p.n_sink + p.window;
+  CUtensorMap mk, mv;
+  if (!make_tmap_3d_plain(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, kChunkRows) ||
+      !make_tmap_3d_plain(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, kChunkRows))
+    return SINKATTN_ERR_CUDA;
+  auto kern = decode_tma_kernel<D, G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM) !=
+      cudaSuccess)
+    return SINKATTN_ERR_CUDA;
+  dim3 grid(p.num_splits, p.Hkv, p.B);
+  record_start(SINKATTN_KERNEL_DECODE, stream);
+  kern<<<grid, kDecThreads, Geo::SMEM, stream>>>(mk, mv, p, chunk);
+  record_stop(SINKATTN_KERNEL_DECODE, stream);
+  dim3 g2(p.Hq, p.B);
+  decode_combine_kernel<__nv_bfloat16, D><<<g2, D, 0, stream>>>(p, p.num_splits);
+  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
 template <typename T, int D, int G>
 int launch_split(const DecodeProblem& p, int chunk, cudaStream_t stream) {
+  if constexpr (sizeof(T) == 2) return launch_tma<D, G>(p, chunk, stream);
   using Geo = DecGeom<D>;
   const size_t smem = sizeof(float) * ((size_t)G * chunk + (size_t)Geo::NGRP * G * D);
   auto kern = decode_split_kernel<T, D, G>;

@@ -50,6 +50,10 @@ struct AttnProblem {
 };
 
 bool make_tmap_3d(CUtensorMap* map, const void* base, int T, int H, int D, int box_h, int box_t);
+bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
+                      int box_t);
+bool make_tmap_3d_plain(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
+                        int box_t);
 
 // forward
 int launch_fwd_simt(const AttnProblem& p, void* out, float* lse, float* sink_s,

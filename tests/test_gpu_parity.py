@@ -290,3 +290,36 @@ def test_bf16_backward(name):
     inp = _bf16_inputs(name, BF16_BWD[name], seed=21)
     out, lse, ss, m, plan = run_fwd(inp)
     _compare_bwd(inp, run_bwd(inp, out, lse, m, plan))
+
+
+@pytest.mark.parametrize("G,D,block", [(8, 64, 64), (2, 64, 64), (4, 128, 64), (4, 128, 128)])
+def test_bf16_backward_block_sparse(G, D, block):
+    cu = W.random_cu_seqlens(1400, 100, 600, 31)
+    bi = W.random_block_indices(cu, 2, block, block, 4, 32, shuffle=True)
+    mask = W.MaskSpec(causal=True, cu_seqlens=cu, block_indices=bi, block_q=block, block_k=block)
+    inp = W.make_attn("bs_bwd", T_tot=int(cu[-1]), Hq=2 * G, Hkv=2, D=D, dtype=torch.bfloat16,
+                      mask=mask, seed=33)
+    out, lse, ss, m, plan = run_fwd(inp)
+    _compare_bwd(inp, run_bwd(inp, out, lse, m, plan))
+
+
+def test_bf16_block_sparse_empty_rows_and_unselected_keys():
+    """Query blocks that select nothing, and key blocks no query selects
+    (their dK/dV must come out as exact zeros)."""
+    cu = torch.tensor([0, 300, 520], dtype=torch.int32)
+    bi = W.random_block_indices(cu, 2, 64, 64, 1, 41)
+    bi[:, 2, :] = -1
+    bi[0, 6, :] = -1
+    mask = W.MaskSpec(causal=True, cu_seqlens=cu, block_indices=bi, block_q=64, block_k=64)
+    for sink_std in (1.0, None):
+        inp = W.make_attn("bs_empty_bf16", T_tot=520, Hq=8, Hkv=2, D=64, dtype=torch.bfloat16,
+                          mask=mask, seed=43, sink_std=sink_std)
+        out, lse, ss, m, plan = run_fwd(inp)
+        _compare_fwd(inp, out, lse, ss)
+        grads = run_bwd(inp, out, lse, m, plan)
+        _compare_bwd(inp, grads)
+        vis = [oracle.visible_dense(520, 8, 2, g, **mask.oracle_kwargs()) for g in range(2)]
+        for g in range(2):
+            unseen = vis[g].sum(0) == 0
+            assert torch.all(grads[1].cpu()[torch.from_numpy(unseen), g].float() == 0)
+            assert torch.all(grads[2].cpu()[torch.from_numpy(unseen), g].float() == 0)
