@@ -21,9 +21,10 @@
 //   S^T = K Q^T (SS) | dP^T = V dO^T (SS) | dV += P^T dO (TS) |
 //   dK += dS^T Q (TS) | dQ = dS K (SS; dS^T also staged in shared memory)
 // Warps 0-7 compute (warpgroup c owns query columns [64c, 64c + 64), thread =
-// key row), warp 8 is the TMA producer, warp 9 issues MMAs.  The compute
-// warps also move each dQ tile out of tensor memory into an fp32 buffer with
-// vector reductions (a query row gets one contribution per visible key
+// key row), warp 8 is the TMA producer, warp 9 issues MMAs, warp 10 flushes
+// dQ.  The compute warps move each dQ tile out of tensor memory into the
+// finished stage's shared memory; the reducer adds it into an fp32 buffer with
+// bulk tensor reductions (a query row gets one contribution per visible key
 // tile); a small kernel converts it to bf16.
 #include "internal.h"
 
@@ -47,8 +48,8 @@ struct BwdCfg {
   static constexpr int NS_RAW = (SMEM_LIMIT - FIXED) / (2 * Q_BYTES);
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "shared memory");
-  static constexpr int THREADS = 10 * 32;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+  static constexpr int THREADS = 11 * 32;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, REDUCER_WARP = 10;
   static constexpr int S_COL = 0, DP_COL = 128, DK_COL = 256, DV_COL = 256 + D;
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_K = 0;
@@ -59,7 +60,7 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[128]
   static constexpr int OFF_DL = OFF_LSE + 512;            // float[128]
   static constexpr int OFF_BAR = OFF_DL + 512;
-  static constexpr int N_BARS = 1 + 2 * NS + 7;
+  static constexpr int N_BARS = 1 + 3 * NS + 7;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
@@ -123,7 +124,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* bar_kv = bars;
   uint64_t* bar_qf = bars + 1;
   uint64_t* bar_qe = bar_qf + NS;
-  uint64_t* bar_s = bar_qe + NS;
+  uint64_t* bar_dqs = bar_qe + NS;   // dQ tile of stage s staged in smem
+  uint64_t* bar_s = bar_dqs + NS;
   uint64_t* bar_dp = bar_s + 1;
   uint64_t* bar_p = bar_dp + 1;
   uint64_t* bar_ds = bar_p + 1;
@@ -152,7 +154,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(bar_kv, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_qf + s, 1);
-      mbar_init(bar_qe + s, 2);  // released by the two compute warpgroups
+      mbar_init(bar_qe + s, 1);    // released by the reducer warp
+      mbar_init(bar_dqs + s, 256); // every compute thread staged its dQ part
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
@@ -278,10 +281,35 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int kk = 0; kk < KT / 16; ++kk)
           mma_ss(tmem + C::DP_COL, sdesc_sw128(sDS + kk * 2048, KT * 128, 1024),
                  sdesc_sw128(sK + kk * 2048, C::KV_BYTES / DH, 1024), id_q, kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq);  // the compute warps release stage s after flushing dQ
+        mma_commit(bar_dq);  // stage s is released once its dQ tile has been flushed
       }
       mma_commit(bar_fin);
       wait_noabort(bar_fin, 0);
+    }
+  } else if (warp == C::REDUCER_WARP) {
+    // ------------------------------------------------------------ dQ reducer
+    // Adds each staged fp32 dQ tile into the global accumulator with bulk
+    // tensor reductions, waits until they have read the stage, and hands the
+    // stage back to the producer; the compute warps never wait for this.
+    if (lane == 0 && n_it > 0) {
+      for (int i = 0; i < n_it; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(bar_dqs + s, (i / NS) & 1, abort_flag, p.status)) break;
+        const int e = __ldg(ent + i / GH);
+        const int q_tok = it.seq_start + (e >> 1) * TQ;
+        const int h0 = kvh * p.G + (i % GH) * HPT;
+#pragma unroll
+        for (int cw = 0; cw < 2; ++cw) {
+          const uint8_t* stage = smem + (cw == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_reduce_add_3d(&tmap_dq, stage + c * (128 * 128), (D / 2) * cw + 32 * c, h0, q_tok);
+        }
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(bar_qe + s);
+      }
+      bulk_wait0();  // reductions complete before the CTA exits
     }
   } else {
     // ------------------------------------------------------------ compute
@@ -426,19 +454,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
         }
         fence_async_smem();
-        named_bar_sync(1 + cw, 128);
-        if (tw == 0) {
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_reduce_add_3d(&tmap_dq, stage + c * (128 * 128), (D / 2) * cw + 32 * c, h0,
-                              it.seq_start + q0);
-          bulk_commit();
-          bulk_wait_read0();      // the stage buffer has been read
-          mbar_arrive(bar_qe + s);
-        }
+        mbar_arrive(bar_dqs + s);  // the reducer warp takes it from here
       }
     }
-    if (tw == 0) bulk_wait0();    // reductions complete before the CTA exits
     // dK (warpgroup 0) and dV (warpgroup 1) rows of this key tile
     const bool have = n_it > 0 && ok &&
                       __all_sync(0xffffffffu, mbar_wait(bar_fin, 0, abort_flag, p.status));
