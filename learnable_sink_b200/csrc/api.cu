@@ -252,11 +252,10 @@ int sinkattn_decode_num_splits(int B, int Hq, int Hkv, int D, int n_sink, int wi
   if (B < 1 || Hkv < 1 || S < 1) return 1;
   int sms = 148, dev;
   if (current_device(&dev)) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // one 128-slot piece per CTA, and at least two CTAs per SM
+  // enough (sequence, KV head, split) items for about six per SM, so the
+  // persistent streaming kernel balances within a few percent
   const long long pairs = (long long)B * Hkv;
-  long long want = (S + 127) / 128;
-  const long long by_sms = ((long long)sms * 2 + pairs - 1) / pairs;
-  if (by_sms > want) want = by_sms;
+  long long want = ((long long)sms * 6 + pairs - 1) / pairs;
   long long max_split = (S + 63) / 64;
   if (want > max_split) want = max_split;
   if (want < 1) want = 1;

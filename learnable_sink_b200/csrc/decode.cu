@@ -176,159 +176,260 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeProblem
   }
 }
 
-// bf16 variant of the split kernel: the split's K and V rows are fetched
-// into shared memory by TMA bulk tensor copies (every byte requested at once,
-// no per-thread load latency), then scored and accumulated from shared memory
-// exactly as above.  A split longer than kChunkRows is processed in pieces
-// with an online rescale.
-constexpr int kChunkRows = 128;
+// Persistent streaming variant (bf16): one CTA per SM loops over work items
+// (sequence, KV head, split).  Warp 8 streams 64-row pieces of K and V with
+// TMA through an NSTG-stage ring that runs ahead across item boundaries, so
+// HBM stays busy while warps 0-7 compute.  A group of D/8 lanes holds one
+// row's 8-element slices; each group takes PR rows of a piece and reduces its
+// PR x G partial dot products with a butterfly that splits the values across
+// the group's lanes (log2 steps, each halving the values a lane keeps).
+constexpr int kPieceRows = 64;
+constexpr int kStreamStages = 4;
+constexpr int kConsumerThreads = 256;
 
 template <int D, int G>
-struct TmaDecGeom {
+struct StreamGeom {
   static constexpr int DH = D / 64;
-  static constexpr int ROWS_BYTES = kChunkRows * 128;         // one 64-column half
-  static constexpr int KV_BYTES = DH * ROWS_BYTES;            // K (or V) piece
-  static constexpr int OFF_K = 0, OFF_V = KV_BYTES, OFF_SC = 2 * KV_BYTES;
-  static constexpr int OFF_RED = OFF_SC + G * kChunkRows * 4;
-  static constexpr int LPR = D / 8, NGRP = kDecThreads / LPR;
-  static constexpr int OFF_BAR = OFF_RED + NGRP * G * D * 4;
-  static constexpr int SMEM = OFF_BAR + 64 + 128;
+  static constexpr int LPR = D / 8;                          // lanes per row
+  static constexpr int NGRP = kConsumerThreads / LPR;        // row groups
+  static constexpr int PR = kPieceRows / NGRP;               // rows per group per piece
+  static constexpr int V = PR * G;                           // values per lane before reduce
+  static constexpr int HALF_BYTES = kPieceRows * 128;        // one 64-column half of a piece
+  static constexpr int PIECE_BYTES = DH * HALF_BYTES;        // K or V piece
+  static constexpr int STAGE_BYTES = 2 * PIECE_BYTES;
+  static constexpr int OFF_SC = kStreamStages * STAGE_BYTES; // float [G][kPieceRows]
+  static constexpr int OFF_RED = OFF_SC + G * kPieceRows * 4;  // float [8 warps][G][D]
+  static constexpr int OFF_BAR = OFF_RED + 8 * G * D * 4;
+  // + 1024: the kernel rounds the dynamic shared-memory base up to 1024 bytes
+  static constexpr int SMEM = OFF_BAR + 2 * kStreamStages * 8 + 1024;
+  static constexpr int LOG_LPR = LPR == 16 ? 4 : 3;
+  static constexpr int LOG_V = V >= 32 ? 5 : V >= 16 ? 4 : V >= 8 ? 3 : V >= 4 ? 2 : V >= 2 ? 1 : 0;
+  static constexpr int KS = LOG_V < LOG_LPR ? LOG_V : LOG_LPR;  // splitting steps
+  static constexpr int KEEP = V >> KS;                        // values a lane ends with
+  static_assert(PR >= 1 && (1 << LOG_V) == V, "power-of-two rows x heads");
 };
 
+// Sum each of the V values over the LPR lanes of a group; afterwards lane gl
+// holds KEEP totals, value index idx(gl, j) (see decode_value_index).
+template <int V, int LPR>
+__device__ __forceinline__ void butterfly_reduce(float (&v)[V], int gl) {
+  int c = V;
+#pragma unroll
+  for (int o = LPR / 2; o >= 1; o >>= 1) {
+    if (c > 1) {
+      const int half = c / 2;
+      const bool upper = (gl & o) != 0;
+#pragma unroll
+      for (int i = 0; i < V / 2; ++i) {
+        if (i < half) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      c = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+}
+
+template <int LOG_V, int LOG_LPR, int KS>
+__device__ __forceinline__ int decode_value_index(int gl, int j) {
+  int idx = 0;
+#pragma unroll
+  for (int k = 0; k < KS; ++k)
+    idx |= ((gl >> (LOG_LPR - 1 - k)) & 1) << (LOG_V - 1 - k);
+  return idx | j;
+}
+
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads) decode_tma_kernel(
+__global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-    DecodeProblem p, int chunk) {
-  using Geo = TmaDecGeom<D, G>;
-  constexpr int LPR = Geo::LPR, NGRP = Geo::NGRP, DH = Geo::DH;
+    DecodeProblem p, int chunk, int n_items) {
+  using Geo = StreamGeom<D, G>;
+  constexpr int LPR = Geo::LPR, NGRP = Geo::NGRP, PR = Geo::PR, V = Geo::V, DH = Geo::DH;
   extern __shared__ uint8_t dsm_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
-  float* sc = reinterpret_cast<float*>(sm + Geo::OFF_SC);    // [G][kChunkRows]
-  float* red = reinterpret_cast<float*>(sm + Geo::OFF_RED);  // [NGRP][G][D]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR);
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  float* sc = reinterpret_cast<float*>(sm + Geo::OFF_SC);
+  float* red = reinterpret_cast<float*>(sm + Geo::OFF_RED);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR);
+  uint64_t* empty = full + kStreamStages;
   __shared__ float m_s[G], l_s[G], f_s[G];
   __shared__ int abort_s;
-
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int S = p.n_sink + p.window;
-  const int n_valid = min(max(p.cache_seqlens[b], 0), S);
-  const int s0 = split * chunk;
-  const int n = max(min(s0 + chunk, n_valid) - s0, 0);
-  const int tid = threadIdx.x, grp = tid / LPR, gl = tid % LPR;
-  const int c0 = gl * 8, hf = c0 / 64, cin = c0 % 64;
-  const int warp = tid >> 5, lane = tid & 31;
-  const float scale_log2 = p.scale * kLog2e;
-
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(bar, 1);
+    for (int i = 0; i < kStreamStages; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, kConsumerThreads);
+    }
     abort_s = 0;
     fence_mbar_init();
   }
-  if (tid < G) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
   __syncthreads();
+  auto item_rows = [&](int item, int& b, int& kvh, int& split, int& n) {
+    split = item % p.num_splits;
+    kvh = (item / p.num_splits) % p.Hkv;
+    b = item / (p.num_splits * p.Hkv);
+    const int n_valid = min(max(p.cache_seqlens[b], 0), S);
+    n = max(min(split * chunk + chunk, n_valid) - split * chunk, 0);
+  };
 
-  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.Hq + kvh * G) * D;
-  float qv[G][8];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    load8<__nv_bfloat16>(qb + h * D + c0, qv[h]);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) qv[h][c] *= scale_log2;
+  if (warp == kConsumerThreads / 32) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int pc = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        int b, kvh, split, n;
+        item_rows(item, b, kvh, split, n);
+        for (int r0 = 0; r0 < n; r0 += kPieceRows, ++pc) {
+          const int st = pc % kStreamStages;
+          if (!mbar_wait(empty + st, ((pc / kStreamStages) & 1) ^ 1, &abort_s, p.status)) return;
+          mbar_expect_tx(full + st, Geo::STAGE_BYTES);
+          const int row0 = b * S + split * chunk + r0;  // rows past the split are unused
+          uint8_t* base = sm + st * Geo::STAGE_BYTES;
+          for (int h = 0; h < DH; ++h) {
+            tma_load_3d(base + h * Geo::HALF_BYTES, &tmap_k, full + st, h * 64, kvh, row0);
+            tma_load_3d(base + Geo::PIECE_BYTES + h * Geo::HALF_BYTES, &tmap_v, full + st, h * 64,
+                        kvh, row0);
+          }
+        }
+      }
+    }
+    return;
   }
-  float acc[G][8];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
 
-  const int n_pieces = (n + kChunkRows - 1) / kChunkRows;
-  for (int pc = 0; pc < n_pieces; ++pc) {
-    const int base = pc * kChunkRows;
-    const int rows = min(kChunkRows, n - base);
-    if (tid == 0) {
-      mbar_expect_tx(bar, 2 * Geo::KV_BYTES);
-      const int row0 = b * S + s0 + base;  // rows past the split are read but unused
-      for (int h = 0; h < DH; ++h) {
-        tma_load_3d(sm + Geo::OFF_K + h * Geo::ROWS_BYTES, &tmap_k, bar, h * 64, kvh, row0);
-        tma_load_3d(sm + Geo::OFF_V + h * Geo::ROWS_BYTES, &tmap_v, bar, h * 64, kvh, row0);
-      }
-    }
-    if (!mbar_wait(bar, pc & 1, &abort_s, p.status)) break;
-    // scores of this piece
-    for (int r = grp; r < kChunkRows; r += NGRP) {
-      float kf[8];
-      const uint4 u = *reinterpret_cast<const uint4*>(sm + Geo::OFF_K + hf * Geo::ROWS_BYTES + r * 128 + cin * 2);
-      bf16x8_to_f32(u, kf);
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float s = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) s += qv[h][c] * kf[c];
-#pragma unroll
-        for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (gl == 0 && r < rows) sc[h * kChunkRows + r] = s;
-      }
-    }
-    __syncthreads();
-    // running max / sum per head (warp h handles head h)
-    for (int h = warp; h < G; h += kDecThreads / 32) {
-      float m = -INFINITY;
-      for (int i = lane; i < rows; i += 32) m = fmaxf(m, sc[h * kChunkRows + i]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const float mo = m_s[h];
-      const float mn = fmaxf(mo, m);
-      float l = 0.f;
-      for (int i = lane; i < rows; i += 32) {
-        const float e = exp2f(sc[h * kChunkRows + i] - mn);
-        sc[h * kChunkRows + i] = e;
-        l += e;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      if (lane == 0) {
-        const float f = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-        f_s[h] = f;
-        l_s[h] = l_s[h] * f + l;
-        m_s[h] = mn;
-      }
-    }
-    __syncthreads();
+  // ------------------------------------------------------------ consumers
+  const int grp = tid / LPR, gl = tid % LPR;
+  const int c0 = gl * 8, hf = c0 / 64, cin = c0 % 64;
+  const float scale_log2 = p.scale * kLog2e;
+  int pc = 0;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    int b, kvh, split, n;
+    item_rows(item, b, kvh, split, n);
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.Hq + kvh * G) * D;
+    float qv[G][8];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float f = f_s[h];
+      load8<__nv_bfloat16>(qb + h * D + c0, qv[h]);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[h][c] *= f;
+      for (int c = 0; c < 8; ++c) qv[h][c] *= scale_log2;
     }
-    for (int r = grp; r < rows; r += NGRP) {
-      float vf[8];
-      const uint4 u = *reinterpret_cast<const uint4*>(sm + Geo::OFF_V + hf * Geo::ROWS_BYTES + r * 128 + cin * 2);
-      bf16x8_to_f32(u, vf);
+    float acc[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
+    if (tid < G) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
+    named_bar_sync(1, kConsumerThreads);
+    for (int r0 = 0; r0 < n; r0 += kPieceRows, ++pc) {
+      const int st = pc % kStreamStages;
+      const int rows = min(kPieceRows, n - r0);
+      if (!mbar_wait(full + st, (pc / kStreamStages) & 1, &abort_s, p.status)) return;
+      const uint8_t* kbuf = sm + st * Geo::STAGE_BYTES;
+      const uint8_t* vbuf = kbuf + Geo::PIECE_BYTES;
+      // scores: this group's PR rows, all G heads
+      float v[V];
+#pragma unroll
+      for (int rr = 0; rr < PR; ++rr) {
+        const int r = grp * PR + rr;
+        float kf[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), kf);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float a = 0.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) a += qv[h][c] * kf[c];
+          v[rr * G + h] = a;
+        }
+      }
+      butterfly_reduce<V, LPR>(v, gl);
+#pragma unroll
+      for (int j = 0; j < Geo::KEEP; ++j) {
+        const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
+        const int rr = idx / G, h = idx % G, r = grp * PR + rr;
+        if (r < rows) sc[h * kPieceRows + r] = v[j];
+      }
+      named_bar_sync(1, kConsumerThreads);
+      // online softmax over this piece (warp h handles head h)
+      for (int h = warp; h < G; h += kConsumerThreads / 32) {
+        float m = -INFINITY;
+        for (int i = lane; i < rows; i += 32) m = fmaxf(m, sc[h * kPieceRows + i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float mo = m_s[h];
+        const float mn = fmaxf(mo, m);
+        float l = 0.f;
+        for (int i = lane; i < rows; i += 32) {
+          const float e = exp2f(sc[h * kPieceRows + i] - mn);
+          sc[h * kPieceRows + i] = e;
+          l += e;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) {
+          const float f = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+          f_s[h] = f;
+          l_s[h] = l_s[h] * f + l;
+          m_s[h] = mn;
+        }
+      }
+      named_bar_sync(1, kConsumerThreads);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float pr = sc[h * kChunkRows + r];
+        const float f = f_s[h];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[h][c] += pr * vf[c];
+        for (int c = 0; c < 8; ++c) acc[h][c] *= f;
       }
+#pragma unroll
+      for (int rr = 0; rr < PR; ++rr) {
+        const int r = grp * PR + rr;
+        if (r < rows) {
+          float vf[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(vbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), vf);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pr = sc[h * kPieceRows + r];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[h][c] += pr * vf[c];
+          }
+        }
+      }
+      mbar_arrive(empty + st);            // the stage may be refilled
+      named_bar_sync(1, kConsumerThreads);  // sc may be overwritten
     }
-    __syncthreads();  // the piece's buffers may be refilled
-  }
+    // reduce the groups: lanes with equal gl in the two halves of a warp,
+    // then the eight warps through shared memory (fixed order)
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) red[((long long)grp * G + h) * D + c0 + c] = acc[h][c];
-  __syncthreads();
-  float* part = p.part + (((long long)b * p.Hq + kvh * G) * gridDim.x + split) * (D + 2);
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    const int h = i / D, d = i % D;
-    float s = 0.f;
-    for (int g = 0; g < NGRP; ++g) s += red[((long long)g * G + h) * D + d];
-    part[(long long)h * gridDim.x * (D + 2) + d] = s;
-  }
-  if (tid < G) {
-    float* ph = part + (long long)tid * gridDim.x * (D + 2);
-    ph[D] = n > 0 ? m_s[tid] : -INFINITY;
-    ph[D + 1] = n > 0 ? l_s[tid] : 0.f;
+      for (int c = 0; c < 8; ++c) {
+        float x = acc[h][c];
+        for (int o = 16; o >= LPR; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        acc[h][c] = x;
+      }
+    if (lane < LPR) {
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red[(warp * G + h) * D + c0 + c] = acc[h][c];
+    }
+    named_bar_sync(1, kConsumerThreads);
+    float* part = p.part + (((long long)b * p.Hq + kvh * G) * p.num_splits + split) * (D + 2);
+    for (int i = tid; i < G * D; i += kConsumerThreads) {
+      const int h = i / D, d = i % D;
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerThreads / 32; ++w) s += red[(w * G + h) * D + d];
+      part[(long long)h * p.num_splits * (D + 2) + d] = s;
+    }
+    if (tid < G) {
+      float* ph = part + (long long)tid * p.num_splits * (D + 2);
+      ph[D] = n > 0 ? m_s[tid] : -INFINITY;
+      ph[D + 1] = n > 0 ? l_s[tid] : 0.f;
+    }
+    named_bar_sync(1, kConsumerThreads);  // red / m_s reused by the next item
   }
 }
 
@@ -365,19 +466,23 @@ __global__ void decode_combine_kernel(DecodeProblem p, int n_splits) {
 
 template <int D, int G>
 int launch_tma(const DecodeProblem& p, int chunk, cudaStream_t stream) {
-  using Geo = TmaDecGeom<D, G>;
+  using Geo = StreamGeom<D, G>;
   const int S = p.n_sink + p.window;
   CUtensorMap mk, mv;
-  if (!make_tmap_3d_plain(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, kChunkRows) ||
-      !make_tmap_3d_plain(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, kChunkRows))
+  if (!make_tmap_3d_plain(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, kPieceRows) ||
+      !make_tmap_3d_plain(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, kPieceRows))
     return SINKATTN_ERR_CUDA;
-  auto kern = decode_tma_kernel<D, G>;
+  auto kern = decode_stream_kernel<D, G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
-  dim3 grid(p.num_splits, p.Hkv, p.B);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int n_items = p.B * p.Hkv * p.num_splits;
+  const int grid = n_items < sms ? n_items : sms;
   record_start(SINKATTN_KERNEL_DECODE, stream);
-  kern<<<grid, kDecThreads, Geo::SMEM, stream>>>(mk, mv, p, chunk);
+  kern<<<grid, kConsumerThreads + 32, Geo::SMEM, stream>>>(mk, mv, p, chunk, n_items);
   record_stop(SINKATTN_KERNEL_DECODE, stream);
   dim3 g2(p.Hq, p.B);
   decode_combine_kernel<__nv_bfloat16, D><<<g2, D, 0, stream>>>(p, p.num_splits);
