@@ -86,7 +86,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -195,6 +195,52 @@ def run_reference(args, world, rank):
                 e2e={"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                      "d2h_bytes_per_step": 0})
     print(json.dumps(line), flush=True)
+
+
+def measure_config(S, inp, dev, steps=10, warmup=3):
+    """Plan+fwd+bwd of one workload: per-call and per-kernel times (CUDA events)."""
+    T, Hq, Hkv, D = inp.shape
+    pairs = W.visible_pairs(inp.mask, Hq, Hkv)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    sink, dout = inp.sink.to(dev), inp.dout.to(dev)
+    mask = S.Mask.from_spec(inp.mask, dev)
+    plan = S.Plan(T, Hq, Hkv, mask)
+    out = torch.empty_like(q)
+    lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+    ss = torch.empty_like(lse)
+    ws = torch.empty(S.bwd_workspace_bytes(q, k, mask), dtype=torch.uint8, device=dev)
+
+    def step():
+        plan.rebuild()
+        S.fwd(q, k, v, sink, mask, plan, scale=inp.scale, out=out, lse=lse, sink_s=ss)
+        S.bwd(q, k, v, out, dout, lse, sink, mask, plan, scale=inp.scale, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    ev = {n: [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+          for n in ("s0", "s1", "f0", "f1", "b0", "b1")}
+    for lst in ev.values():
+        for e in lst:
+            e.record()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        S.set_kernel_events(S.KERNEL_FWD, ev["f0"][i], ev["f1"][i])
+        S.set_kernel_events(S.KERNEL_BWD, ev["b0"][i], ev["b1"][i])
+        ev["s0"][i].record()
+        step()
+        ev["s1"][i].record()
+    torch.cuda.synchronize()
+    S.set_kernel_events(S.KERNEL_FWD, None, None)
+    S.set_kernel_events(S.KERNEL_BWD, None, None)
+
+    def mean(a, b):
+        return sum(x.elapsed_time(y) for x, y in zip(ev[a], ev[b])) / steps
+
+    step_ms, f_ms, b_ms = mean("s0", "s1"), mean("f0", "f1"), mean("b0", "b1")
+    return {"workload": inp.name, "visible_pairs": pairs,
+            "plan_fwd_bwd_ms": step_ms, "tflops": 14 * D * pairs / (step_ms * 1e-3) / 1e12,
+            "fwd_kernel_ms": f_ms, "fwd_kernel_tflops": 4 * D * pairs / (f_ms * 1e-3) / 1e12,
+            "bwd_kernel_ms": b_ms, "bwd_kernel_tflops": 10 * D * pairs / (b_ms * 1e-3) / 1e12}
 
 
 def run_ours(args, world, rank, local):
@@ -374,6 +420,13 @@ def run_ours(args, world, rank, local):
                                     "frac_of_hbm": dec_ach / peaks["hbm_gbs"]},
         },
     }
+    if args.configs:
+        extra = []
+        for mk in (W.band, W.varlen):
+            r = measure_config(S, mk(), dev)
+            r["frac_of_sustained"] = r["tflops"] / peak_tf
+            extra.append(r)
+        line["other_configs"] = extra
     if world == 1:
         dt, fl, desc, cores = cpu_oracle_sample(inp, 4096, 2)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
@@ -384,9 +437,11 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the band / varlen block-sparse measurements")
     args = ap.parse_args()
     world, rank, local = init_dist() if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)

@@ -59,6 +59,8 @@ def _load():
             lib.oracle_fwd_rows.argtypes = _PROBLEM + [
                 _d, _d, _d, _d, ctypes.c_int, _i32, _d, _d, _d]
             lib.oracle_bwd.argtypes = _PROBLEM + [_d, _d, _d, _d, _d, _d, _d, _d, _d]
+            lib.oracle_bwd_sampled.argtypes = _PROBLEM + [
+                _d, _d, _d, _d, _d, ctypes.c_int, _i32, _d, ctypes.c_int, _i32, _d, _d]
             lib.oracle_decode.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [
                 _d, _d, _d, _i32, ctypes.c_int, ctypes.c_int, _d, _d, _d, _d]
             lib.oracle_visible_dense.argtypes = _PROBLEM + [ctypes.c_int, _u8]
@@ -154,6 +156,24 @@ def bwd(q, k, v, sink, dout, scale, **mask):
     if rc != 0:
         raise MemoryError("oracle_bwd: allocation failed")
     return dq, dk, dv, dsink
+
+
+def bwd_sampled(q, k, v, sink, dout, scale, rows, keys, **mask):
+    """Gradients on samples of a problem: dQ of rows [(token, head), ...] and
+    dK / dV of keys [(token, kv_head), ...].  Returns (dq [n_rows, D],
+    dk [n_keys, D], dv [n_keys, D]) in float64."""
+    q, k, v, sink, dout = _f64(q), _f64(k), _f64(v), _f64(sink), _f64(dout)
+    T, Hq, Hkv, D = _shapes(q, k)
+    rows = _i32arr(rows).reshape(-1, 2)
+    keys = _i32arr(keys).reshape(-1, 2)
+    pr = _Problem(T, Hq, Hkv, D, scale, **mask)
+    dq = np.zeros((rows.shape[0], D)); dk = np.zeros((keys.shape[0], D)); dv = np.zeros((keys.shape[0], D))
+    rc = _load().oracle_bwd_sampled(*pr.args, _p(q, _d), _p(k, _d), _p(v, _d), _p(sink, _d),
+                                    _p(dout, _d), rows.shape[0], _p(rows, _i32), _p(dq, _d),
+                                    keys.shape[0], _p(keys, _i32), _p(dk, _d), _p(dv, _d))
+    if rc != 0:
+        raise MemoryError("oracle_bwd_sampled: allocation failed")
+    return dq, dk, dv
 
 
 def decode(q, k_cache, v_cache, cache_seqlens, n_sink, window, sink, scale):

@@ -338,6 +338,104 @@ int oracle_bwd(OM_PROBLEM_ARGS, const double *q, const double *k,
     return 0;
 }
 
+/* Backward on samples of a large problem: dQ of selected rows (i, h) and
+ * dK / dV of selected keys (j, g), each from the same explicit Jacobian as
+ * oracle_bwd.  A key's gradient needs the statistics (M, den, mu) of every
+ * row that sees it, so phase 1 computes them for every row of the KV heads
+ * the sampled keys belong to; phase 2 sums over those rows key by key. */
+int oracle_bwd_sampled(OM_PROBLEM_ARGS, const double *q, const double *k,
+                       const double *v, const double *sink, const double *dout,
+                       int n_rows, const int32_t *rows, double *dq_rows,
+                       int n_keys, const int32_t *keys, double *dk_keys,
+                       double *dv_keys) {
+    om_problem p = make_problem(OM_PROBLEM_PASS);
+    const int G = Hq / Hkv;
+    const int L = max_seq_len(T_tot, cu_seqlens, n_seq, seqlen);
+    /* dQ rows */
+#pragma omp parallel
+    {
+        int *js = (int *)malloc(sizeof(int) * (size_t)L);
+        double *xs = (double *)malloc(sizeof(double) * (size_t)L);
+        double *o_row = (double *)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < n_rows; ++r) {
+            int i = rows[2 * r], h = rows[2 * r + 1], g = h / G;
+            om_rowstat st;
+            row_forward(&p, q, k, v, sink, i, h, o_row, &st, js, xs);
+            double *dqrow = dq_rows + (size_t)r * D;
+            for (int d = 0; d < D; ++d) dqrow[d] = 0.0;
+            if (st.M == -INFINITY) continue;
+            const double *dorow = dout + ((size_t)i * Hq + h) * D;
+            double m = 0.0;
+            for (int t = 0; t < st.n_vis; ++t)
+                m += exp(xs[t] - st.M) / st.den * dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D);
+            for (int t = 0; t < st.n_vis; ++t) {
+                const double *krow = k + ((size_t)js[t] * Hkv + g) * D;
+                double P = exp(xs[t] - st.M) / st.den;
+                double dx = P * (dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D) - m);
+                for (int d = 0; d < D; ++d) dqrow[d] += scale * dx * krow[d];
+            }
+        }
+        free(js); free(xs); free(o_row);
+    }
+    if (n_keys <= 0) return 0;
+    /* phase 1: statistics of every row of the involved KV heads */
+    const long long R = (long long)T_tot * Hq;
+    om_rowstat *st = (om_rowstat *)malloc(sizeof(om_rowstat) * (size_t)R);
+    double *mu = (double *)malloc(sizeof(double) * (size_t)R);
+    uint8_t *need = (uint8_t *)calloc((size_t)Hkv, 1);
+    if (!st || !mu || !need) { free(st); free(mu); free(need); return 1; }
+    for (int c = 0; c < n_keys; ++c) need[keys[2 * c + 1]] = 1;
+#pragma omp parallel
+    {
+        int *js = (int *)malloc(sizeof(int) * (size_t)L);
+        double *xs = (double *)malloc(sizeof(double) * (size_t)L);
+        double *o_row = (double *)malloc(sizeof(double) * (size_t)D);
+#pragma omp for schedule(dynamic, 4)
+        for (long r = 0; r < R; ++r) {
+            int i = (int)(r / Hq), h = (int)(r % Hq), g = h / G;
+            mu[r] = 0.0;
+            st[r].M = -INFINITY;
+            if (!need[g]) continue;
+            row_forward(&p, q, k, v, sink, i, h, o_row, &st[r], js, xs);
+            if (st[r].M == -INFINITY) continue;
+            const double *dorow = dout + (size_t)r * D;
+            double m = 0.0;
+            for (int t = 0; t < st[r].n_vis; ++t)
+                m += exp(xs[t] - st[r].M) / st[r].den *
+                     dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D);
+            mu[r] = m;
+        }
+        free(js); free(xs); free(o_row);
+    }
+    /* phase 2: per sampled key */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int c = 0; c < n_keys; ++c) {
+        int j = keys[2 * c], g = keys[2 * c + 1];
+        double *dkrow = dk_keys + (size_t)c * D, *dvrow = dv_keys + (size_t)c * D;
+        for (int d = 0; d < D; ++d) { dkrow[d] = 0.0; dvrow[d] = 0.0; }
+        int s = seq_of(&p, j);
+        const double *krow = k + ((size_t)j * Hkv + g) * D;
+        const double *vrow = v + ((size_t)j * Hkv + g) * D;
+        for (int i = seq_start(&p, s); i < seq_end(&p, s); ++i) {
+            if (!visible(&p, i, j, g)) continue;
+            for (int h = g * G; h < (g + 1) * G; ++h) {
+                long r = (long)i * Hq + h;
+                if (st[r].M == -INFINITY) continue;
+                const double *qrow = q + (size_t)r * D, *dorow = dout + (size_t)r * D;
+                double P = exp(scale * dot(qrow, krow, D) - st[r].M) / st[r].den;
+                double dx = P * (dot(dorow, vrow, D) - mu[r]);
+                for (int d = 0; d < D; ++d) {
+                    dkrow[d] += scale * dx * qrow[d];
+                    dvrow[d] += P * dorow[d];
+                }
+            }
+        }
+    }
+    free(st); free(mu); free(need);
+    return 0;
+}
+
 /* Ring-buffer decode.  q [B,Hq,D]; caches [B,S,Hkv,D] with S = n_sink+window;
  * cache_seqlens[b] = tokens ever appended (current token included). */
 int oracle_decode(int B, int Hq, int Hkv, int D, double scale,

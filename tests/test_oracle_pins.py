@@ -464,3 +464,20 @@ def test_decode_invariant_to_ring_rotation():
         got = oracle.decode(q, kr, vr, np.array([n0 + r], np.int32), n_sink, window, a, 0.4)
         for x, y in zip(ref, got):
             np.testing.assert_allclose(x, y, atol=1e-13)
+
+
+@pytest.mark.parametrize("mname", ["varlen_band", "block_sparse"])
+def test_sampled_backward_equals_full_backward(mname):
+    """The sampled-gradient routine (used at full sizes) reproduces the full
+    explicit-Jacobian backward on every sampled row and key."""
+    T, Hq, Hkv, D = 37, 4, 2, 16
+    mask = MASKS[mname] if mname != "block_sparse" else _block_sparse_mask()
+    q, k, v, a, dout = _random_problem(T, Hq, Hkv, D, seed=14)
+    dq, dk, dv, _ = oracle.bwd(q, k, v, a, dout, 0.3, **mask)
+    rng = np.random.default_rng(1)
+    rows = np.stack([rng.integers(0, T, 20), rng.integers(0, Hq, 20)], 1)
+    keys = np.stack([rng.integers(0, T, 15), rng.integers(0, Hkv, 15)], 1)
+    sq, sk, sv = oracle.bwd_sampled(q, k, v, a, dout, 0.3, rows, keys, **mask)
+    np.testing.assert_allclose(sq, dq[rows[:, 0], rows[:, 1]], atol=1e-13)
+    np.testing.assert_allclose(sk, dk[keys[:, 0], keys[:, 1]], atol=1e-13)
+    np.testing.assert_allclose(sv, dv[keys[:, 0], keys[:, 1]], atol=1e-13)
