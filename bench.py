@@ -305,6 +305,12 @@ def run_ours(args, world, rank, local):
         flush.zero_()
         decode_step()
     torch.cuda.synchronize()
+    if args.profile:  # launches for an external profiler only; nothing is timed
+        for _ in range(args.steps):
+            prefill_step()
+            decode_step()
+        torch.cuda.synchronize()
+        return
 
     K = args.steps
     evs = {n: [ev() for _ in range(K)] for n in
@@ -440,6 +446,9 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--profile", action="store_true",
+                    help="run warm-up + steps of the prefill and decode stages for a profiler "
+                         "(no timing, no JSON line)")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the band / varlen block-sparse measurements")
     args = ap.parse_args()

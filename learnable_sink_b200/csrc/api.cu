@@ -97,14 +97,14 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct BwdLayout {
   size_t delta, lse2, part, dq_accum, total;
 };
-BwdLayout bwd_layout(int dt, int T_tot, int Hq, int D) {
+BwdLayout bwd_layout(int dt, int T_tot, int Hq, int Hkv, int D) {
   BwdLayout L{};
   size_t off = 0;
   L.delta = off; off += round_up(sizeof(float) * (size_t)T_tot * Hq);
   L.lse2 = off; off += round_up(sizeof(float) * (size_t)T_tot * Hq);
   L.part = off; off += round_up(sizeof(float) * (size_t)preprocess_blocks(T_tot) * Hq);
   L.dq_accum = off;
-  if (dt == SINKATTN_BF16) off += round_up(bwd_tc_workspace_bytes(T_tot, Hq, D));
+  if (dt == SINKATTN_BF16) off += round_up(bwd_tc_workspace_bytes(T_tot, Hq, Hkv, D));
   L.total = off;
   return L;
 }
@@ -206,7 +206,7 @@ size_t sinkattn_bwd_workspace_bytes(sinkattn_dtype dt, int T_tot, int Hq, int Hk
                                     const sinkattn_mask* mask) {
   if (!mask_ok(T_tot, Hq, Hkv, mask) || (D != 64 && D != 128)) return 0;
   if (dt != SINKATTN_BF16 && dt != SINKATTN_FP32) return 0;
-  return bwd_layout(dt, T_tot, Hq, D).total;
+  return bwd_layout(dt, T_tot, Hq, Hkv, D).total;
 }
 
 int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
@@ -222,7 +222,7 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
   if (!aligned16(out) || !aligned16(dout) || !aligned16(lse_new) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (dsink && !aligned16(dsink)))
     return SINKATTN_ERR_INVALID_ARG;
-  const BwdLayout L = bwd_layout(dt, T_tot, Hq, D);
+  const BwdLayout L = bwd_layout(dt, T_tot, Hq, Hkv, D);
   if (workspace_bytes < L.total) return SINKATTN_ERR_WORKSPACE;
   p.scale = scale;
   char* ws = static_cast<char*>(workspace);
@@ -238,6 +238,8 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
   b.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   b.dsink_part = reinterpret_cast<float*>(ws + L.part);
   b.dq_accum = reinterpret_cast<float*>(ws + L.dq_accum);
+  b.dk_accum = b.dq_accum + (size_t)T_tot * Hq * D;
+  b.dv_accum = b.dk_accum + (size_t)T_tot * Hkv * D;
   b.n_part_blocks = preprocess_blocks(T_tot);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   rc = launch_bwd_preprocess(p, b, s);

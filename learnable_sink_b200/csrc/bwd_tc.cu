@@ -64,6 +64,7 @@ struct BwdCfg {
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+  static_assert(NS * Q_BYTES >= KT * D * 4, "Q stages must hold an fp32 dK tile");
 };
 
 struct BwdParams {
@@ -116,7 +117,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                   const __grid_constant__ CUtensorMap tmap_do,
                   const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v,
-                  const __grid_constant__ CUtensorMap tmap_dq, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmap_dq,
+                  const __grid_constant__ CUtensorMap tmap_dkacc,
+                  const __grid_constant__ CUtensorMap tmap_dvacc, const BwdParams p) {
   constexpr int D = C::D, KT = C::KT, TQ = C::TQ, HPT = C::HPT, NS = C::NS, DH = C::DH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -139,14 +142,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const PlanHdr* hdr = reinterpret_cast<const PlanHdr*>(p.plan);
   const int rank = blockIdx.x / p.per_item;
-  if (rank >= hdr->n_bwd_items) return;
+  if (rank >= min(hdr->n_bwd_units, hdr->cap_units)) return;
   const int rem = blockIdx.x % p.per_item;
-  const int idx = p.plan[hdr->off_bwd_order + rank];
-  const TileItem it = reinterpret_cast<const TileItem*>(p.plan + hdr->off_bwd_items)[idx];
+  // work unit: a slice of one key tile's reverse list (long lists are split)
+  const int4 unit = reinterpret_cast<const int4*>(p.plan + hdr->off_bwd_units)[
+      p.plan[hdr->off_bwd_unit_order + rank]];
+  const TileItem it = reinterpret_cast<const TileItem*>(p.plan + hdr->off_bwd_items)[unit.x];
+  const bool split_tile = unit.w > 1;  // partial dK/dV go through fp32 reductions
   const int kvh = it.kvh >= 0 ? it.kvh : rem;
-  const int* ent = p.plan + hdr->off_bwd_entries + it.entry_off;
+  const int* ent = p.plan + hdr->off_bwd_entries + it.entry_off + unit.y;
   const int GH = p.G / HPT;             // query-head groups per key tile
-  const int n_it = it.entry_len * GH;   // (query tile, head group) iterations
+  const int n_it = unit.z * GH;         // (query tile, head group) iterations
   const int k0 = it.tile_start;         // sequence-local first key
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -460,30 +466,68 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // dK (warpgroup 0) and dV (warpgroup 1) rows of this key tile
     const bool have = n_it > 0 && ok &&
                       __all_sync(0xffffffffu, mbar_wait(bar_fin, 0, abort_flag, p.status));
-    const bool store = (n_it == 0 || have) && row_ok && kj < it.seq_len;
-    __nv_bfloat16* dst_base = (cw == 0 ? p.dk : p.dv);
-    uint4* dst = reinterpret_cast<uint4*>(dst_base + ((long long)(it.seq_start + kj) * p.Hkv + kvh) * D);
-    const float f = cw == 0 ? p.alpha : 1.f;
-    if (have) {
+    if (!split_tile) {
+      const bool store = (n_it == 0 || have) && row_ok && kj < it.seq_len;
+      __nv_bfloat16* dst_base = (cw == 0 ? p.dk : p.dv);
+      uint4* dst = reinterpret_cast<uint4*>(dst_base + ((long long)(it.seq_start + kj) * p.Hkv + kvh) * D);
+      const float f = cw == 0 ? p.alpha : 1.f;
+      if (have) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + (cw == 0 ? C::DK_COL : C::DV_COL) + 32 * c, a);
+          tmem_ld_wait();
+          if (store) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[4 * c + v] = make_uint4(
+                  pack_bf16x2(__uint_as_float(a[8 * v]) * f, __uint_as_float(a[8 * v + 1]) * f),
+                  pack_bf16x2(__uint_as_float(a[8 * v + 2]) * f, __uint_as_float(a[8 * v + 3]) * f),
+                  pack_bf16x2(__uint_as_float(a[8 * v + 4]) * f, __uint_as_float(a[8 * v + 5]) * f),
+                  pack_bf16x2(__uint_as_float(a[8 * v + 6]) * f, __uint_as_float(a[8 * v + 7]) * f));
+          }
+        }
+      } else if (store) {
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+      }
+    } else if (have) {
+      // Split key tile: add this unit's fp32 dK (warpgroup 0) / dV (warpgroup 1)
+      // into the zeroed accumulators.  The Q (resp. dO) stages are reused for
+      // staging once the reducer warp has released every stage this unit used.
+      bool free_ok = true;
+      for (int s = 0; s < NS && s < n_it; ++s) {
+        const int last = s + ((n_it - 1 - s) / NS) * NS;  // last iteration on stage s
+        free_ok = free_ok && mbar_wait(bar_qe + s, (last / NS) & 1, abort_flag, p.status);
+      }
+      free_ok = __all_sync(0xffffffffu, free_ok);
       tc_fence_after();
+      uint8_t* stage = smem + (cw == 0 ? C::OFF_Q : C::OFF_DO);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t a[32];
         tmem_ld32(tmem + lane_off + (cw == 0 ? C::DK_COL : C::DV_COL) + 32 * c, a);
         tmem_ld_wait();
-        if (store) {
+        if (free_ok && row_ok) {
+          // box c: [KT rows][32 floats], 128-byte swizzle
+          uint8_t* row = stage + c * (KT * 128) + r * 128;
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[4 * c + v] = make_uint4(
-                pack_bf16x2(__uint_as_float(a[8 * v]) * f, __uint_as_float(a[8 * v + 1]) * f),
-                pack_bf16x2(__uint_as_float(a[8 * v + 2]) * f, __uint_as_float(a[8 * v + 3]) * f),
-                pack_bf16x2(__uint_as_float(a[8 * v + 4]) * f, __uint_as_float(a[8 * v + 5]) * f),
-                pack_bf16x2(__uint_as_float(a[8 * v + 6]) * f, __uint_as_float(a[8 * v + 7]) * f));
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) * 16)) =
+                make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
         }
       }
-    } else if (store) {
+      fence_async_smem();
+      named_bar_sync(1 + cw, 128);
+      if (free_ok && tw == 0) {
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < D / 32; ++c)
+          tma_reduce_add_3d(cw == 0 ? &tmap_dkacc : &tmap_dvacc, stage + c * (KT * 128), 32 * c,
+                            kvh, it.seq_start + k0);
+        bulk_commit();
+        bulk_wait0();
+      }
     }
   }
   tc_fence_before();
@@ -491,6 +535,37 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Key tiles whose reverse list was split into several work units: zero their
+// fp32 dK/dV accumulator rows before the backward kernel, and round them to
+// bf16 (dK scaled by alpha) after it.  One CTA per backward item; unsplit
+// items return at once.
+__global__ void split_tiles_kernel(const int* plan, float* dk_acc, float* dv_acc,
+                                   __nv_bfloat16* dk, __nv_bfloat16* dv, int Hkv, int D,
+                                   float alpha, int finish) {
+  // blockIdx.x = backward item, blockIdx.y = row of its key tile
+  const PlanHdr* h = reinterpret_cast<const PlanHdr*>(plan);
+  if ((int)blockIdx.x >= h->cap_items) return;
+  const TileItem it = reinterpret_cast<const TileItem*>(plan + h->off_bwd_items)[blockIdx.x];
+  if (it.entry_len < 0 || bwd_units_of(it.entry_len) <= 1 || (int)blockIdx.y >= it.tile_len) return;
+  const int kv0 = it.kvh >= 0 ? it.kvh : 0, kv1 = it.kvh >= 0 ? it.kvh + 1 : Hkv;
+  const long long base = ((long long)(it.seq_start + it.tile_start + blockIdx.y) * Hkv + kv0) * D;
+  const int n4 = (kv1 - kv0) * D / 4;
+  float4* ka = reinterpret_cast<float4*>(dk_acc + base);
+  float4* va = reinterpret_cast<float4*>(dv_acc + base);
+  for (int e = threadIdx.x; e < n4; e += blockDim.x) {
+    if (finish) {
+      const float4 x = ka[e], y = va[e];
+      reinterpret_cast<uint2*>(dk + base)[e] =
+          make_uint2(pack_bf16x2(x.x * alpha, x.y * alpha), pack_bf16x2(x.z * alpha, x.w * alpha));
+      reinterpret_cast<uint2*>(dv + base)[e] =
+          make_uint2(pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
+    } else {
+      ka[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      va[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 }
 
@@ -505,12 +580,14 @@ __global__ void dq_convert_kernel(const float4* acc, uint2* dq, long long n4, fl
 template <int D, int KT>
 int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   using C = BwdCfg<D, KT>;
-  CUtensorMap mq, mdo, mk, mv, mdq;
+  CUtensorMap mq, mdo, mk, mv, mdq, mdk, mdv;
   if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
       !make_tmap_3d(&mdo, b.dout, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
       !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::KT) ||
       !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::KT) ||
-      !make_tmap_3d_f32(&mdq, b.dq_accum, p.T_tot, p.Hq, D, C::HPT, C::TQ))
+      !make_tmap_3d_f32(&mdq, b.dq_accum, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
+      !make_tmap_3d_f32(&mdk, b.dk_accum, p.T_tot, p.Hkv, D, 1, C::KT) ||
+      !make_tmap_3d_f32(&mdv, b.dv_accum, p.T_tot, p.Hkv, D, 1, C::KT))
     return SINKATTN_ERR_CUDA;
   BwdParams bp{};
   bp.plan = p.plan;
@@ -532,15 +609,20 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   bp.alpha = p.scale;
   const size_t acc_bytes = sizeof(float) * (size_t)p.T_tot * p.Hq * D;
   if (cudaMemsetAsync(b.dq_accum, 0, acc_bytes, stream) != cudaSuccess) return SINKATTN_ERR_CUDA;
-  const long long grid = (long long)p.ps.cap_items * bp.per_item;
+  const long long grid = (long long)p.ps.cap_units * bp.per_item;
   if (grid < 1 || grid > 0x7fffffffLL) return SINKATTN_ERR_INVALID_ARG;
   auto kern = bwd_tc_kernel<C>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
+  const dim3 split_grid(p.ps.cap_items, C::KT);
+  split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
+                                                     p.Hkv, D, p.scale, 0);
   record_start(SINKATTN_KERNEL_BWD, stream);
-  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, mdq, bp);
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, mdq, mdk, mdv, bp);
   record_stop(SINKATTN_KERNEL_BWD, stream);
+  split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
+                                                     p.Hkv, D, p.scale, 1);
   const long long n4 = (long long)p.T_tot * p.Hq * D / 4;
   dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(
       reinterpret_cast<const float4*>(b.dq_accum), reinterpret_cast<uint2*>(b.dq), n4, p.scale);
@@ -549,8 +631,8 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
 
 }  // namespace
 
-size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int D) {
-  return sizeof(float) * (size_t)T_tot * Hq * D;
+size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int Hkv, int D) {
+  return sizeof(float) * (size_t)T_tot * D * (Hq + 2 * Hkv);  // dQ, dK, dV accumulators
 }
 
 int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {

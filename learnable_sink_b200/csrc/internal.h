@@ -74,13 +74,15 @@ struct BwdBuffers {
   float* lse2;          // [Hq, T_tot] workspace: LSE_new * log2(e), -inf -> +inf
   float* dsink_part;    // [n_part_blocks, Hq] workspace
   float* dq_accum;      // [T_tot, Hq, D] fp32 workspace (tensor path)
+  float* dk_accum;      // [T_tot, Hkv, D] fp32 workspace: split key tiles only
+  float* dv_accum;      // [T_tot, Hkv, D] fp32 workspace: split key tiles only
   int n_part_blocks;
 };
 int preprocess_blocks(int T_tot);
 int launch_bwd_preprocess(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream);
 int launch_bwd_simt(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream);
 int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream);
-size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int D);
+size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int Hkv, int D);
 
 // decode
 struct DecodeProblem {

@@ -19,6 +19,7 @@ struct PlanArgs {
   int causal, n_sink, window, n_qblk, max_blocks;
   int off_tile_base, off_fwd_items, off_fwd_order, off_fwd_entries;
   int off_bwd_items, off_bwd_order, off_bwd_entries, off_bwd_cursor;
+  int cap_units, off_bwd_units, off_bwd_unit_order, off_unit_base;
 };
 
 constexpr int kScanThreads = 1024;
@@ -313,6 +314,71 @@ __global__ void plan_zero_kernel(int* p, int n) {
   if (i < n) p[i] = 0;
 }
 
+// H: backward work units.  One CTA scans the per-item unit counts (item
+// order), then every item writes its units, then the units are ordered
+// longest first (counting sort on the entry count, at most kBwdChunk).
+__global__ void __launch_bounds__(kScanThreads) plan_units_scan_kernel(PlanArgs a) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const TileItem* items = reinterpret_cast<const TileItem*>(a.plan + a.off_bwd_items);
+  int* base = a.plan + a.off_unit_base;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < a.cap_items; b0 += kScanThreads) {
+    const int i = b0 + threadIdx.x;
+    int n = 0;
+    if (i < a.cap_items) {
+      const int len = items[i].entry_len;
+      n = len < 0 ? 0 : bwd_units_of(len);
+    }
+    int total;
+    const int ex = block_excl_scan(n, warp_tot, &total);
+    if (i < a.cap_items) base[i] = carry + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    hdr(a)->n_bwd_units = carry;
+    if (carry > a.cap_units) set_status(a.status, SINKATTN_ERR_BOUNDS);
+  }
+}
+
+__global__ void plan_units_fill_kernel(PlanArgs a) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.cap_items) return;
+  const TileItem it = reinterpret_cast<const TileItem*>(a.plan + a.off_bwd_items)[i];
+  if (it.entry_len < 0) return;
+  const int n = bwd_units_of(it.entry_len);
+  const int b = a.plan[a.off_unit_base + i];
+  int4* units = reinterpret_cast<int4*>(a.plan + a.off_bwd_units);
+  for (int c = 0; c < n && b + c < a.cap_units; ++c) {
+    const int first = c * kBwdChunk;
+    const int cnt = min(kBwdChunk, it.entry_len - first);
+    units[b + c] = make_int4(i, first, max(cnt, 0), n);
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) plan_units_order_kernel(PlanArgs a) {
+  __shared__ int cursor[kBwdChunk + 1];
+  __shared__ int hist[kBwdChunk + 1];
+  const int n_units = min(hdr(a)->n_bwd_units, a.cap_units);
+  const int4* units = reinterpret_cast<const int4*>(a.plan + a.off_bwd_units);
+  int* order = a.plan + a.off_bwd_unit_order;
+  if (threadIdx.x <= kBwdChunk) hist[threadIdx.x] = 0;
+  __syncthreads();
+  for (int u = threadIdx.x; u < n_units; u += kScanThreads)
+    atomicAdd(&hist[kBwdChunk - units[u].z], 1);  // bin 0 = longest
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int b = 0; b <= kBwdChunk; ++b) { cursor[b] = run; run += hist[b]; }
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < n_units; u += kScanThreads)
+    order[atomicAdd(&cursor[kBwdChunk - units[u].z], 1)] = u;
+}
+
 // G: sort every reverse list by query tile (insertion sort; lists are short).
 __global__ void plan_bwd_sort_kernel(PlanArgs a) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -356,6 +422,10 @@ int launch_plan(const PlanLaunch& L, cudaStream_t stream) {
   a.off_bwd_order = z.off_bwd_order;
   a.off_bwd_entries = z.off_bwd_entries;
   a.off_bwd_cursor = z.off_bwd_cursor;
+  a.cap_units = z.cap_units;
+  a.off_bwd_units = z.off_bwd_units;
+  a.off_bwd_unit_order = z.off_bwd_unit_order;
+  a.off_unit_base = z.off_unit_base;
 
   // header scalars known on the host (written by the first kernel)
   PlanHdr h{};
@@ -378,6 +448,10 @@ int launch_plan(const PlanLaunch& L, cudaStream_t stream) {
   h.off_bwd_entries = z.off_bwd_entries;
   h.off_bwd_cursor = z.off_bwd_cursor;
   h.total_words = z.total_words;
+  h.cap_units = z.cap_units;
+  h.off_bwd_units = z.off_bwd_units;
+  h.off_bwd_unit_order = z.off_bwd_unit_order;
+  h.off_unit_base = z.off_unit_base;
   const int nb = (z.cap_items + 255) / 256;
   plan_tiles_kernel<<<1, kScanThreads, 0, stream>>>(a, h);
   plan_fwd_count_kernel<<<nb, 256, 0, stream>>>(a);
@@ -388,6 +462,9 @@ int launch_plan(const PlanLaunch& L, cudaStream_t stream) {
   plan_zero_kernel<<<nb, 256, 0, stream>>>(a.plan + a.off_bwd_cursor, z.cap_items);
   plan_bwd_scatter_kernel<<<nb, 256, 0, stream>>>(a);
   plan_bwd_sort_kernel<<<nb, 256, 0, stream>>>(a);
+  plan_units_scan_kernel<<<1, kScanThreads, 0, stream>>>(a);
+  plan_units_fill_kernel<<<nb, 256, 0, stream>>>(a);
+  plan_units_order_kernel<<<1, kScanThreads, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

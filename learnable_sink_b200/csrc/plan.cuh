@@ -15,6 +15,12 @@
 //                        query tiles that see it), entries (query tile << 1) |
 //                        partial, each list sorted by query tile
 //   bwd_cursor[cap_items] scratch for the reverse scatter
+//   bwd_units[cap_units][4] backward work units: (bwd item, first entry,
+//                        entry count, number of units of that item); a
+//                        reverse list longer than kBwdChunk entries is split
+//                        so no single CTA serialises a very popular key tile
+//   bwd_unit_order[cap_units] units, longest first
+//   unit_base[cap_items] first unit of every bwd item
 // With no block_indices the lists do not depend on the KV head: one slot
 // (kvh = -1) serves every KV head.
 #pragma once
@@ -24,6 +30,7 @@ namespace sk {
 
 constexpr int kPlanMagic = 0x534b4150;  // 'SKAP'
 constexpr int kHdrWords = 32;
+constexpr int kBwdChunk = 32;  // reverse-list entries per backward work unit
 
 struct PlanHdr {
   int magic;
@@ -39,7 +46,10 @@ struct PlanHdr {
   int off_tile_base, off_fwd_items, off_fwd_order, off_fwd_entries;
   int off_bwd_items, off_bwd_order, off_bwd_entries, off_bwd_cursor;
   int total_words;
-  int pad[kHdrWords - 23];
+  int n_bwd_units;    // device-written
+  int cap_units;
+  int off_bwd_units, off_bwd_unit_order, off_unit_base;
+  int pad[kHdrWords - 28];
 };
 static_assert(sizeof(PlanHdr) == kHdrWords * 4, "plan header size");
 
@@ -96,10 +106,15 @@ __host__ __device__ __forceinline__ int classify_tile(int q0, int qlen, int k0, 
 
 // Host-side sizes of the plan for a problem.
 struct PlanSizes {
-  int tile, kh_slots, cap_tiles, cap_items, cap_entries, max_list;
+  int tile, kh_slots, cap_tiles, cap_items, cap_entries, max_list, cap_units;
   int off_tile_base, off_fwd_items, off_fwd_order, off_fwd_entries;
-  int off_bwd_items, off_bwd_order, off_bwd_entries, off_bwd_cursor, total_words;
+  int off_bwd_items, off_bwd_order, off_bwd_entries, off_bwd_cursor;
+  int off_bwd_units, off_bwd_unit_order, off_unit_base, total_words;
 };
+
+__host__ __device__ __forceinline__ int bwd_units_of(int entry_len) {
+  return entry_len <= kBwdChunk ? 1 : (entry_len + kBwdChunk - 1) / kBwdChunk;
+}
 
 inline PlanSizes plan_sizes(int T_tot, int Hkv, int n_seq, int max_seqlen, bool sparse,
                             int block, int max_blocks) {
@@ -129,6 +144,10 @@ inline PlanSizes plan_sizes(int T_tot, int Hkv, int n_seq, int max_seqlen, bool 
   s.off_bwd_order = take(s.cap_items);
   s.off_bwd_entries = take(s.cap_entries);
   s.off_bwd_cursor = take(s.cap_items);
+  s.cap_units = (int)((long long)s.cap_items + cap_entries / kBwdChunk + 1);
+  s.off_bwd_units = take((long long)s.cap_units * 4);
+  s.off_bwd_unit_order = take(s.cap_units);
+  s.off_unit_base = take(s.cap_items);
   s.total_words = (int)off;
   return s;
 }
