@@ -41,7 +41,14 @@ struct FwdCfg {
   static constexpr int NS_RAW = (SMEM_BUDGET - NQT * Q_BYTES) / (2 * KV_BYTES);
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "not enough shared memory for a two-stage ring");
-  static constexpr int THREADS = (4 * NQT + 2) * 32;
+  static constexpr int MIN_BLOCKS = 1;
+  // With two softmax warpgroups and one CTA per SM, registers are moved to the
+  // softmax warpgroups: the producer and MMA warps then share a warpgroup with
+  // two idle warps (setmaxnreg works on whole warpgroups), 12 warps in all,
+  // 168 registers per thread at launch and 256 x 224 + 128 x 56 = 384 x 168.
+  static constexpr bool REBALANCE = (NQT == 2 && MIN_BLOCKS == 1);
+  static constexpr int SOFTMAX_REGS = 224, AUX_REGS = 56;
+  static constexpr int THREADS = (4 * NQT + (REBALANCE ? 4 : 2)) * 32;
   static constexpr int PRODUCER_WARP = 4 * NQT;
   static constexpr int MMA_WARP = 4 * NQT + 1;
   static constexpr int S_COL = 0;                // S_t at t * TK
@@ -58,7 +65,6 @@ struct FwdCfg {
   static constexpr int N_BARS = 1 + 4 * NS + 3 * NQT + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
-  static constexpr int MIN_BLOCKS = (TK == 64 && D == 64) ? 2 : 1;
 };
 
 struct FwdParams {
@@ -145,6 +151,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 4 * NQT) {
+    if constexpr (C::REBALANCE) regs_dec<C::AUX_REGS>();
+  }
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n > 0) {
@@ -234,8 +243,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       mma_commit(bar_fin);
       wait_noabort(bar_fin, 0);
     }
-  } else {
+  } else if (warp < 4 * NQT) {
     // ------------------------------------------------------------ softmax
+    if constexpr (C::REBALANCE) regs_inc<C::SOFTMAX_REGS>();
     const int t = warp / 4;                     // query tile of this warpgroup
     const int wq = warp % 4;                    // TMEM lane quadrant
     const int r = wq * 32 + lane;               // row of the tile
@@ -253,6 +263,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s + t, j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      // raw scores x = Q.K (the scale is folded into the exponent below)
       float x[TK];
 #pragma unroll
       for (int c = 0; c < TK / 32; ++c) {
@@ -260,16 +271,23 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
         tmem_ld32(s_addr + c * 32, rr);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(rr[i]) * p.scale_log2;
+        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(rr[i]);
       }
       if (e & 1) {  // partial tile: element mask
 #pragma unroll
         for (int c = 0; c < TK; ++c)
           if (!visible_elem(qi, k0 + c, it.seq_len, p.causal, p.n_sink, p.window)) x[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max with eight independent accumulators (short dependency chains)
+      float m8[8];
 #pragma unroll
-      for (int c = 0; c < TK; ++c) mx = fmaxf(mx, x[c]);
+      for (int a = 0; a < 8; ++a) m8[a] = x[a];
+#pragma unroll
+      for (int c = 8; c < TK; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+#pragma unroll
+      for (int a = 0; a < 4; ++a) m8[a] = fmaxf(m8[a], m8[a + 4]);
+      const float mraw = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+      const float mx = mraw * p.scale_log2;  // scale > 0: max commutes with it
       // Lazy rescale: the running reference max m only moves when the tile
       // max exceeds it by more than 2^8.  Per-row decision, but the TMEM
       // load/store are warp-collective, so the warp rescales together and
@@ -297,20 +315,24 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       }
       if (need) m = mx;
       const float mu = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
+      float rs8[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
 #pragma unroll
       for (int c = 0; c < TK / 64; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = fast_exp2(x[c * 64 + 2 * i] - mu);
-          const float p1 = fast_exp2(x[c * 64 + 2 * i + 1] - mu);
-          rs += p0 + p1;
+          // p = 2^(x * alpha * log2(e) - m): one FMA feeding the exponential
+          const float p0 = fast_exp2(fmaf(x[c * 64 + 2 * i], p.scale_log2, -mu));
+          const float p1 = fast_exp2(fmaf(x[c * 64 + 2 * i + 1], p.scale_log2, -mu));
+          rs8[(2 * i) & 7] += p0;
+          rs8[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_addr + c * 32, pk);  // P over the first TK/2 columns of S_t
       }
-      l += rs;
+      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p + t);
