@@ -255,6 +255,14 @@ int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, fl
 #define SINKATTN_KERNEL_DECODE 2
 int sinkattn_set_kernel_events(int which, void *start, void *stop);
 
+/* ---- failure-detection self-test ---------------------------------------------
+ * Launches a one-warp kernel that waits, through the same bounded barrier wait
+ * every kernel of this library uses, on a barrier nothing ever arrives at.  The
+ * wait gives up after its budget (about one second), records
+ * SINKATTN_ERR_TIMEOUT in the status word and the kernel returns normally, so
+ * the CUDA context stays usable.  Read the outcome with sinkattn_get_status. */
+int sinkattn_selftest_timeout(sinkattn_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------
  * sinkattn_get_status synchronises `stream`, then returns the first error code
  * any kernel of this library recorded on the current device since the last

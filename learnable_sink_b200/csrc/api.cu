@@ -323,6 +323,13 @@ int sinkattn_set_kernel_events(int which, void* start, void* stop) {
   return SINKATTN_OK;
 }
 
+int sinkattn_selftest_timeout(sinkattn_stream_t stream) {
+  if (!device_is_sm100()) return SINKATTN_ERR_UNSUPPORTED;
+  int* st = status_word();
+  if (!st) return SINKATTN_ERR_CUDA;
+  return launch_wait_selftest(st, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int sinkattn_get_status(sinkattn_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SINKATTN_ERR_CUDA;

@@ -177,18 +177,26 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeProblem
 }
 
 // Persistent streaming variant (bf16): one CTA per SM loops over work items
-// (sequence, KV head, split).  Warp 8 streams 64-row pieces of K and V with
-// TMA through an NSTG-stage ring that runs ahead across item boundaries, so
-// HBM stays busy while warps 0-7 compute.  A group of D/8 lanes holds one
-// row's 8-element slices; each group takes PR rows of a piece and reduces its
-// PR x G partial dot products with a butterfly that splits the values across
-// the group's lanes (log2 steps, each halving the values a lane keeps).
+// (sequence, KV head, split).  Warp 16 streams 64-row pieces of K and V with
+// TMA through a kStreamStages-deep ring that runs ahead across item
+// boundaries, so HBM stays busy while warps 0-15 compute.  A group of D/8
+// lanes holds one row's 8-element slices; each group takes PR rows of every
+// piece and keeps its own online-softmax state per head (running max, sum and
+// output slice), so groups never wait for each other inside an item; they
+// merge, max-rescaled, once per item.  Dot products of a group's PR x G
+// (row, head) pairs are reduced by a butterfly that splits the values across
+// the group's lanes.
 constexpr int kPieceRows = 64;
 constexpr int kStreamStages = 4;
-constexpr int kConsumerThreads = 256;
+// consumer threads: 16 warps, or 8 when eight query heads share a KV head
+// (their per-head state would not fit 16 warps' register budget)
+template <int G>
+constexpr int consumer_threads() { return G >= 8 ? 256 : 512; }
 
 template <int D, int G>
 struct StreamGeom {
+  static constexpr int kConsumerThreads = consumer_threads<G>();
+  static constexpr int kConsumerWarps = kConsumerThreads / 32;
   static constexpr int DH = D / 64;
   static constexpr int LPR = D / 8;                          // lanes per row
   static constexpr int NGRP = kConsumerThreads / LPR;        // row groups
@@ -197,9 +205,10 @@ struct StreamGeom {
   static constexpr int HALF_BYTES = kPieceRows * 128;        // one 64-column half of a piece
   static constexpr int PIECE_BYTES = DH * HALF_BYTES;        // K or V piece
   static constexpr int STAGE_BYTES = 2 * PIECE_BYTES;
-  static constexpr int OFF_SC = kStreamStages * STAGE_BYTES; // float [G][kPieceRows]
-  static constexpr int OFF_RED = OFF_SC + G * kPieceRows * 4;  // float [8 warps][G][D]
-  static constexpr int OFF_BAR = OFF_RED + 8 * G * D * 4;
+  static constexpr int OFF_SC = kStreamStages * STAGE_BYTES; // float [NGRP][V] group scratch
+  static constexpr int OFF_RED = OFF_SC + NGRP * V * 4;      // float [warps][G][D]
+  static constexpr int OFF_ML = OFF_RED + kConsumerWarps * G * D * 4;  // float [warps][G][2]
+  static constexpr int OFF_BAR = OFF_ML + kConsumerWarps * G * 2 * 4;
   // + 1024: the kernel rounds the dynamic shared-memory base up to 1024 bytes
   static constexpr int SMEM = OFF_BAR + 2 * kStreamStages * 8 + 1024;
   static constexpr int LOG_LPR = LPR == 16 ? 4 : 3;
@@ -210,7 +219,7 @@ struct StreamGeom {
 };
 
 // Sum each of the V values over the LPR lanes of a group; afterwards lane gl
-// holds KEEP totals, value index idx(gl, j) (see decode_value_index).
+// holds KEEP totals, value index decode_value_index(gl, j).
 template <int V, int LPR>
 __device__ __forceinline__ void butterfly_reduce(float (&v)[V], int gl) {
   int c = V;
@@ -244,18 +253,18 @@ __device__ __forceinline__ int decode_value_index(int gl, int j) {
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel(
+__global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     DecodeProblem p, int chunk, int n_items) {
   using Geo = StreamGeom<D, G>;
-  constexpr int LPR = Geo::LPR, NGRP = Geo::NGRP, PR = Geo::PR, V = Geo::V, DH = Geo::DH;
+  constexpr int LPR = Geo::LPR, PR = Geo::PR, V = Geo::V, DH = Geo::DH;
+  constexpr int kConsumerThreads = Geo::kConsumerThreads, kConsumerWarps = Geo::kConsumerWarps;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  float* sc = reinterpret_cast<float*>(sm + Geo::OFF_SC);
   float* red = reinterpret_cast<float*>(sm + Geo::OFF_RED);
+  float* ml = reinterpret_cast<float*>(sm + Geo::OFF_ML);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR);
   uint64_t* empty = full + kStreamStages;
-  __shared__ float m_s[G], l_s[G], f_s[G];
   __shared__ int abort_s;
   const int S = p.n_sink + p.window;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel
     n = max(min(split * chunk + chunk, n_valid) - split * chunk, 0);
   };
 
-  if (warp == kConsumerThreads / 32) {
+  if (warp == kConsumerWarps) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
       int pc = 0;
@@ -303,6 +312,7 @@ __global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel
   // ------------------------------------------------------------ consumers
   const int grp = tid / LPR, gl = tid % LPR;
   const int c0 = gl * 8, hf = c0 / 64, cin = c0 % 64;
+  float* scg = reinterpret_cast<float*>(sm + Geo::OFF_SC) + grp * V;  // group scratch
   const float scale_log2 = p.scale * kLog2e;
   int pc = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
@@ -316,20 +326,21 @@ __global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel
 #pragma unroll
       for (int c = 0; c < 8; ++c) qv[h][c] *= scale_log2;
     }
-    float acc[G][8];
+    float acc[G][8], m_run[G], l_run[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h) {
+      m_run[h] = -INFINITY;
+      l_run[h] = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
-    if (tid < G) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
-    named_bar_sync(1, kConsumerThreads);
+    }
     for (int r0 = 0; r0 < n; r0 += kPieceRows, ++pc) {
       const int st = pc % kStreamStages;
       const int rows = min(kPieceRows, n - r0);
       if (!mbar_wait(full + st, (pc / kStreamStages) & 1, &abort_s, p.status)) return;
       const uint8_t* kbuf = sm + st * Geo::STAGE_BYTES;
       const uint8_t* vbuf = kbuf + Geo::PIECE_BYTES;
-      // scores: this group's PR rows, all G heads
+      // scores of this group's PR rows for all G heads
       float v[V];
 #pragma unroll
       for (int rr = 0; rr < PR; ++rr) {
@@ -348,39 +359,37 @@ __global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel
 #pragma unroll
       for (int j = 0; j < Geo::KEEP; ++j) {
         const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
-        const int rr = idx / G, h = idx % G, r = grp * PR + rr;
-        if (r < rows) sc[h * kPieceRows + r] = v[j];
+        scg[idx] = (grp * PR + idx / G < rows) ? v[j] : -INFINITY;
       }
-      named_bar_sync(1, kConsumerThreads);
-      // online softmax over this piece (warp h handles head h)
-      for (int h = warp; h < G; h += kConsumerThreads / 32) {
-        float m = -INFINITY;
-        for (int i = lane; i < rows; i += 32) m = fmaxf(m, sc[h * kPieceRows + i]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const float mo = m_s[h];
-        const float mn = fmaxf(mo, m);
-        float l = 0.f;
-        for (int i = lane; i < rows; i += 32) {
-          const float e = exp2f(sc[h * kPieceRows + i] - mn);
-          sc[h * kPieceRows + i] = e;
-          l += e;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (lane == 0) {
-          const float f = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-          f_s[h] = f;
-          l_s[h] = l_s[h] * f + l;
-          m_s[h] = mn;
-        }
-      }
-      named_bar_sync(1, kConsumerThreads);
+      __syncwarp();
+      // per-head maximum over the group's rows, new running max, rescale
+      float mnew[G], corr[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float f = f_s[h];
+        float mx = m_run[h];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[h][c] *= f;
+        for (int rr = 0; rr < PR; ++rr) mx = fmaxf(mx, scg[rr * G + h]);
+        mnew[h] = mx;
+        corr[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mx);
+      }
+      __syncwarp();  // every lane has read the scores before they become probabilities
+#pragma unroll
+      for (int j = 0; j < Geo::KEEP; ++j) {
+        const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
+        const int h = idx % G;
+        const float sv = (grp * PR + idx / G < rows) ? v[j] : -INFINITY;
+        scg[idx] = (mnew[h] == -INFINITY) ? 0.f : exp2f(sv - mnew[h]);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float ps = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < PR; ++rr) ps += scg[rr * G + h];
+        l_run[h] = l_run[h] * corr[h] + ps;
+        m_run[h] = mnew[h];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[h][c] *= corr[h];
       }
 #pragma unroll
       for (int rr = 0; rr < PR; ++rr) {
@@ -390,46 +399,71 @@ __global__ void __launch_bounds__(kConsumerThreads + 32, 1) decode_stream_kernel
           bf16x8_to_f32(*reinterpret_cast<const uint4*>(vbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), vf);
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float pr = sc[h * kPieceRows + r];
+            const float pr = scg[rr * G + h];
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[h][c] += pr * vf[c];
           }
         }
       }
-      mbar_arrive(empty + st);            // the stage may be refilled
-      named_bar_sync(1, kConsumerThreads);  // sc may be overwritten
+      __syncwarp();  // scratch reads done before the next piece's writes
+      mbar_arrive(empty + st);  // this thread is done with the stage
     }
-    // reduce the groups: lanes with equal gl in the two halves of a warp,
-    // then the eight warps through shared memory (fixed order)
+    // merge the groups of a warp (lanes gl and gl + LPR, ...) with max rescaling
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int o = 16; o >= LPR; o >>= 1) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float x = acc[h][c];
-        for (int o = 16; o >= LPR; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        acc[h][c] = x;
+      for (int h = 0; h < G; ++h) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m_run[h], o);
+        const float lo = __shfl_xor_sync(0xffffffffu, l_run[h], o);
+        const float mm = fmaxf(m_run[h], mo);
+        const float fa = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mm);
+        const float fb = (mo == -INFINITY) ? 0.f : exp2f(mo - mm);
+        l_run[h] = l_run[h] * fa + lo * fb;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float ao = __shfl_xor_sync(0xffffffffu, acc[h][c], o);
+          acc[h][c] = acc[h][c] * fa + ao * fb;
+        }
+        m_run[h] = mm;
       }
+    }
     if (lane < LPR) {
 #pragma unroll
-      for (int h = 0; h < G; ++h)
+      for (int h = 0; h < G; ++h) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) red[(warp * G + h) * D + c0 + c] = acc[h][c];
+        if (gl == 0) {
+          ml[(warp * G + h) * 2] = m_run[h];
+          ml[(warp * G + h) * 2 + 1] = l_run[h];
+        }
+      }
     }
     named_bar_sync(1, kConsumerThreads);
+    // merge the warps (fixed order) and write the split's partial
     float* part = p.part + (((long long)b * p.Hq + kvh * G) * p.num_splits + split) * (D + 2);
     for (int i = tid; i < G * D; i += kConsumerThreads) {
       const int h = i / D, d = i % D;
-      float s = 0.f;
+      float mm = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kConsumerThreads / 32; ++w) s += red[(w * G + h) * D + d];
-      part[(long long)h * p.num_splits * (D + 2) + d] = s;
+      for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, ml[(w * G + h) * 2]);
+      float sacc = 0.f, sl = 0.f;
+      if (mm != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = ml[(w * G + h) * 2];
+          if (mw == -INFINITY) continue;
+          const float f = exp2f(mw - mm);
+          sacc += red[(w * G + h) * D + d] * f;
+          sl += ml[(w * G + h) * 2 + 1] * f;
+        }
+      }
+      part[(long long)h * p.num_splits * (D + 2) + d] = sacc;
+      if (d == 0) {
+        part[(long long)h * p.num_splits * (D + 2) + D] = n > 0 ? mm : -INFINITY;
+        part[(long long)h * p.num_splits * (D + 2) + D + 1] = n > 0 ? sl : 0.f;
+      }
     }
-    if (tid < G) {
-      float* ph = part + (long long)tid * p.num_splits * (D + 2);
-      ph[D] = n > 0 ? m_s[tid] : -INFINITY;
-      ph[D + 1] = n > 0 ? l_s[tid] : 0.f;
-    }
-    named_bar_sync(1, kConsumerThreads);  // red / m_s reused by the next item
+    named_bar_sync(1, kConsumerThreads);  // red / ml reused by the next item
   }
 }
 
@@ -482,7 +516,7 @@ int launch_tma(const DecodeProblem& p, int chunk, cudaStream_t stream) {
   const int n_items = p.B * p.Hkv * p.num_splits;
   const int grid = n_items < sms ? n_items : sms;
   record_start(SINKATTN_KERNEL_DECODE, stream);
-  kern<<<grid, kConsumerThreads + 32, Geo::SMEM, stream>>>(mk, mv, p, chunk, n_items);
+  kern<<<grid, Geo::kConsumerThreads + 32, Geo::SMEM, stream>>>(mk, mv, p, chunk, n_items);
   record_stop(SINKATTN_KERNEL_DECODE, stream);
   dim3 g2(p.Hq, p.B);
   decode_combine_kernel<__nv_bfloat16, D><<<g2, D, 0, stream>>>(p, p.num_splits);

@@ -101,4 +101,7 @@ struct DecodeProblem {
 };
 int launch_decode(const DecodeProblem& p, cudaStream_t stream);
 
+// failure-detection self-test: a bounded wait on a barrier nobody arrives at
+int launch_wait_selftest(int* status, cudaStream_t stream);
+
 }  // namespace sk

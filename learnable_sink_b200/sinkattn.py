@@ -71,6 +71,7 @@ def lib():
         L.sinkattn_decode.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _i, _i,
                                       _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
         L.sinkattn_set_kernel_events.argtypes = [_i, _vp, _vp]
+        L.sinkattn_selftest_timeout.argtypes = [_vp]
         L.sinkattn_get_status.argtypes = [_vp]
         L.sinkattn_clear_status.argtypes = [_vp]
         L.sinkattn_error_string.restype = _c.c_char_p
@@ -254,6 +255,11 @@ def set_kernel_events(which: int, start=None, stop=None) -> None:
     sp = None if start is None else _vp(start.cuda_event)
     ep = None if stop is None else _vp(stop.cuda_event)
     _check("sinkattn_set_kernel_events", lib().sinkattn_set_kernel_events(int(which), sp, ep))
+
+
+def selftest_timeout(stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see include/sinkattn.h)."""
+    _check("sinkattn_selftest_timeout", lib().sinkattn_selftest_timeout(_stream(stream)))
 
 
 def get_status(stream=None) -> int:
