@@ -9,56 +9,88 @@
 // (section 7) and is not touched here.  Section 10 describes a backward split
 // by KV block over reverse lists; this kernel is that split.
 //
-// One CTA = one 128-key tile of one KV head (the plan's reverse list gives
-// the query tiles that see it); it loops over (query tile, query head) pairs.
+// One CTA = one key tile of one KV head (a slice of the plan's reverse list
+// gives the query tiles that see it); it loops over (query sub-tile, query
+// head) pairs of QR = QT tokens x HPT heads = 64 or 128 query rows.
 // Tensor memory (512 columns):
-//   S^T  [keys x 128 query rows] fp32, overwritten in place by P^T (bf16,
-//        packed two per column at the front of each warpgroup's slice)
-//   dP^T [keys x 128] fp32, overwritten by dS^T (bf16, same packing); then reused for the
-//        dQ tile [128 query rows x D] once dK has consumed dS^T
+//   S^T  [keys x QR] fp32, overwritten in place by P^T (bf16, packed two per
+//        column at the front of each compute warpgroup's slice)
+//   dP^T [keys x QR] fp32, overwritten by dS^T (bf16, same packing)
 //   dK, dV [keys x D] fp32 accumulators for the whole CTA
-// MMAs per (query tile, head), issued by one thread in this order:
-//   S^T = K Q^T (SS) | dP^T = V dO^T (SS) | dV += P^T dO (TS) |
-//   dK += dS^T Q (TS) | dQ = dS K (SS; dS^T also staged in shared memory)
-// Warps 0-7 compute (warpgroup c owns query columns [64c, 64c + 64), thread =
-// key row), warp 8 is the TMA producer, warp 9 issues MMAs, warp 10 flushes
-// dQ.  The compute warps move each dQ tile out of tensor memory into the
-// finished stage's shared memory; the reducer adds it into an fp32 buffer with
-// bulk tensor reductions (a query row gets one contribution per visible key
-// tile); a small kernel converts it to bf16.
+//   dQ   [QR x D] fp32 in its own columns when they fit, else over dP^T once
+//        dK has consumed dS^T
+// MMAs of iteration i, issued by one thread:
+//   dV += P^T dO (TS) | S^T(i+1) = K Q^T (SS) | dK += dS^T Q (TS) |
+//   dQ = dS K (SS; dS^T also staged in shared memory) | dP^T(i+1) = V dO^T (SS)
+// so the tensor cores run dK/dQ of tile i while the compute warps
+// exponentiate tile i+1 (S^T(i+1) moves behind dQ(i) when its Q tile has not
+// landed yet).  Warps 0-7 compute (warpgroup c owns query columns
+// [c QR/2, (c + 1) QR/2), thread = key row); warps 8-11 move each dQ tile out
+// of tensor memory into the finished stage's shared memory; warp 12 is the TMA
+// producer, warp 13 issues MMAs and warp 14 adds the staged dQ tiles into an
+// fp32 buffer with bulk tensor reductions (a query row gets one contribution
+// per visible key tile); a small kernel converts it to bf16.
+//
+// Two limits shape the schedule: the tensor cores read shared-memory operands
+// at about 128 bytes per cycle (a 128 x 128 x 16 SS MMA is already at that
+// rate, so every other shared-memory byte slows the MMAs), and an SM drains
+// about 20 bytes of dQ reductions per cycle, so a stage stays busy until its
+// fp32 dQ tile has left.  With 128-key tiles the query side uses 128 rows per
+// iteration: 64-row sub-tiles (supported by the template) halve the stage but
+// re-read K and V twice as often, which costs more shared-memory bandwidth
+// than the extra stages save.
 #include "internal.h"
 
 namespace sk {
 
 namespace {
 
-// KT = 128: 128-key tiles, query tiles of 128 tokens x 1 head.
-// KT = 64 (64-key block selection): M = 64 for the key-side MMAs (tensor-memory
-// rows m at lanes m % 16 + 32 (m / 16)), query tiles of 64 tokens x 2 heads so
-// the dQ MMA keeps M = 128.
-template <int D_, int KT_>
+// KT = key-tile tokens (the plan's tile), QT x HPT = query rows per iteration.
+//   <D, 128, 128, 1>: 128-key tiles, query tiles of 128 tokens x 1 head.
+//   <D, 128, 64, 1>:  the same with 64-token sub-tiles; the dQ MMA then has
+//                     M = 64 (tensor-memory rows m at lanes m % 16 + 32 (m / 16)).
+//   <D, 64, 64, 2>:   64-key block selection: M = 64 for the key-side MMAs
+//                     (same lane layout), query tiles of 64 tokens x 2 heads
+//                     so the dQ MMA keeps M = 128.
+template <int D_, int KT_, int QT_, int HPT_>
 struct BwdCfg {
-  static constexpr int D = D_, KT = KT_, TQ = KT_, HPT = 128 / KT_;
+  static constexpr int D = D_, KT = KT_, QT = QT_, HPT = HPT_;
+  static constexpr int QR = QT * HPT;           // query rows per iteration
+  static constexpr int NSUB = KT / QT;          // sub-tiles per plan tile
+  static constexpr int CW = QR / 2;             // query columns per compute warpgroup
   static constexpr int DH = D / 64;
-  static constexpr int Q_BYTES = 128 * D * 2;   // Q or dO tile (128 rows)
+  static_assert(QR == 64 || QR == 128, "query rows");
+  static constexpr int Q_BYTES = QR * D * 2;    // Q or dO tile
   static constexpr int KV_BYTES = KT * D * 2;   // K or V tile
-  static constexpr int DS_BYTES = KT * 128 * 2; // dS^T tile
+  static constexpr int DS_BYTES = KT * QR * 2;  // dS^T tile
   static constexpr int SMEM_LIMIT = 227 * 1024;
   static constexpr int FIXED = 2 * KV_BYTES + DS_BYTES + 1024 /*lse, delta*/ + 512 /*bars*/ + 1024;
   static constexpr int NS_RAW = (SMEM_LIMIT - FIXED) / (2 * Q_BYTES);
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "shared memory");
-  static constexpr int THREADS = 11 * 32;
-  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, REDUCER_WARP = 10;
-  static constexpr int S_COL = 0, DP_COL = 128, DK_COL = 256, DV_COL = 256 + D;
+  static constexpr int THREADS = 16 * 32;
+  static constexpr int EPI_WARP0 = 8, PRODUCER_WARP = 12, MMA_WARP = 13, REDUCER_WARP = 14;
+  // 2 compute warpgroups, 1 dQ-epilogue warpgroup, 1 warpgroup of single-warp
+  // roles.  With 128 query rows a compute thread holds 64 probabilities and
+  // registers move to the compute warpgroups; with 64 the launch split fits.
+  static constexpr int LAUNCH_REGS = 65536 / THREADS;
+  static constexpr bool REBALANCE = QR == 128;
+  static constexpr int COMPUTE_REGS = REBALANCE ? 184 : LAUNCH_REGS;
+  static constexpr int EPI_REGS = REBALANCE ? 72 : LAUNCH_REGS;
+  static constexpr int AUX_REGS = REBALANCE ? 72 : LAUNCH_REGS;
+  static_assert(256 * COMPUTE_REGS + 128 * EPI_REGS + 128 * AUX_REGS <= 65536,
+                "register split exceeds the block's allocation");
+  static constexpr int S_COL = 0, DP_COL = QR, DK_COL = 2 * QR, DV_COL = 2 * QR + D;
+  static constexpr bool DQ_OWN = 2 * QR + 3 * D <= 512;   // dQ in columns of its own
+  static constexpr int DQ_COL = DQ_OWN ? 2 * QR + 2 * D : DP_COL;
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
   static constexpr int OFF_DS = OFF_V + KV_BYTES;
   static constexpr int OFF_Q = OFF_DS + DS_BYTES;
   static constexpr int OFF_DO = OFF_Q + NS * Q_BYTES;
-  static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[128]
-  static constexpr int OFF_DL = OFF_LSE + 512;            // float[128]
+  static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[QR]
+  static constexpr int OFF_DL = OFF_LSE + 512;            // float[QR]
   static constexpr int OFF_BAR = OFF_DL + 512;
   static constexpr int N_BARS = 1 + 3 * NS + 7;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
@@ -71,7 +103,6 @@ struct BwdParams {
   const int* plan;
   const float* lse2;   // [Hq, T] head-major, log2 domain
   const float* delta;  // [Hq, T]
-  float* dq_accum;     // [T, Hq, D] fp32
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int* status;
@@ -86,11 +117,15 @@ __device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// Packed bf16 P^T / dS^T columns: warpgroup c writes its 64 query columns
-// as 32 packed words at the front of its own fp32 slice [64c, 64c + 64), so
-// it never overwrites fp32 values the other warpgroup has yet to read.  K step
-// kk (16 query columns) of the TS-MMA A operand therefore starts at:
-__device__ __forceinline__ constexpr uint32_t a_col(int kk) { return (kk / 4) * 64 + (kk % 4) * 8; }
+// Packed bf16 P^T / dS^T columns: compute warpgroup c writes its CW query
+// columns as CW/2 packed words at the front of its own fp32 slice
+// [c CW, c CW + CW), so it never overwrites fp32 values the other warpgroup
+// has yet to read.  K step kk (16 query columns) of the TS-MMA A operand
+// therefore starts at:
+template <int CW>
+__device__ __forceinline__ constexpr uint32_t a_col(int kk) {
+  return (kk / (CW / 16)) * CW + (kk % (CW / 16)) * 8;
+}
 
 // fp32 add of a shared-memory box into global memory through the tensor map
 // (bulk reduction; rows past the tensor's extent are skipped by the hardware)
@@ -120,7 +155,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                   const __grid_constant__ CUtensorMap tmap_dq,
                   const __grid_constant__ CUtensorMap tmap_dkacc,
                   const __grid_constant__ CUtensorMap tmap_dvacc, const BwdParams p) {
-  constexpr int D = C::D, KT = C::KT, TQ = C::TQ, HPT = C::HPT, NS = C::NS, DH = C::DH;
+  constexpr int D = C::D, KT = C::KT, QT = C::QT, HPT = C::HPT, QR = C::QR, CW = C::CW;
+  constexpr int NS = C::NS, DH = C::DH, NSUB = C::NSUB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -151,8 +187,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const bool split_tile = unit.w > 1;  // partial dK/dV go through fp32 reductions
   const int kvh = it.kvh >= 0 ? it.kvh : rem;
   const int* ent = p.plan + hdr->off_bwd_entries + it.entry_off + unit.y;
-  const int GH = p.G / HPT;             // query-head groups per key tile
-  const int n_it = unit.z * GH;         // (query tile, head group) iterations
+  // iteration i: entry i / PER_E, head group (i % PER_E) / NSUB, sub-tile i % NSUB
+  const int GH = p.G / HPT;
+  const int PER_E = GH * NSUB;
+  const int n_it = unit.z * PER_E;
   const int k0 = it.tile_start;         // sequence-local first key
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,14 +199,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_qf + s, 1);
       mbar_init(bar_qe + s, 1);    // released by the reducer warp
-      mbar_init(bar_dqs + s, 256); // every compute thread staged its dQ part
+      mbar_init(bar_dqs + s, 128); // every epilogue thread staged its dQ part
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
     mbar_init(bar_p, 256);
     mbar_init(bar_ds, 256);
     mbar_init(bar_dq, 1);
-    mbar_init(bar_dqf, 256);
+    mbar_init(bar_dqf, 128);
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -189,137 +227,221 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == C::PRODUCER_WARP) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && n_it > 0) {
-      const int krow = it.seq_start + k0;
-      mbar_expect_tx(bar_kv, 2 * C::KV_BYTES);
-      for (int h = 0; h < DH; ++h) {
-        tma_load_3d(smem + C::OFF_K + h * (C::KV_BYTES / DH), &tmap_k, bar_kv, h * 64, kvh, krow);
-        tma_load_3d(smem + C::OFF_V + h * (C::KV_BYTES / DH), &tmap_v, bar_kv, h * 64, kvh, krow);
-      }
-      int last[NS];
-      for (int s = 0; s < NS; ++s) last[s] = -1;
-      bool ok = true;
-      for (int i = 0; i < n_it && ok; ++i) {
-        const int s = i % NS;
-        const int e = __ldg(ent + i / GH);
-        const int q_tok = it.seq_start + (e >> 1) * TQ;
-        const int h0 = kvh * p.G + (i % GH) * HPT;
-        ok = mbar_wait(bar_qe + s, ((i / NS) & 1) ^ 1, abort_flag, p.status);
-        if (!ok) break;
-        mbar_expect_tx(bar_qf + s, 2 * C::Q_BYTES);
+  // sequence-local first query token and first query head of iteration i
+  // (entry e of the reverse list)
+  auto q_first = [&](int i, int e) { return (e >> 1) * KT + (i % NSUB) * QT; };
+  auto h_first = [&](int i) { return kvh * p.G + ((i % PER_E) / NSUB) * HPT; };
+
+  if (warp >= C::PRODUCER_WARP) {
+    regs_to<C::AUX_REGS, C::LAUNCH_REGS>();
+    if (warp == C::PRODUCER_WARP) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0 && n_it > 0) {
+        const int krow = it.seq_start + k0;
+        mbar_expect_tx(bar_kv, 2 * C::KV_BYTES);
         for (int h = 0; h < DH; ++h) {
-          tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_q,
-                      bar_qf + s, h * 64, h0, q_tok);
-          tma_load_3d(smem + C::OFF_DO + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_do,
-                      bar_qf + s, h * 64, h0, q_tok);
+          tma_load_3d(smem + C::OFF_K + h * (C::KV_BYTES / DH), &tmap_k, bar_kv, h * 64, kvh, krow);
+          tma_load_3d(smem + C::OFF_V + h * (C::KV_BYTES / DH), &tmap_v, bar_kv, h * 64, kvh, krow);
         }
-        last[s] = i;
+        int last[NS];
+        for (int s = 0; s < NS; ++s) last[s] = -1;
+        bool ok = true;
+        for (int i = 0; i < n_it && ok; ++i) {
+          const int s = i % NS;
+          const int e = __ldg(ent + i / PER_E);
+          const int q_tok = it.seq_start + q_first(i, e);
+          const int h0 = h_first(i);
+          ok = mbar_wait(bar_qe + s, ((i / NS) & 1) ^ 1, abort_flag, p.status);
+          if (!ok) break;
+          mbar_expect_tx(bar_qf + s, 2 * C::Q_BYTES);
+          for (int h = 0; h < DH; ++h) {
+            tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_q,
+                        bar_qf + s, h * 64, h0, q_tok);
+            tma_load_3d(smem + C::OFF_DO + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_do,
+                        bar_qf + s, h * 64, h0, q_tok);
+          }
+          last[s] = i;
+        }
+        if (!ok) {
+          wait_noabort(bar_kv, 0);
+          for (int s = 0; s < NS; ++s)
+            if (last[s] >= 0) wait_noabort(bar_qf + s, (last[s] / NS) & 1);
+        }
       }
-      if (!ok) {
-        wait_noabort(bar_kv, 0);
-        for (int s = 0; s < NS; ++s)
-          if (last[s] >= 0) wait_noabort(bar_qf + s, (last[s] / NS) & 1);
-      }
-    }
-  } else if (warp == C::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_it > 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(KT, 128, 0, 0);   // S^T, dP^T
-      constexpr uint32_t id_kv = idesc_bf16_f32(KT, D, 0, 1);    // dV, dK (B MN-major)
-      constexpr uint32_t id_q = idesc_bf16_f32(128, D, 1, 1);    // dQ (A, B MN-major)
-      const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V),
-                     sDS = smem_u32(smem + C::OFF_DS), sQ = smem_u32(smem + C::OFF_Q),
-                     sDO = smem_u32(smem + C::OFF_DO);
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status);
-      for (int i = 0; i < n_it && ok; ++i) {
-        const int s = i % NS;
-        ok = mbar_wait(bar_qf + s, (i / NS) & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t q_s = sQ + s * C::Q_BYTES, do_s = sDO + s * C::Q_BYTES;
-        // S^T = K Q^T (both K-major)
+    } else if (warp == C::MMA_WARP) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0 && n_it > 0) {
+        constexpr uint32_t id_s = idesc_bf16_f32(KT, QR, 0, 0);  // S^T, dP^T
+        constexpr uint32_t id_kv = idesc_bf16_f32(KT, D, 0, 1);  // dV, dK (B MN-major)
+        constexpr uint32_t id_q = idesc_bf16_f32(QR, D, 1, 1);   // dQ (A, B MN-major)
+        const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V),
+                       sDS = smem_u32(smem + C::OFF_DS), sQ = smem_u32(smem + C::OFF_Q),
+                       sDO = smem_u32(smem + C::OFF_DO);
+        // S^T = K Q^T (both K-major) of iteration j; its Q/dO stage has landed
+        auto issue_s = [&](int j) {
+          const uint32_t q_s = sQ + (j % NS) * C::Q_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          mma_ss(tmem + C::S_COL,
-                 sdesc_sw128(sK + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
-                 sdesc_sw128(q_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            mma_ss(tmem + C::S_COL,
+                   sdesc_sw128(sK + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
+                   sdesc_sw128(q_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_s);
+        };
+        // dP^T = V dO^T of iteration j
+        auto issue_dp = [&](int j) {
+          const uint32_t do_s = sDO + (j % NS) * C::Q_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            mma_ss(tmem + C::DP_COL,
+                   sdesc_sw128(sV + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
+                   sdesc_sw128(do_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_dp);
+        };
+        bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status) &&
+                  mbar_wait(bar_qf, 0, abort_flag, p.status);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          issue_dp(0);
         }
-        mma_commit(bar_s);
-        // dP^T = V dO^T, into the columns the previous dQ tile occupied
-        if (i > 0) {
-          ok = mbar_wait(bar_dqf, (i - 1) & 1, abort_flag, p.status);
+        for (int i = 0; i < n_it && ok; ++i) {
+          const int s = i % NS;
+          const uint32_t q_s = sQ + s * C::Q_BYTES, do_s = sDO + s * C::Q_BYTES;
+          const bool more = i + 1 < n_it;
+          const int s1 = (i + 1) % NS;
+          const uint32_t par1 = ((i + 1) / NS) & 1;
+          // dV += P^T dO  (P^T bf16 in tensor memory over S^T; dO MN-major)
+          ok = mbar_wait(bar_p, i & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < QR / 16; ++kk)
+            mma_ts(tmem + C::DV_COL, tmem + C::S_COL + a_col<CW>(kk),
+                   sdesc_sw128(do_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          // S^T of the next iteration right behind dV (which frees the S^T
+          // columns), if its tiles are already in shared memory
+          bool s_next = false;
+          if (more && mbar_try_wait(bar_qf + s1, par1)) {
+            tc_fence_after();
+            issue_s(i + 1);
+            s_next = true;
+          }
+          // dK += dS^T Q  (dS^T bf16 in tensor memory over dP^T)
+          ok = mbar_wait(bar_ds, i & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < QR / 16; ++kk)
+            mma_ts(tmem + C::DK_COL, tmem + C::DP_COL + a_col<CW>(kk),
+                   sdesc_sw128(q_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
+                   (i > 0 || kk > 0) ? 1u : 0u);
+          // dQ = dS K  (A = dS from the staged dS^T tile, both MN-major); in
+          // columns of its own it waits until the previous tile was read out
+          if (C::DQ_OWN && i > 0) {
+            ok = mbar_wait(bar_dqf, (i - 1) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < KT / 16; ++kk)
+            mma_ss(tmem + C::DQ_COL, sdesc_sw128(sDS + kk * 2048, KT * 128, 1024),
+                   sdesc_sw128(sK + kk * 2048, C::KV_BYTES / DH, 1024), id_q, kk > 0 ? 1u : 0u);
+          mma_commit(bar_dq);  // the stage is released once its dQ tile has been flushed
+          if (more) {
+            if (!s_next) {
+              ok = mbar_wait(bar_qf + s1, par1, abort_flag, p.status);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(i + 1);
+            }
+            if (!C::DQ_OWN) {  // dP^T(i+1) overwrites the dQ tile
+              ok = mbar_wait(bar_dqf, i & 1, abort_flag, p.status);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_dp(i + 1);
+          }
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          mma_ss(tmem + C::DP_COL,
-                 sdesc_sw128(sV + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
-                 sdesc_sw128(do_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar_dp);
-        // dV += P^T dO  (P^T bf16 in tensor memory over S^T; dO MN-major)
-        ok = mbar_wait(bar_p, i & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::DV_COL, tmem + C::S_COL + a_col(kk),
-                 sdesc_sw128(do_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q  (dS^T bf16 in tensor memory over dP^T)
-        ok = mbar_wait(bar_ds, i & 1, abort_flag, p.status);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::DK_COL, tmem + C::DP_COL + a_col(kk),
-                 sdesc_sw128(q_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
-                 (i > 0 || kk > 0) ? 1u : 0u);
-        // dQ = dS K  (A = dS from the staged dS^T tile, both MN-major)
-#pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk)
-          mma_ss(tmem + C::DP_COL, sdesc_sw128(sDS + kk * 2048, KT * 128, 1024),
-                 sdesc_sw128(sK + kk * 2048, C::KV_BYTES / DH, 1024), id_q, kk > 0 ? 1u : 0u);
-        mma_commit(bar_dq);  // stage s is released once its dQ tile has been flushed
+        mma_commit(bar_fin);
+        wait_noabort(bar_fin, 0);
       }
-      mma_commit(bar_fin);
-      wait_noabort(bar_fin, 0);
-    }
-  } else if (warp == C::REDUCER_WARP) {
-    // ------------------------------------------------------------ dQ reducer
-    // Adds each staged fp32 dQ tile into the global accumulator with bulk
-    // tensor reductions, waits until they have read the stage, and hands the
-    // stage back to the producer; the compute warps never wait for this.
-    if (lane == 0 && n_it > 0) {
-      for (int i = 0; i < n_it; ++i) {
-        const int s = i % NS;
-        if (!mbar_wait(bar_dqs + s, (i / NS) & 1, abort_flag, p.status)) break;
-        const int e = __ldg(ent + i / GH);
-        const int q_tok = it.seq_start + (e >> 1) * TQ;
-        const int h0 = kvh * p.G + (i % GH) * HPT;
+    } else if (warp == C::REDUCER_WARP) {
+      // ---------------------------------------------------------- dQ reducer
+      // Adds each staged fp32 dQ tile into the global accumulator with bulk
+      // tensor reductions, waits until they have read the stage, and hands
+      // the stage back to the producer; no other warp waits for this.
+      if (lane == 0 && n_it > 0) {
+        for (int i = 0; i < n_it; ++i) {
+          const int s = i % NS;
+          if (!mbar_wait(bar_dqs + s, (i / NS) & 1, abort_flag, p.status)) break;
+          const int e = __ldg(ent + i / PER_E);
+          const int q_tok = it.seq_start + q_first(i, e);
+          const int h0 = h_first(i);
 #pragma unroll
-        for (int cw = 0; cw < 2; ++cw) {
-          const uint8_t* stage = smem + (cw == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
+          for (int half = 0; half < 2; ++half) {
+            const uint8_t* stage = smem + (half == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_reduce_add_3d(&tmap_dq, stage + c * (128 * 128), (D / 2) * cw + 32 * c, h0, q_tok);
+            for (int c = 0; c < D / 64; ++c)
+              tma_reduce_add_3d(&tmap_dq, stage + c * (QR * 128), (D / 2) * half + 32 * c, h0,
+                                q_tok);
+          }
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(bar_qe + s);
         }
-        bulk_commit();
-        bulk_wait_read0();
-        mbar_arrive(bar_qe + s);
+        bulk_wait0();  // reductions complete before the CTA exits
       }
-      bulk_wait0();  // reductions complete before the CTA exits
+    }  // warp 15: idle
+  } else if (warp >= C::EPI_WARP0) {
+    // ------------------------------------------------------------ dQ epilogue
+    // Query row m of the dQ tile sits at lane m (QR = 128) or at lane
+    // m % 16 + 32 (m / 16) (QR = 64).  All MMAs of the iteration are complete,
+    // so the stage's Q buffer takes columns [0, D/2) and its dO buffer columns
+    // [D/2, D), as fp32 boxes of 32 columns with the 128-byte swizzle.  Query
+    // rows past the sequence end carry exact zeros (their P is 0), so adding
+    // them is harmless.
+    regs_to<C::EPI_REGS, C::LAUNCH_REGS>();
+    const int wq = warp % 4;
+    const bool lane_ok = QR == 128 || lane < 16;
+    const int qrow = QR == 128 ? wq * 32 + lane : wq * 16 + (lane & 15);
+    const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    for (int i = 0; i < n_it; ++i) {
+      const int s = i % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, p.status))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c32 = 0; c32 < D / 32; ++c32) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + C::DQ_COL + 32 * c32, a);
+        tmem_ld_wait();
+        if (c32 == D / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(bar_dqf);  // the dQ columns may be overwritten
+        }
+        const int half = c32 / (D / 64), c = c32 % (D / 64);
+        uint8_t* row = smem + (half == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES +
+                       c * (QR * 128) + qrow * 128;
+        if (lane_ok) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
+                make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(bar_dqs + s);  // the reducer warp takes it from here
     }
   } else {
     // ------------------------------------------------------------ compute
-    const int cw = warp / 4;          // query-column half
+    regs_to<C::COMPUTE_REGS, C::LAUNCH_REGS>();
+    const int cw = warp / 4;          // query-column block
     const int wq = warp % 4;          // TMEM lane quadrant
     const int tw = wq * 32 + lane;    // 0..127 within the warpgroup
     // key row held by this thread's TMEM lane (with KT = 64 only lanes 0-15
@@ -328,22 +450,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const bool row_ok = KT == 128 || lane < 16;
     const int kj = k0 + r;            // sequence-local key
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const float* lse_s = s_lse + 64 * cw;
-    const float* dl_s = s_dl + 64 * cw;
-    // The next iteration's entry and (for 64 of the threads) its LSE2 / Delta
+    const float* lse_s = s_lse + CW * cw;
+    const float* dl_s = s_dl + CW * cw;
+    // The next iteration's entry and (for CW of the threads) its LSE2 / Delta
     // values are loaded one iteration ahead, so global-load latency stays off
     // the critical path.
     auto fetch = [&](int i, int& e, float& l2, float& dl) {
-      e = __ldg(ent + i / GH);
+      e = __ldg(ent + i / PER_E);
       l2 = INFINITY;
       dl = 0.f;
-      if (tw < 64) {
-        const int q0 = (e >> 1) * TQ;
-        const int col = 64 * cw + tw;
+      if (tw < CW) {
+        const int q0 = q_first(i, e);
+        const int col = CW * cw + tw;
         const int tok = col / HPT, hh = col % HPT;
-        const int h0 = kvh * p.G + (i % GH) * HPT;
         if (tok < it.seq_len - q0) {
-          const long long gi = (long long)(h0 + hh) * p.T_tot + it.seq_start + q0 + tok;
+          const long long gi = (long long)(h_first(i) + hh) * p.T_tot + it.seq_start + q0 + tok;
           l2 = __ldg(p.lse2 + gi);
           dl = __ldg(p.delta + gi);
         }
@@ -355,14 +476,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     bool ok = true;
     for (int i = 0; i < n_it; ++i) {
       const int e = e_nx;
-      const int q0 = (e >> 1) * TQ;
+      const int q0 = q_first(i, e);
       const bool partial = (e & 1) != 0;
-      const int h0 = kvh * p.G + (i % GH) * HPT;
-      const int q_len = min(TQ, it.seq_len - q0);
       named_bar_sync(1 + cw, 128);  // previous iteration's smem reads are done
-      if (tw < 64) {
-        s_lse[64 * cw + tw] = l2_nx;
-        s_dl[64 * cw + tw] = dl_nx;
+      if (tw < CW) {
+        s_lse[CW * cw + tw] = l2_nx;
+        s_dl[CW * cw + tw] = dl_nx;
       }
       named_bar_sync(1 + cw, 128);
       if (i + 1 < n_it) fetch(i + 1, e_nx, l2_nx, dl_nx);
@@ -370,11 +489,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s, i & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      float P[64];
+      float P[CW];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < CW / 32; ++h2) {
         uint32_t a[32];
-        tmem_ld32(tmem + lane_off + C::S_COL + 64 * cw + 32 * h2, a);
+        tmem_ld32(tmem + lane_off + C::S_COL + CW * cw + 32 * h2, a);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 32; ++c)
@@ -382,16 +501,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       if (partial) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int tok = (64 * cw + c) / HPT;
+        for (int c = 0; c < CW; ++c) {
+          const int tok = (CW * cw + c) / HPT;
           if (!visible_elem(q0 + tok, kj, it.seq_len, p.causal, p.n_sink, p.window)) P[c] = 0.f;
         }
       }
       {
-        uint32_t pk[32];
+        uint32_t pk[CW / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(P[2 * c], P[2 * c + 1]);
-        tmem_st32(tmem + lane_off + C::S_COL + 64 * cw, pk);
+        for (int c = 0; c < CW / 2; ++c) pk[c] = pack_bf16x2(P[2 * c], P[2 * c + 1]);
+        if constexpr (CW == 64)
+          tmem_st32(tmem + lane_off + C::S_COL + CW * cw, pk);
+        else
+          tmem_st16(tmem + lane_off + C::S_COL + CW * cw, pk);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -400,11 +522,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, i & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t ds[32];
+      uint32_t ds[CW / 2];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      for (int h2 = 0; h2 < CW / 32; ++h2) {
         uint32_t a[32];
-        tmem_ld32(tmem + lane_off + C::DP_COL + 64 * cw + 32 * h2, a);
+        tmem_ld32(tmem + lane_off + C::DP_COL + CW * cw + 32 * h2, a);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -413,55 +535,26 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                         P[x + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[x + 1]));
         }
       }
-      tmem_st32(tmem + lane_off + C::DP_COL + 64 * cw, ds);
-      // the previous dQ MMA must be done reading the staged dS tile
-      if (i > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, (i - 1) & 1, abort_flag, p.status));
-        if (!ok) break;
-      }
+      if constexpr (CW == 64)
+        tmem_st32(tmem + lane_off + C::DP_COL + CW * cw, ds);
+      else
+        tmem_st16(tmem + lane_off + C::DP_COL + CW * cw, ds);
+      // The staged dS tile is free: dP^T of this iteration was issued after
+      // the previous dQ MMA, and its completion covers that MMA.  Layout:
+      // [QR / 64 atoms][keys][64 queries] with the 128-byte swizzle.
       if (row_ok) {
-        // row r of the [keys][64 queries] half-tile, 128-byte swizzle
-        uint8_t* row = smem + C::OFF_DS + cw * (KT * 128) + r * 128;
+        constexpr int CHUNKS = CW / 8;  // 16-byte chunks of this warpgroup's queries
+        uint8_t* row = smem + C::OFF_DS + ((CW * cw) / 64) * (KT * 128) + r * 128;
+        const int j0 = ((CW * cw) % 64) / 8;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) * 16)) =
+        for (int j = 0; j < CHUNKS; ++j)
+          *reinterpret_cast<uint4*>(row + (((j0 + j) ^ (r & 7)) * 16)) =
               make_uint4(ds[4 * j], ds[4 * j + 1], ds[4 * j + 2], ds[4 * j + 3]);
       }
       fence_async_smem();
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_ds);
-      // dQ tile: lanes are query rows; this warpgroup takes D/2 columns, 32
-      // at a time.  All MMAs of this iteration are complete, so the stage's
-      // Q (warpgroup 0) or dO (warpgroup 1) buffer takes the fp32 values
-      // (128-byte swizzle), and one thread adds them into the fp32 dQ buffer
-      // with bulk tensor reductions.  Query rows past the sequence end carry
-      // exact zeros (their P is 0), so adding them is harmless.
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, p.status));
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const int s = i % NS;
-        uint8_t* stage = smem + (cw == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
-        const int qrow = tw;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t a[32];
-          tmem_ld32(tmem + lane_off + C::DP_COL + (D / 2) * cw + 32 * c, a);
-          tmem_ld_wait();
-          if (c == D / 64 - 1) {
-            tc_fence_before();
-            mbar_arrive(bar_dqf);  // the dP region may be overwritten
-          }
-          uint8_t* row = stage + c * (128 * 128) + qrow * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
-                make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
-        }
-        fence_async_smem();
-        mbar_arrive(bar_dqs + s);  // the reducer warp takes it from here
-      }
     }
     // dK (warpgroup 0) and dV (warpgroup 1) rows of this key tile
     const bool have = n_it > 0 && ok &&
@@ -577,15 +670,15 @@ __global__ void dq_convert_kernel(const float4* acc, uint2* dq, long long n4, fl
   dq[i] = make_uint2(pack_bf16x2(v.x * alpha, v.y * alpha), pack_bf16x2(v.z * alpha, v.w * alpha));
 }
 
-template <int D, int KT>
+template <class C>
 int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
-  using C = BwdCfg<D, KT>;
+  constexpr int D = C::D;
   CUtensorMap mq, mdo, mk, mv, mdq, mdk, mdv;
-  if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
-      !make_tmap_3d(&mdo, b.dout, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
+  if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, C::QT) ||
+      !make_tmap_3d(&mdo, b.dout, p.T_tot, p.Hq, D, C::HPT, C::QT) ||
       !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::KT) ||
       !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::KT) ||
-      !make_tmap_3d_f32(&mdq, b.dq_accum, p.T_tot, p.Hq, D, C::HPT, C::TQ) ||
+      !make_tmap_3d_f32(&mdq, b.dq_accum, p.T_tot, p.Hq, D, C::HPT, C::QT) ||
       !make_tmap_3d_f32(&mdk, b.dk_accum, p.T_tot, p.Hkv, D, 1, C::KT) ||
       !make_tmap_3d_f32(&mdv, b.dv_accum, p.T_tot, p.Hkv, D, 1, C::KT))
     return SINKATTN_ERR_CUDA;
@@ -593,7 +686,6 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   bp.plan = p.plan;
   bp.lse2 = b.lse2;
   bp.delta = b.delta;
-  bp.dq_accum = b.dq_accum;
   bp.dk = static_cast<__nv_bfloat16*>(b.dk);
   bp.dv = static_cast<__nv_bfloat16*>(b.dv);
   bp.status = p.status;
@@ -615,6 +707,13 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
+  if constexpr (C::REBALANCE) {
+    // the register split assumes the launch-bound count per thread; with
+    // fewer, a setmaxnreg.inc would wait for registers that never come
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != C::LAUNCH_REGS)
+      return SINKATTN_ERR_UNSUPPORTED;
+  }
   const dim3 split_grid(p.ps.cap_items, C::KT);
   split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
                                                      p.Hkv, D, p.scale, 0);
@@ -637,9 +736,11 @@ size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int Hkv, int D) {
 
 int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   if (p.ps.tile == 128)
-    return p.D == 128 ? launch_cfg<128, 128>(p, b, stream) : launch_cfg<64, 128>(p, b, stream);
+    return p.D == 128 ? launch_cfg<BwdCfg<128, 128, 128, 1>>(p, b, stream)
+                      : launch_cfg<BwdCfg<64, 128, 128, 1>>(p, b, stream);
   if ((p.Hq / p.Hkv) % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;  // 64-token tiles pair heads
-  return p.D == 128 ? launch_cfg<128, 64>(p, b, stream) : launch_cfg<64, 64>(p, b, stream);
+  return p.D == 128 ? launch_cfg<BwdCfg<128, 64, 64, 2>>(p, b, stream)
+                    : launch_cfg<BwdCfg<64, 64, 64, 2>>(p, b, stream);
 }
 
 }  // namespace sk

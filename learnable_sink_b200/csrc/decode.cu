@@ -36,6 +36,19 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   }
 }
 
+// bf16 -> fp32 is exact and needs only the 16 bits moved up: integer ops,
+// no conversion unit.  Pair i holds elements 2i (low half) and 2i + 1.
+__device__ __forceinline__ void bf16x8_to_f32x2(const uint4& u, float2 (&f)[4]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+
+// The streaming decode moves its running maximum only past this margin
+// (log2 units): probabilities stay below 2^8, far from fp32 overflow.
+constexpr float kLazyLog2 = 8.f;
+
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
   if constexpr (sizeof(T) == 2) {
@@ -177,21 +190,28 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeProblem
 }
 
 // Persistent streaming variant (bf16): one CTA per SM loops over work items
-// (sequence, KV head, split).  Warp 16 streams 64-row pieces of K and V with
-// TMA through a kStreamStages-deep ring that runs ahead across item
-// boundaries, so HBM stays busy while warps 0-15 compute.  A group of D/8
+// (sequence, KV head, split).  The last warp streams 64-row pieces of K and V
+// with TMA through a kStreamStages-deep ring that runs ahead across item
+// boundaries, so HBM stays busy while the consumer warps compute.  A group of D/8
 // lanes holds one row's 8-element slices; each group takes PR rows of every
 // piece and keeps its own online-softmax state per head (running max, sum and
 // output slice), so groups never wait for each other inside an item; they
 // merge, max-rescaled, once per item.  Dot products of a group's PR x G
 // (row, head) pairs are reduced by a butterfly that splits the values across
-// the group's lanes.
+// the group's lanes.  The loop is kept short because the consumers, not HBM,
+// set the pace: bf16 is widened with integer ops, products use the packed
+// fp32x2 FMA, and the running maximum moves only when a score exceeds it by
+// more than 2^8 (so the output rescale is rare; the final O = acc / l does not
+// depend on which reference maximum was used).
 constexpr int kPieceRows = 64;
 constexpr int kStreamStages = 4;
-// consumer threads: 16 warps, or 8 when eight query heads share a KV head
-// (their per-head state would not fit 16 warps' register budget)
+// consumer threads: 8 warps; with the producer warp the CTA has 9 warps, and
+// registers are handed out per group of four warps, so a thread may use
+// 65536 / (12 x 32) = 170 -> 168 registers (17 warps would leave 96)
 template <int G>
-constexpr int consumer_threads() { return G >= 8 ? 256 : 512; }
+constexpr int consumer_threads() { return 256; }
+template <int G>
+constexpr int stream_regs() { return 65536 / ((consumer_threads<G>() + 32 + 127) / 128 * 128) / 8 * 8; }
 
 template <int D, int G>
 struct StreamGeom {
@@ -205,8 +225,8 @@ struct StreamGeom {
   static constexpr int HALF_BYTES = kPieceRows * 128;        // one 64-column half of a piece
   static constexpr int PIECE_BYTES = DH * HALF_BYTES;        // K or V piece
   static constexpr int STAGE_BYTES = 2 * PIECE_BYTES;
-  static constexpr int OFF_SC = kStreamStages * STAGE_BYTES; // float [NGRP][V] group scratch
-  static constexpr int OFF_RED = OFF_SC + NGRP * V * 4;      // float [warps][G][D]
+  static constexpr int OFF_SC = kStreamStages * STAGE_BYTES; // float [2][NGRP][V] scores, probabilities
+  static constexpr int OFF_RED = OFF_SC + 2 * NGRP * V * 4;  // float [warps][G][D]
   static constexpr int OFF_ML = OFF_RED + kConsumerWarps * G * D * 4;  // float [warps][G][2]
   static constexpr int OFF_BAR = OFF_ML + kConsumerWarps * G * 2 * 4;
   // + 1024: the kernel rounds the dynamic shared-memory base up to 1024 bytes
@@ -253,7 +273,7 @@ __device__ __forceinline__ int decode_value_index(int gl, int j) {
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_kernel(
+__global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     DecodeProblem p, int chunk, int n_items) {
   using Geo = StreamGeom<D, G>;
@@ -271,7 +291,7 @@ __global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_k
   if (tid == 0) {
     for (int i = 0; i < kStreamStages; ++i) {
       mbar_init(full + i, 1);
-      mbar_init(empty + i, kConsumerThreads);
+      mbar_init(empty + i, kConsumerWarps);  // one arrival per consumer warp
     }
     abort_s = 0;
     fence_mbar_init();
@@ -312,27 +332,30 @@ __global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_k
   // ------------------------------------------------------------ consumers
   const int grp = tid / LPR, gl = tid % LPR;
   const int c0 = gl * 8, hf = c0 / 64, cin = c0 % 64;
-  float* scg = reinterpret_cast<float*>(sm + Geo::OFF_SC) + grp * V;  // group scratch
+  float* sc_s = reinterpret_cast<float*>(sm + Geo::OFF_SC) + grp * V;               // scores
+  float* sc_p = reinterpret_cast<float*>(sm + Geo::OFF_SC) + (Geo::NGRP + grp) * V;  // probabilities
   const float scale_log2 = p.scale * kLog2e;
   int pc = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     int b, kvh, split, n;
     item_rows(item, b, kvh, split, n);
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.Hq + kvh * G) * D;
-    float qv[G][8];
+    float2 qv[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      load8<__nv_bfloat16>(qb + h * D + c0, qv[h]);
+      float2 t[4];
+      bf16x8_to_f32x2(__ldg(reinterpret_cast<const uint4*>(qb + h * D + c0)), t);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) qv[h][c] *= scale_log2;
+      for (int i = 0; i < 4; ++i) qv[h][i] = make_float2(t[i].x * scale_log2, t[i].y * scale_log2);
     }
-    float acc[G][8], m_run[G], l_run[G];
+    float2 acc[G][4];
+    float m_run[G], l_run[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_run[h] = -INFINITY;
       l_run[h] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
+      for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
     }
     for (int r0 = 0; r0 < n; r0 += kPieceRows, ++pc) {
       const int st = pc % kStreamStages;
@@ -345,68 +368,71 @@ __global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_k
 #pragma unroll
       for (int rr = 0; rr < PR; ++rr) {
         const int r = grp * PR + rr;
-        float kf[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(kbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), kf);
+        float2 kf[4];
+        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(kbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), kf);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          float a = 0.f;
+          float2 a = __fmul2_rn(qv[h][0], kf[0]);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) a += qv[h][c] * kf[c];
-          v[rr * G + h] = a;
+          for (int i = 1; i < 4; ++i) a = __ffma2_rn(qv[h][i], kf[i], a);
+          v[rr * G + h] = a.x + a.y;
         }
       }
       butterfly_reduce<V, LPR>(v, gl);
 #pragma unroll
       for (int j = 0; j < Geo::KEEP; ++j) {
         const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
-        scg[idx] = (grp * PR + idx / G < rows) ? v[j] : -INFINITY;
+        sc_s[idx] = (grp * PR + idx / G < rows) ? v[j] : -INFINITY;
       }
       __syncwarp();
-      // per-head maximum over the group's rows, new running max, rescale
-      float mnew[G], corr[G];
+      // Running maximum per head over the group's rows; it moves (and the
+      // group's sum and output are rescaled) only when a score exceeds it by
+      // more than 2^kLazyLog2.  From -inf any finite score moves it; an
+      // all-masked piece leaves it alone.
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float mx = m_run[h];
+        float mx = -INFINITY;
 #pragma unroll
-        for (int rr = 0; rr < PR; ++rr) mx = fmaxf(mx, scg[rr * G + h]);
-        mnew[h] = mx;
-        corr[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mx);
+        for (int rr = 0; rr < PR; ++rr) mx = fmaxf(mx, sc_s[rr * G + h]);
+        if (mx > m_run[h] + kLazyLog2) {
+          const float corr = fast_exp2(m_run[h] - mx);  // 0 when m_run was -inf
+          l_run[h] *= corr;
+          const float2 c2 = make_float2(corr, corr);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[h][i] = __fmul2_rn(acc[h][i], c2);
+          m_run[h] = mx;
+        }
       }
-      __syncwarp();  // every lane has read the scores before they become probabilities
 #pragma unroll
       for (int j = 0; j < Geo::KEEP; ++j) {
         const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
-        const int h = idx % G;
-        const float sv = (grp * PR + idx / G < rows) ? v[j] : -INFINITY;
-        scg[idx] = (mnew[h] == -INFINITY) ? 0.f : exp2f(sv - mnew[h]);
+        const int hj = idx % G;
+        float mh = m_run[0];
+#pragma unroll
+        for (int h = 1; h < G; ++h) mh = hj == h ? m_run[h] : mh;
+        sc_p[idx] = (grp * PR + idx / G < rows) ? fast_exp2(v[j] - mh) : 0.f;
       }
       __syncwarp();
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float ps = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < PR; ++rr) ps += scg[rr * G + h];
-        l_run[h] = l_run[h] * corr[h] + ps;
-        m_run[h] = mnew[h];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[h][c] *= corr[h];
-      }
+      // P V over the group's rows (rows past the valid range may hold any
+      // bits, so they are skipped rather than weighted by zero)
 #pragma unroll
       for (int rr = 0; rr < PR; ++rr) {
         const int r = grp * PR + rr;
         if (r < rows) {
-          float vf[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(vbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), vf);
+          float2 vf[4];
+          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(vbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), vf);
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float pr = scg[rr * G + h];
+            const float pr = sc_p[rr * G + h];
+            l_run[h] += pr;
+            const float2 p2 = make_float2(pr, pr);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[h][c] += pr * vf[c];
+            for (int i = 0; i < 4; ++i) acc[h][i] = __ffma2_rn(p2, vf[i], acc[h][i]);
           }
         }
       }
-      __syncwarp();  // scratch reads done before the next piece's writes
-      mbar_arrive(empty + st);  // this thread is done with the stage
+      __syncwarp();  // every lane of the warp is done with the stage and the scratch
+      if (lane == 0) mbar_arrive(empty + st);
     }
     // merge the groups of a warp (lanes gl and gl + LPR, ...) with max rescaling
 #pragma unroll
@@ -420,9 +446,10 @@ __global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_k
         const float fb = (mo == -INFINITY) ? 0.f : exp2f(mo - mm);
         l_run[h] = l_run[h] * fa + lo * fb;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float ao = __shfl_xor_sync(0xffffffffu, acc[h][c], o);
-          acc[h][c] = acc[h][c] * fa + ao * fb;
+        for (int i = 0; i < 4; ++i) {
+          const float ax = __shfl_xor_sync(0xffffffffu, acc[h][i].x, o);
+          const float ay = __shfl_xor_sync(0xffffffffu, acc[h][i].y, o);
+          acc[h][i] = make_float2(acc[h][i].x * fa + ax * fb, acc[h][i].y * fa + ay * fb);
         }
         m_run[h] = mm;
       }
@@ -431,7 +458,10 @@ __global__ void __launch_bounds__(consumer_threads<G>() + 32, 1) decode_stream_k
 #pragma unroll
       for (int h = 0; h < G; ++h) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) red[(warp * G + h) * D + c0 + c] = acc[h][c];
+        for (int i = 0; i < 4; ++i) {
+          red[(warp * G + h) * D + c0 + 2 * i] = acc[h][i].x;
+          red[(warp * G + h) * D + c0 + 2 * i + 1] = acc[h][i].y;
+        }
         if (gl == 0) {
           ml[(warp * G + h) * 2] = m_run[h];
           ml[(warp * G + h) * 2 + 1] = l_run[h];

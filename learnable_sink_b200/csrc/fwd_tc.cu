@@ -498,6 +498,13 @@ int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaS
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
+  if constexpr (C::REBALANCE) {
+    // the register split assumes the launch-bound count per thread; with
+    // fewer, a setmaxnreg.inc would wait for registers that never come
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != 65536 / C::THREADS / 8 * 8)
+      return SINKATTN_ERR_UNSUPPORTED;
+  }
   record_start(SINKATTN_KERNEL_FWD, stream);
   kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, fp);
   record_stop(SINKATTN_KERNEL_FWD, stream);

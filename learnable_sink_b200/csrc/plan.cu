@@ -379,7 +379,8 @@ __global__ void __launch_bounds__(kScanThreads) plan_units_order_kernel(PlanArgs
     order[atomicAdd(&cursor[kBwdChunk - units[u].z], 1)] = u;
 }
 
-// G: sort every reverse list by query tile (insertion sort; lists are short).
+// G: sort every reverse list by query tile, latest first (insertion sort;
+// lists are short).
 __global__ void plan_bwd_sort_kernel(PlanArgs a) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= a.cap_items) return;
@@ -389,7 +390,7 @@ __global__ void plan_bwd_sort_kernel(PlanArgs a) {
   for (int x = 1; x < it.entry_len; ++x) {
     const int v = e[x];
     int p = x;
-    while (p > 0 && e[p - 1] > v) { e[p] = e[p - 1]; --p; }
+    while (p > 0 && e[p - 1] < v) { e[p] = e[p - 1]; --p; }
     e[p] = v;
   }
 }

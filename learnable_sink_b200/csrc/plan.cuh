@@ -13,7 +13,10 @@
 //   fwd_entries[cap_entries]  (key tile << 1) | partial
 //   bwd_items / bwd_order / bwd_entries: the reverse lists (per key tile, the
 //                        query tiles that see it), entries (query tile << 1) |
-//                        partial, each list sorted by query tile
+//                        partial, each list latest query tile first (the
+//                        CTAs of one sequence and KV head then read the
+//                        same query tiles at about the same time, so the
+//                        second and later reads hit L2)
 //   bwd_cursor[cap_items] scratch for the reverse scatter
 //   bwd_units[cap_units][4] backward work units: (bwd item, first entry,
 //                        entry count, number of units of that item); a

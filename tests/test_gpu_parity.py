@@ -47,7 +47,7 @@ def expected_lists(ms, T, Hq, Hkv, tile):
                 fwd[(g, int(base[s] + qt))] = ents
             for kt in range(nt):
                 ents = [(qt << 1) | int(st[g, base[s] + qt, kt] == 1)
-                        for qt in range(nt) if st[g, base[s] + qt, kt] > 0]
+                        for qt in range(nt - 1, -1, -1) if st[g, base[s] + qt, kt] > 0]
                 bwd[(g, int(base[s] + kt))] = ents
     return fwd, bwd
 
