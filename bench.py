@@ -431,7 +431,7 @@ def run_ours(args, world, rank, local):
                               "frac_of_sustained": fwd_ach / peak_tf},
             "bwd_tc_kernel": {"ms": kb_ms, "achieved_tflops": bwd_ach,
                               "frac_of_sustained": bwd_ach / peak_tf},
-            "decode_split_kernel": {"ms": kd_ms, "achieved_gbs": dec_ach,
+            "decode_warp_kernel": {"ms": kd_ms, "achieved_gbs": dec_ach,
                                     "frac_of_hbm": dec_ach / peaks["hbm_gbs"]},
         },
     }

@@ -248,25 +248,31 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
   return launch_bwd_tc(p, b, s);
 }
 
+// the split merge handles up to this many splits
+constexpr int kMaxDecodeSplits = 128;
+
 int sinkattn_decode_num_splits(int B, int Hq, int Hkv, int D, int n_sink, int window) {
   (void)Hq; (void)D;
   const int S = n_sink + window;
   if (B < 1 || Hkv < 1 || S < 1) return 1;
   int sms = 148, dev;
   if (current_device(&dev)) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // enough (sequence, KV head, split) items for about six per SM, so the
-  // persistent streaming kernel balances within a few percent
+  // enough (sequence, KV head, split) items for about three per warp of the
+  // streaming kernel (8 warps per SM take items from a shared counter), and
+  // no split shorter than 16 slots
   const long long pairs = (long long)B * Hkv;
-  long long want = ((long long)sms * 6 + pairs - 1) / pairs;
-  long long max_split = (S + 63) / 64;
+  long long want = ((long long)sms * 8 * 3 + pairs - 1) / pairs;
+  long long max_split = (S + 15) / 16;
   if (want > max_split) want = max_split;
+  if (want > kMaxDecodeSplits) want = kMaxDecodeSplits;
   if (want < 1) want = 1;
   return (int)want;
 }
 
 size_t sinkattn_decode_workspace_bytes(int B, int Hq, int D, int num_splits) {
   if (B < 1 || Hq < 1 || num_splits < 1 || (D != 64 && D != 128)) return 0;
-  return round_up(sizeof(float) * (size_t)B * Hq * num_splits * (D + 2));
+  // per-split partials, then the streaming kernel's work-item counter
+  return round_up(sizeof(float) * (size_t)B * Hq * num_splits * (D + 2)) + kAlign;
 }
 
 int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scale,
@@ -289,6 +295,7 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
     return SINKATTN_ERR_INVALID_ARG;
   if (num_splits <= 0) num_splits = sinkattn_decode_num_splits(B, Hq, Hkv, D, n_sink, window);
   if (num_splits > n_sink + window) num_splits = n_sink + window;
+  if (num_splits > kMaxDecodeSplits) num_splits = kMaxDecodeSplits;  // same result, fewer splits
   if (workspace_bytes < sinkattn_decode_workspace_bytes(B, Hq, D, num_splits))
     return SINKATTN_ERR_WORKSPACE;
   if (!device_is_sm100()) return SINKATTN_ERR_UNSUPPORTED;
@@ -311,6 +318,8 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
   p.lse = lse_new;
   p.sink_s = sink_s;
   p.part = static_cast<float*>(workspace);
+  p.counter = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                     round_up(sizeof(float) * (size_t)B * Hq * num_splits * (D + 2)));
   p.status = status_word();
   return launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
 }

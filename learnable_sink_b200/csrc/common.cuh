@@ -79,6 +79,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 // 3-D tiled bulk tensor load global -> shared, completing on `bar`.
 // c0 is the innermost (contiguous) coordinate; callers keep c0 * elem_size a
 // multiple of 16 bytes.
+// Untiled bulk copy global -> shared, completing on `bar` (both addresses
+// 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes),
+      "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map,
                                             uint64_t* bar, int c0, int c1, int c2) {
   asm volatile(

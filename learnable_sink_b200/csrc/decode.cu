@@ -189,53 +189,49 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeProblem
   }
 }
 
-// Persistent streaming variant (bf16): one CTA per SM loops over work items
-// (sequence, KV head, split).  The last warp streams 64-row pieces of K and V
-// with TMA through a kStreamStages-deep ring that runs ahead across item
-// boundaries, so HBM stays busy while the consumer warps compute.  A group of D/8
-// lanes holds one row's 8-element slices; each group takes PR rows of every
-// piece and keeps its own online-softmax state per head (running max, sum and
-// output slice), so groups never wait for each other inside an item; they
-// merge, max-rescaled, once per item.  Dot products of a group's PR x G
-// (row, head) pairs are reduced by a butterfly that splits the values across
-// the group's lanes.  The loop is kept short because the consumers, not HBM,
-// set the pace: bf16 is widened with integer ops, products use the packed
-// fp32x2 FMA, and the running maximum moves only when a score exceeds it by
-// more than 2^8 (so the output rescale is rare; the final O = acc / l does not
-// depend on which reference maximum was used).
-constexpr int kPieceRows = 64;
-constexpr int kStreamStages = 4;
-// consumer threads: 8 warps; with the producer warp the CTA has 9 warps, and
-// registers are handed out per group of four warps, so a thread may use
-// 65536 / (12 x 32) = 170 -> 168 registers (17 warps would leave 96)
-template <int G>
-constexpr int consumer_threads() { return 256; }
-template <int G>
-constexpr int stream_regs() { return 65536 / ((consumer_threads<G>() + 32 + 127) / 128 * 128) / 8 * 8; }
+// Warp-streaming variant (bf16).  Every warp works alone: it takes work
+// items (sequence, KV head, split) from a global counter, streams its items'
+// K and V rows with TMA through a private ring of RS stages (the loads for the
+// next pieces, and for the first pieces of its next item, are in flight while
+// it computes), and writes one partial (m, l, acc) per query head and item.
+// No warp ever waits for another, so nothing couples the warps of an SM
+// beyond sharing its load bandwidth.  A group of D/8 lanes holds one row's
+// 8-element slices; the warp's groups split each piece's rows (PR each) and
+// merge their online-softmax states, max-rescaled, once per item.  Dot
+// products of a group's PR x G (row, head) pairs are reduced by a butterfly
+// that splits the values across the group's lanes.  bf16 is widened with
+// integer ops, products use the packed fp32x2 FMA, and the running maximum
+// moves only when a score exceeds it by more than 2^8 (so the output rescale
+// is rare; O = acc / l does not depend on which reference maximum was used).
+constexpr int kDecWarps = 8;      // warps per CTA (one CTA per SM)
+constexpr int kDecStages = 3;     // ring stages per warp
+constexpr int kLenSlots = 1024;   // sequences whose cache lengths are staged in shared memory
 
 template <int D, int G>
-struct StreamGeom {
-  static constexpr int kConsumerThreads = consumer_threads<G>();
-  static constexpr int kConsumerWarps = kConsumerThreads / 32;
-  static constexpr int DH = D / 64;
+struct WarpGeom {
   static constexpr int LPR = D / 8;                          // lanes per row
-  static constexpr int NGRP = kConsumerThreads / LPR;        // row groups
-  static constexpr int PR = kPieceRows / NGRP;               // rows per group per piece
+  static constexpr int NGW = 32 / LPR;                       // row groups per warp
+  static constexpr int PR0 = 16 / NGW;
+  static constexpr int PR = PR0 * G <= 32 ? PR0 : 32 / G;    // rows per group per piece
+  static constexpr int R = NGW * PR;                         // rows per piece
   static constexpr int V = PR * G;                           // values per lane before reduce
-  static constexpr int HALF_BYTES = kPieceRows * 128;        // one 64-column half of a piece
-  static constexpr int PIECE_BYTES = DH * HALF_BYTES;        // K or V piece
+  static constexpr int ROW_BYTES = D * 2;                    // one row of one head
+  static constexpr int PIECE_BYTES = R * ROW_BYTES;          // K or V piece [R][D]
   static constexpr int STAGE_BYTES = 2 * PIECE_BYTES;
-  static constexpr int OFF_SC = kStreamStages * STAGE_BYTES; // float [2][NGRP][V] scores, probabilities
-  static constexpr int OFF_RED = OFF_SC + 2 * NGRP * V * 4;  // float [warps][G][D]
-  static constexpr int OFF_ML = OFF_RED + kConsumerWarps * G * D * 4;  // float [warps][G][2]
-  static constexpr int OFF_BAR = OFF_ML + kConsumerWarps * G * 2 * 4;
-  // + 1024: the kernel rounds the dynamic shared-memory base up to 1024 bytes
-  static constexpr int SMEM = OFF_BAR + 2 * kStreamStages * 8 + 1024;
+  static constexpr int Q_BYTES = G * D * 2;                  // an item's query heads (bf16)
+  static constexpr int OFF_Q = kDecStages * STAGE_BYTES;     // 2 q slots (this item, next)
+  static constexpr int OFF_SC = OFF_Q + 2 * Q_BYTES;         // float [2][NGW][V] scores, probabilities
+  static constexpr int WARP_BYTES = (OFF_SC + 2 * NGW * V * 4 + 127) / 128 * 128;
+  static constexpr int OFF_BAR = kDecWarps * WARP_BYTES;
+  static constexpr int OFF_LEN = OFF_BAR + kDecWarps * kDecStages * 8;  // int [kLenSlots]
+  // + 128: the kernel rounds the dynamic shared-memory base up to 128 bytes
+  static constexpr int SMEM = OFF_LEN + kLenSlots * 4 + 128;
   static constexpr int LOG_LPR = LPR == 16 ? 4 : 3;
   static constexpr int LOG_V = V >= 32 ? 5 : V >= 16 ? 4 : V >= 8 ? 3 : V >= 4 ? 2 : V >= 2 ? 1 : 0;
   static constexpr int KS = LOG_V < LOG_LPR ? LOG_V : LOG_LPR;  // splitting steps
   static constexpr int KEEP = V >> KS;                        // values a lane ends with
   static_assert(PR >= 1 && (1 << LOG_V) == V, "power-of-two rows x heads");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
 // Sum each of the V values over the LPR lanes of a group; afterwards lane gl
@@ -272,82 +268,189 @@ __device__ __forceinline__ int decode_value_index(int gl, int j) {
   return idx | j;
 }
 
-template <int D, int G>
-__global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
-    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-    DecodeProblem p, int chunk, int n_items) {
-  using Geo = StreamGeom<D, G>;
-  constexpr int LPR = Geo::LPR, PR = Geo::PR, V = Geo::V, DH = Geo::DH;
-  constexpr int kConsumerThreads = Geo::kConsumerThreads, kConsumerWarps = Geo::kConsumerWarps;
-  extern __shared__ uint8_t dsm_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  float* red = reinterpret_cast<float*>(sm + Geo::OFF_RED);
-  float* ml = reinterpret_cast<float*>(sm + Geo::OFF_ML);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR);
-  uint64_t* empty = full + kStreamStages;
-  __shared__ int abort_s;
-  const int S = p.n_sink + p.window;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    for (int i = 0; i < kStreamStages; ++i) {
-      mbar_init(full + i, 1);
-      mbar_init(empty + i, kConsumerWarps);  // one arrival per consumer warp
-    }
-    abort_s = 0;
-    fence_mbar_init();
+// Merge the splits of query head h of sequence b with the sink column (page
+// "Attention Sink, Learnable Sink and dsink", section 4: e^{a_h} joins the
+// denominator, the sink value is zero) and write O, LSE_new and sink_s.  One
+// warp; lane l owns output columns [l D/32, (l + 1) D/32).  Every split's
+// (m, l) is loaded at once (split i in lane i % 32), then eight splits' output
+// columns per step, so the merge costs a few L2 round trips, not one per split.
+template <typename T, int D>
+__device__ __forceinline__ void combine_head(const DecodeProblem& p, int b, int h, int lane) {
+  constexpr int DPL = D / 32;
+  const int ns = p.num_splits;
+  const float* part = p.part + ((long long)b * p.Hq + h) * ns * (D + 2);
+  const float a2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
+  // split i's (m, l) in lane i % 32 (all loads in flight at once)
+  constexpr int MAXR = 4;  // up to 128 splits
+  float mi[MAXR], li[MAXR];
+  float mt = a2;
+#pragma unroll
+  for (int r = 0; r < MAXR; ++r) {
+    const int i = r * 32 + lane;
+    mi[r] = i < ns ? __ldcg(part + i * (D + 2) + D) : -INFINITY;
+    li[r] = i < ns ? __ldcg(part + i * (D + 2) + D + 1) : 0.f;
+    mt = fmaxf(mt, mi[r]);
   }
-  __syncthreads();
-  auto item_rows = [&](int item, int& b, int& kvh, int& split, int& n) {
-    split = item % p.num_splits;
-    kvh = (item / p.num_splits) % p.Hkv;
-    b = item / (p.num_splits * p.Hkv);
-    const int n_valid = min(max(p.cache_seqlens[b], 0), S);
-    n = max(min(split * chunk + chunk, n_valid) - split * chunk, 0);
-  };
-
-  if (warp == kConsumerWarps) {
-    // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      int pc = 0;
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        int b, kvh, split, n;
-        item_rows(item, b, kvh, split, n);
-        for (int r0 = 0; r0 < n; r0 += kPieceRows, ++pc) {
-          const int st = pc % kStreamStages;
-          if (!mbar_wait(empty + st, ((pc / kStreamStages) & 1) ^ 1, &abort_s, p.status)) return;
-          mbar_expect_tx(full + st, Geo::STAGE_BYTES);
-          const int row0 = b * S + split * chunk + r0;  // rows past the split are unused
-          uint8_t* base = sm + st * Geo::STAGE_BYTES;
-          for (int h = 0; h < DH; ++h) {
-            tma_load_3d(base + h * Geo::HALF_BYTES, &tmap_k, full + st, h * 64, kvh, row0);
-            tma_load_3d(base + Geo::PIECE_BYTES + h * Geo::HALF_BYTES, &tmap_v, full + st, h * 64,
-                        kvh, row0);
-          }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+  float l = 0.f, o[DPL];
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) o[k] = 0.f;
+  if (mt != -INFINITY) {
+    float wi[MAXR];
+#pragma unroll
+    for (int r = 0; r < MAXR; ++r) {
+      wi[r] = mi[r] == -INFINITY ? 0.f : exp2f(mi[r] - mt);
+      l += li[r] * wi[r];
+    }
+#pragma unroll
+    for (int o2 = 16; o2 >= 1; o2 >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o2);
+    // output columns: eight splits' loads in flight per step
+    for (int i0 = 0; i0 < ns; i0 += 8) {
+      float2 x[8][DPL / 2];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int k = 0; k < DPL; k += 2)
+          x[u][k / 2] = i0 + u < ns
+              ? __ldcg(reinterpret_cast<const float2*>(part + (i0 + u) * (D + 2) + lane * DPL + k))
+              : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u;
+        float w = 0.f;
+#pragma unroll
+        for (int r = 0; r < MAXR; ++r) {
+          const float wr = __shfl_sync(0xffffffffu, wi[r], i & 31);
+          w = (i >> 5) == r ? wr : w;
+        }
+#pragma unroll
+        for (int k = 0; k < DPL; k += 2) {
+          o[k] += x[u][k / 2].x * w;
+          o[k + 1] += x[u][k / 2].y * w;
         }
       }
     }
-    return;
   }
+  const float den = l + (p.sink && mt != -INFINITY ? exp2f(a2 - mt) : 0.f);
+  const long long row = (long long)b * p.Hq + h;
+#pragma unroll
+  for (int k = 0; k < DPL; k += 2) {
+    const float o0 = den > 0.f ? o[k] / den : 0.f, o1 = den > 0.f ? o[k + 1] / den : 0.f;
+    if constexpr (sizeof(T) == 2)
+      *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) + row * D + lane * DPL + k) =
+          pack_bf16x2(o0, o1);
+    else
+      *reinterpret_cast<float2*>(static_cast<float*>(p.out) + row * D + lane * DPL + k) =
+          make_float2(o0, o1);
+  }
+  if (lane == 0) {
+    p.lse[row] = den > 0.f ? (mt + log2f(den)) * kLn2 : -INFINITY;
+    if (p.sink_s) p.sink_s[row] = den > 0.f ? l / den : 0.f;
+  }
+}
 
-  // ------------------------------------------------------------ consumers
-  const int grp = tid / LPR, gl = tid % LPR;
-  const int c0 = gl * 8, hf = c0 / 64, cin = c0 % 64;
-  float* sc_s = reinterpret_cast<float*>(sm + Geo::OFF_SC) + grp * V;               // scores
-  float* sc_p = reinterpret_cast<float*>(sm + Geo::OFF_SC) + (Geo::NGRP + grp) * V;  // probabilities
-  const float scale_log2 = p.scale * kLog2e;
-  int pc = 0;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    int b, kvh, split, n;
-    item_rows(item, b, kvh, split, n);
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + ((long long)b * p.Hq + kvh * G) * D;
-    float2 qv[G][4];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float2 t[4];
-      bf16x8_to_f32x2(__ldg(reinterpret_cast<const uint4*>(qb + h * D + c0)), t);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) qv[h][i] = make_float2(t[i].x * scale_log2, t[i].y * scale_log2);
+template <int D, int G>
+__global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+    DecodeProblem p, int chunk, int n_items) {
+  using Geo = WarpGeom<D, G>;
+  constexpr int LPR = Geo::LPR, PR = Geo::PR, V = Geo::V, R = Geo::R;
+  constexpr int RS = kDecStages;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+  __shared__ int abort_s;
+  const int S = p.n_sink + p.window;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* wsm = sm + warp * Geo::WARP_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR) + warp * RS;
+  // cache_seqlens of every sequence, staged once per CTA when they fit
+  int* s_len = reinterpret_cast<int*>(sm + Geo::OFF_LEN);
+  const bool len_in_smem = p.B <= kLenSlots;
+  if (len_in_smem)
+    for (int i = threadIdx.x; i < p.B; i += blockDim.x) s_len[i] = __ldg(p.cache_seqlens + i);
+  if (threadIdx.x == 0) abort_s = 0;
+  if (lane == 0) {
+    for (int i = 0; i < RS; ++i) mbar_init(full + i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // A work item, decoded once when the warp takes it.
+  struct Item {
+    int it, n, row0, kvh, b, split;  // n = valid rows, row0 = first cache row
+  };
+  auto decode_item = [&](int it) {
+    Item I{it, 0, 0, 0, 0, 0};
+    if (it < n_items) {
+      I.split = it % p.num_splits;
+      I.kvh = (it / p.num_splits) % p.Hkv;
+      I.b = it / (p.num_splits * p.Hkv);
+      const int cs = len_in_smem ? s_len[I.b] : __ldg(p.cache_seqlens + I.b);
+      const int n_valid = min(max(cs, 0), S);
+      I.n = max(min(I.split * chunk + chunk, n_valid) - I.split * chunk, 0);
+      I.row0 = I.b * S + I.split * chunk;
     }
+    return I;
+  };
+  // Items come from a global counter.  The atomic for the next item is issued
+  // as soon as the current one starts; its result (held by lane 0) is only
+  // read when the producer side or the next item needs it, so its latency
+  // hides behind the current item's pieces.
+  int raw_next = lane == 0 ? atomicAdd(p.counter, 1) : 0;
+  Item cur = decode_item(__shfl_sync(0xffffffffu, raw_next, 0));
+  if (lane == 0 && cur.it < n_items) raw_next = atomicAdd(p.counter, 1);
+  Item nxt{n_items, 0, 0, 0, 0, 0};
+  bool nxt_ready = cur.it >= n_items;
+  auto ensure_next = [&]() {
+    if (!nxt_ready) {
+      nxt = decode_item(__shfl_sync(0xffffffffu, raw_next, 0));
+      nxt_ready = true;
+    }
+  };
+  int kc = 0;  // items started by this warp (q slot parity)
+
+  // producer side (lane 0 issues): up to RS pieces ahead, at most one item ahead
+  int p_sel = 0, p_r0 = 0;        // issuing from cur (0) or nxt (1), next row
+  int pc_issue = 0, pc_cons = 0;  // pieces issued / consumed
+  auto issue = [&]() {
+    while (pc_issue - pc_cons < RS) {
+      if (p_sel == 1) ensure_next();
+      const Item& I = p_sel == 0 ? cur : nxt;
+      if (I.it >= n_items) break;
+      if (p_r0 >= I.n) {
+        if (p_sel == 0) { p_sel = 1; p_r0 = 0; continue; }
+        break;
+      }
+      if (lane == 0) {
+        const int st = pc_issue % RS;
+        uint8_t* base = wsm + st * Geo::STAGE_BYTES;
+        // The warp's reads of this stage and of the q slot completed before
+        // the __syncwarp that preceded this call (their values are in
+        // registers), so the asynchronous writes may reuse the space.
+        mbar_expect_tx(full + st, Geo::STAGE_BYTES + (p_r0 == 0 ? Geo::Q_BYTES : 0));
+        if (p_r0 == 0)  // the item's G query rows (contiguous) ride with its first piece
+          bulk_load(wsm + Geo::OFF_Q + ((kc + p_sel) & 1) * Geo::Q_BYTES,
+                    static_cast<const __nv_bfloat16*>(p.q) + ((long long)I.b * p.Hq + I.kvh * G) * D,
+                    Geo::Q_BYTES, full + st);
+        const int row0 = I.row0 + p_r0;  // rows past the split are unused
+        tma_load_3d(base, &tmap_k, full + st, 0, I.kvh, row0);
+        tma_load_3d(base + Geo::PIECE_BYTES, &tmap_v, full + st, 0, I.kvh, row0);
+      }
+      p_r0 += R;
+      ++pc_issue;
+    }
+  };
+
+  const int grp = lane / LPR, gl = lane % LPR;
+  const int c0 = gl * 8;
+  float* sc_s = reinterpret_cast<float*>(wsm + Geo::OFF_SC) + grp * V;                // scores
+  float* sc_p = reinterpret_cast<float*>(wsm + Geo::OFF_SC) + (Geo::NGW + grp) * V;   // probabilities
+  const float scale_log2 = p.scale * kLog2e;
+  bool ok = true;
+  while (cur.it < n_items && ok) {
+    const int split = cur.split, kvh = cur.kvh, b = cur.b, n_cur = cur.n;
+    float2 qv[G][4];
     float2 acc[G][4];
     float m_run[G], l_run[G];
 #pragma unroll
@@ -357,11 +460,24 @@ __global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
     }
-    for (int r0 = 0; r0 < n; r0 += kPieceRows, ++pc) {
-      const int st = pc % kStreamStages;
-      const int rows = min(kPieceRows, n - r0);
-      if (!mbar_wait(full + st, (pc / kStreamStages) & 1, &abort_s, p.status)) return;
-      const uint8_t* kbuf = sm + st * Geo::STAGE_BYTES;
+    issue();
+    for (int r0 = 0; r0 < n_cur; r0 += R) {
+      const int st = pc_cons % RS;
+      ok = __all_sync(0xffffffffu, mbar_wait(full + st, (pc_cons / RS) & 1, &abort_s, p.status));
+      if (!ok) break;
+      const int rows = min(R, n_cur - r0);
+      if (r0 == 0) {
+        const __nv_bfloat16* qs =
+            reinterpret_cast<const __nv_bfloat16*>(wsm + Geo::OFF_Q + (kc & 1) * Geo::Q_BYTES);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float2 t[4];
+          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(qs + h * D + c0), t);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) qv[h][i] = make_float2(t[i].x * scale_log2, t[i].y * scale_log2);
+        }
+      }
+      const uint8_t* kbuf = wsm + st * Geo::STAGE_BYTES;
       const uint8_t* vbuf = kbuf + Geo::PIECE_BYTES;
       // scores of this group's PR rows for all G heads
       float v[V];
@@ -369,7 +485,7 @@ __global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
       for (int rr = 0; rr < PR; ++rr) {
         const int r = grp * PR + rr;
         float2 kf[4];
-        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(kbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), kf);
+        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(kbuf + r * Geo::ROW_BYTES + c0 * 2), kf);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float2 a = __fmul2_rn(qv[h][0], kf[0]);
@@ -420,7 +536,7 @@ __global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
         const int r = grp * PR + rr;
         if (r < rows) {
           float2 vf[4];
-          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(vbuf + hf * Geo::HALF_BYTES + r * 128 + cin * 2), vf);
+          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(vbuf + r * Geo::ROW_BYTES + c0 * 2), vf);
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float pr = sc_p[rr * G + h];
@@ -431,10 +547,12 @@ __global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
           }
         }
       }
-      __syncwarp();  // every lane of the warp is done with the stage and the scratch
-      if (lane == 0) mbar_arrive(empty + st);
+      __syncwarp();  // every lane is done with the stage and the scratch
+      ++pc_cons;
+      issue();       // refill the freed stage
     }
-    // merge the groups of a warp (lanes gl and gl + LPR, ...) with max rescaling
+    if (!ok) break;
+    // merge the warp's groups (lanes gl, gl + LPR, ...) with max rescaling
 #pragma unroll
     for (int o = 16; o >= LPR; o >>= 1) {
 #pragma unroll
@@ -442,8 +560,8 @@ __global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
         const float mo = __shfl_xor_sync(0xffffffffu, m_run[h], o);
         const float lo = __shfl_xor_sync(0xffffffffu, l_run[h], o);
         const float mm = fmaxf(m_run[h], mo);
-        const float fa = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mm);
-        const float fb = (mo == -INFINITY) ? 0.f : exp2f(mo - mm);
+        const float fa = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - mm);
+        const float fb = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mm);
         l_run[h] = l_run[h] * fa + lo * fb;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -454,89 +572,67 @@ __global__ void __maxnreg__(stream_regs<G>()) decode_stream_kernel(
         m_run[h] = mm;
       }
     }
+    // the split's partial of every query head: [b][kvh G + h][split][D + 2]
     if (lane < LPR) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
+        // rows of D + 2 floats are only 8-byte aligned: float2 stores
+        float* part = p.part + (((long long)b * p.Hq + kvh * G + h) * p.num_splits + split) * (D + 2);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          red[(warp * G + h) * D + c0 + 2 * i] = acc[h][i].x;
-          red[(warp * G + h) * D + c0 + 2 * i + 1] = acc[h][i].y;
-        }
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<float2*>(part + c0 + 2 * i) = acc[h][i];
         if (gl == 0) {
-          ml[(warp * G + h) * 2] = m_run[h];
-          ml[(warp * G + h) * 2 + 1] = l_run[h];
+          part[D] = n_cur > 0 ? m_run[h] : -INFINITY;
+          part[D + 1] = n_cur > 0 ? l_run[h] : 0.f;
         }
       }
     }
-    named_bar_sync(1, kConsumerThreads);
-    // merge the warps (fixed order) and write the split's partial
-    float* part = p.part + (((long long)b * p.Hq + kvh * G) * p.num_splits + split) * (D + 2);
-    for (int i = tid; i < G * D; i += kConsumerThreads) {
-      const int h = i / D, d = i % D;
-      float mm = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) mm = fmaxf(mm, ml[(w * G + h) * 2]);
-      float sacc = 0.f, sl = 0.f;
-      if (mm != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = ml[(w * G + h) * 2];
-          if (mw == -INFINITY) continue;
-          const float f = exp2f(mw - mm);
-          sacc += red[(w * G + h) * D + d] * f;
-          sl += ml[(w * G + h) * 2 + 1] * f;
-        }
-      }
-      part[(long long)h * p.num_splits * (D + 2) + d] = sacc;
-      if (d == 0) {
-        part[(long long)h * p.num_splits * (D + 2) + D] = n > 0 ? mm : -INFINITY;
-        part[(long long)h * p.num_splits * (D + 2) + D + 1] = n > 0 ? sl : 0.f;
-      }
+    // next item; the producer side may already be streaming it
+    ensure_next();
+    cur = nxt;
+    ++kc;
+    if (p_sel == 1) {
+      p_sel = 0;
+    } else {
+      p_sel = 0;
+      p_r0 = 0;
     }
-    named_bar_sync(1, kConsumerThreads);  // red / ml reused by the next item
+    nxt_ready = cur.it >= n_items;
+    if (lane == 0 && !nxt_ready) raw_next = atomicAdd(p.counter, 1);
+  }
+  // leave no copy in flight: wait for every issued piece
+  if (!ok) {
+    for (; pc_cons < pc_issue; ++pc_cons) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(full + pc_cons % RS, (pc_cons / RS) & 1))
+        if (clock64() - t0 > kWaitBudgetCycles) break;
+    }
   }
 }
 
-// Merge splits + sink.  One CTA per (head, sequence), D threads.
+// Merge splits + sink: one warp per (sequence, query head).
 template <typename T, int D>
-__global__ void decode_combine_kernel(DecodeProblem p, int n_splits) {
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const float* part = p.part + ((long long)b * p.Hq + h) * n_splits * (D + 2);
-  const float a2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-  float mt = a2;
-  for (int i = 0; i < n_splits; ++i) mt = fmaxf(mt, part[i * (D + 2) + D]);
-  float l = 0.f, o = 0.f;
-  if (mt != -INFINITY) {
-    for (int i = 0; i < n_splits; ++i) {
-      const float mi = part[i * (D + 2) + D];
-      if (mi == -INFINITY) continue;
-      const float w = exp2f(mi - mt);
-      l += part[i * (D + 2) + D + 1] * w;
-      o += part[i * (D + 2) + d] * w;
-    }
-  }
-  const float den = l + (p.sink && mt != -INFINITY ? exp2f(a2 - mt) : 0.f);
-  const long long row = (long long)b * p.Hq + h;
-  const float ov = den > 0.f ? o / den : 0.f;
-  if constexpr (sizeof(T) == 2)
-    static_cast<__nv_bfloat16*>(p.out)[row * D + d] = __float2bfloat16_rn(ov);
-  else
-    static_cast<float*>(p.out)[row * D + d] = ov;
-  if (d == 0) {
-    p.lse[row] = den > 0.f ? (mt + log2f(den)) * kLn2 : -INFINITY;
-    if (p.sink_s) p.sink_s[row] = den > 0.f ? l / den : 0.f;
-  }
+__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeProblem p) {
+  const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= p.B * p.Hq) return;
+  combine_head<T, D>(p, w / p.Hq, w % p.Hq, threadIdx.x & 31);
+}
+
+template <typename T, int D>
+int launch_combine(const DecodeProblem& p, cudaStream_t stream) {
+  const int warps = p.B * p.Hq;
+  decode_combine_kernel<T, D><<<(warps + 7) / 8, 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
 template <int D, int G>
 int launch_tma(const DecodeProblem& p, int chunk, cudaStream_t stream) {
-  using Geo = StreamGeom<D, G>;
+  using Geo = WarpGeom<D, G>;
   const int S = p.n_sink + p.window;
   CUtensorMap mk, mv;
-  if (!make_tmap_3d_plain(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, kPieceRows) ||
-      !make_tmap_3d_plain(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, kPieceRows))
+  if (!make_tmap_3d_rows(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, Geo::R) ||
+      !make_tmap_3d_rows(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, Geo::R))
     return SINKATTN_ERR_CUDA;
-  auto kern = decode_stream_kernel<D, G>;
+  auto kern = decode_warp_kernel<D, G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
@@ -544,13 +640,13 @@ int launch_tma(const DecodeProblem& p, int chunk, cudaStream_t stream) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_items = p.B * p.Hkv * p.num_splits;
-  const int grid = n_items < sms ? n_items : sms;
+  const int want = (n_items + kDecWarps - 1) / kDecWarps;
+  const int grid = want < sms ? want : sms;
+  if (cudaMemsetAsync(p.counter, 0, sizeof(int), stream) != cudaSuccess) return SINKATTN_ERR_CUDA;
   record_start(SINKATTN_KERNEL_DECODE, stream);
-  kern<<<grid, Geo::kConsumerThreads + 32, Geo::SMEM, stream>>>(mk, mv, p, chunk, n_items);
+  kern<<<grid, kDecWarps * 32, Geo::SMEM, stream>>>(mk, mv, p, chunk, n_items);
   record_stop(SINKATTN_KERNEL_DECODE, stream);
-  dim3 g2(p.Hq, p.B);
-  decode_combine_kernel<__nv_bfloat16, D><<<g2, D, 0, stream>>>(p, p.num_splits);
-  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+  return launch_combine<__nv_bfloat16, D>(p, stream);
 }
 
 template <typename T, int D, int G>
@@ -566,9 +662,8 @@ int launch_split(const DecodeProblem& p, int chunk, cudaStream_t stream) {
   record_start(SINKATTN_KERNEL_DECODE, stream);
   kern<<<grid, kDecThreads, smem, stream>>>(p, chunk);
   record_stop(SINKATTN_KERNEL_DECODE, stream);
-  dim3 g2(p.Hq, p.B);
-  decode_combine_kernel<T, D><<<g2, D, 0, stream>>>(p, p.num_splits);
-  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return SINKATTN_ERR_CUDA;
+  return launch_combine<T, D>(p, stream);
 }
 
 template <typename T, int D>
@@ -586,7 +681,9 @@ int dispatch_g(const DecodeProblem& p, int chunk, cudaStream_t stream) {
 
 int launch_decode(const DecodeProblem& p, cudaStream_t stream) {
   const int S = p.n_sink + p.window;
-  const int chunk = (S + p.num_splits - 1) / p.num_splits;
+  // slots per split, rounded up to whole 16-row pieces (trailing splits may
+  // then be empty; their partials carry m = -inf and drop out of the merge)
+  const int chunk = ((S + p.num_splits - 1) / p.num_splits + 15) / 16 * 16;
   if (p.dt == SINKATTN_BF16)
     return p.D == 64 ? dispatch_g<__nv_bfloat16, 64>(p, chunk, stream)
                      : dispatch_g<__nv_bfloat16, 128>(p, chunk, stream);

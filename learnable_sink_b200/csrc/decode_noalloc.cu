@@ -62,7 +62,8 @@ extern "C" int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv
   float* scratch = scratch_on_current_device();
   if (!scratch) return SINKATTN_ERR_CUDA;
   // Every entry of the partials is written by the split kernel before the
-  // combine kernel reads it, so nothing needs clearing between calls.
+  // combine kernel reads it, and the decode resets its work counter itself,
+  // so nothing needs clearing between calls.
   return sinkattn_decode(dt, B, Hq, Hkv, D, scale, q, k_cache, v_cache, cache_seqlens, n_sink,
                          window, learnable_sink, out, lse_new, sink_s, num_splits, scratch,
                          capacity, stream);

@@ -52,6 +52,8 @@ struct AttnProblem {
 bool make_tmap_3d(CUtensorMap* map, const void* base, int T, int H, int D, int box_h, int box_t);
 bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
                       int box_t);
+bool make_tmap_3d_rows(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
+                       int box_t);
 bool make_tmap_3d_plain(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
                         int box_t);
 
@@ -97,6 +99,7 @@ struct DecodeProblem {
   float* lse;
   float* sink_s;
   float* part;  // workspace: [B, Hq, splits, D + 2] floats
+  int* counter; // workspace: work-item counter of the streaming kernel (zeroed per call)
   int* status;
 };
 int launch_decode(const DecodeProblem& p, cudaStream_t stream);
