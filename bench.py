@@ -420,7 +420,9 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2,
                 "what": "pinned-host q,k,v,dO,sink -> device, plan+fwd+bwd, dsink -> host"},
-        "gpu_launches": K * (9 + 1 + 4 + 2),
+        # per step: plan 12, forward 1, backward 6 (preprocess, dsink reduce,
+        # split-tile zero/finish, tensor-core kernel, dQ convert), decode 2
+        "gpu_launches": K * (12 + 1 + 6 + 2),
         "roofline": {"kernel": "bwd_tc_kernel (dK/dV/dQ)", "bound": "tensor",
                      "achieved": bwd_ach, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": bwd_ach / peak_tf, "traffic": traffic,

@@ -92,7 +92,7 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[QR]
   static constexpr int OFF_DL = OFF_LSE + 512;            // float[QR]
   static constexpr int OFF_BAR = OFF_DL + 512;
-  static constexpr int N_BARS = 1 + 3 * NS + 7;
+  static constexpr int N_BARS = 1 + 6 * NS + 7;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
@@ -140,6 +140,9 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -161,10 +164,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;
-  uint64_t* bar_qf = bars + 1;
-  uint64_t* bar_qe = bar_qf + NS;
-  uint64_t* bar_dqs = bar_qe + NS;   // dQ tile of stage s staged in smem
-  uint64_t* bar_s = bar_dqs + NS;
+  // Each stage is two buffers, Q and dO, with their own barriers: the dQ tile
+  // is staged as columns [0, D/2) in the Q buffer and [D/2, D) in the dO
+  // buffer, and each buffer goes back to the producer as soon as the bulk
+  // reduction has read its half.
+  uint64_t* bar_qf = bars + 1;       // Q of stage s landed
+  uint64_t* bar_df = bar_qf + NS;    // dO of stage s landed
+  uint64_t* bar_qe = bar_df + NS;    // Q buffer of stage s free
+  uint64_t* bar_de = bar_qe + NS;    // dO buffer of stage s free
+  uint64_t* bar_dqs = bar_de + NS;   // dQ half 0 of stage s staged in the Q buffer
+  uint64_t* bar_dds = bar_dqs + NS;  // dQ half 1 of stage s staged in the dO buffer
+  uint64_t* bar_s = bar_dds + NS;
   uint64_t* bar_dp = bar_s + 1;
   uint64_t* bar_p = bar_dp + 1;
   uint64_t* bar_ds = bar_p + 1;
@@ -198,8 +208,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(bar_kv, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_qf + s, 1);
+      mbar_init(bar_df + s, 1);
       mbar_init(bar_qe + s, 1);    // released by the reducer warp
-      mbar_init(bar_dqs + s, 128); // every epilogue thread staged its dQ part
+      mbar_init(bar_de + s, 1);
+      mbar_init(bar_dqs + s, 128); // every epilogue thread staged its part of the half
+      mbar_init(bar_dds + s, 128);
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
@@ -243,29 +256,36 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tma_load_3d(smem + C::OFF_K + h * (C::KV_BYTES / DH), &tmap_k, bar_kv, h * 64, kvh, krow);
           tma_load_3d(smem + C::OFF_V + h * (C::KV_BYTES / DH), &tmap_v, bar_kv, h * 64, kvh, krow);
         }
-        int last[NS];
-        for (int s = 0; s < NS; ++s) last[s] = -1;
+        int last[NS], lastd[NS];  // last iteration loaded into each Q / dO buffer
+        for (int s = 0; s < NS; ++s) last[s] = lastd[s] = -1;
         bool ok = true;
         for (int i = 0; i < n_it && ok; ++i) {
           const int s = i % NS;
           const int e = __ldg(ent + i / PER_E);
           const int q_tok = it.seq_start + q_first(i, e);
           const int h0 = h_first(i);
-          ok = mbar_wait(bar_qe + s, ((i / NS) & 1) ^ 1, abort_flag, p.status);
+          const uint32_t par = ((i / NS) & 1) ^ 1;
+          ok = mbar_wait(bar_qe + s, par, abort_flag, p.status);
           if (!ok) break;
-          mbar_expect_tx(bar_qf + s, 2 * C::Q_BYTES);
-          for (int h = 0; h < DH; ++h) {
+          mbar_expect_tx(bar_qf + s, C::Q_BYTES);
+          for (int h = 0; h < DH; ++h)
             tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_q,
                         bar_qf + s, h * 64, h0, q_tok);
-            tma_load_3d(smem + C::OFF_DO + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_do,
-                        bar_qf + s, h * 64, h0, q_tok);
-          }
           last[s] = i;
+          ok = mbar_wait(bar_de + s, par, abort_flag, p.status);
+          if (!ok) break;
+          mbar_expect_tx(bar_df + s, C::Q_BYTES);
+          for (int h = 0; h < DH; ++h)
+            tma_load_3d(smem + C::OFF_DO + s * C::Q_BYTES + h * (C::Q_BYTES / DH), &tmap_do,
+                        bar_df + s, h * 64, h0, q_tok);
+          lastd[s] = i;
         }
         if (!ok) {
           wait_noabort(bar_kv, 0);
-          for (int s = 0; s < NS; ++s)
+          for (int s = 0; s < NS; ++s) {
             if (last[s] >= 0) wait_noabort(bar_qf + s, (last[s] / NS) & 1);
+            if (lastd[s] >= 0) wait_noabort(bar_df + s, (lastd[s] / NS) & 1);
+          }
         }
       }
     } else if (warp == C::MMA_WARP) {
@@ -290,7 +310,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           mma_commit(bar_s);
         };
-        // dP^T = V dO^T of iteration j
+        // dP^T = V dO^T of iteration j (its dO tile has landed)
         auto issue_dp = [&](int j) {
           const uint32_t do_s = sDO + (j % NS) * C::Q_BYTES;
 #pragma unroll
@@ -308,7 +328,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (ok) {
           tc_fence_after();
           issue_s(0);
-          issue_dp(0);
+          ok = mbar_wait(bar_df, 0, abort_flag, p.status);
+          tc_fence_after();
+          if (ok) issue_dp(0);
         }
         for (int i = 0; i < n_it && ok; ++i) {
           const int s = i % NS;
@@ -364,8 +386,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (!C::DQ_OWN) {  // dP^T(i+1) overwrites the dQ tile
               ok = mbar_wait(bar_dqf, i & 1, abort_flag, p.status);
               if (!ok) break;
-              tc_fence_after();
             }
+            ok = mbar_wait(bar_df + s1, par1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
             issue_dp(i + 1);
           }
         }
@@ -380,21 +404,27 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (lane == 0 && n_it > 0) {
         for (int i = 0; i < n_it; ++i) {
           const int s = i % NS;
-          if (!mbar_wait(bar_dqs + s, (i / NS) & 1, abort_flag, p.status)) break;
           const int e = __ldg(ent + i / PER_E);
           const int q_tok = it.seq_start + q_first(i, e);
           const int h0 = h_first(i);
+          const uint32_t par = (i / NS) & 1;
+          bool got = true;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+          for (int half = 0; half < 2 && got; ++half) {
+            got = mbar_wait((half == 0 ? bar_dqs : bar_dds) + s, par, abort_flag, p.status);
+            if (!got) break;
             const uint8_t* stage = smem + (half == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
               tma_reduce_add_3d(&tmap_dq, stage + c * (QR * 128), (D / 2) * half + 32 * c, h0,
                                 q_tok);
+            bulk_commit();
           }
-          bulk_commit();
-          bulk_wait_read0();
+          if (!got) break;
+          bulk_wait_read1();         // the Q-buffer half has been read
           mbar_arrive(bar_qe + s);
+          bulk_wait_read0();         // the dO-buffer half too
+          mbar_arrive(bar_de + s);
         }
         bulk_wait0();  // reductions complete before the CTA exits
       }
@@ -434,9 +464,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
                 make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
         }
+        if (c == D / 64 - 1) {  // a half is staged: the reducer warp takes it from here
+          fence_async_smem();
+          mbar_arrive((half == 0 ? bar_dqs : bar_dds) + s);
+        }
       }
-      fence_async_smem();
-      mbar_arrive(bar_dqs + s);  // the reducer warp takes it from here
     }
   } else {
     // ------------------------------------------------------------ compute
@@ -592,7 +624,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       bool free_ok = true;
       for (int s = 0; s < NS && s < n_it; ++s) {
         const int last = s + ((n_it - 1 - s) / NS) * NS;  // last iteration on stage s
-        free_ok = free_ok && mbar_wait(bar_qe + s, (last / NS) & 1, abort_flag, p.status);
+        free_ok = free_ok && mbar_wait((cw == 0 ? bar_qe : bar_de) + s, (last / NS) & 1, abort_flag,
+                                       p.status);
       }
       free_ok = __all_sync(0xffffffffu, free_ok);
       tc_fence_after();
