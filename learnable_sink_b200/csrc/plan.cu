@@ -289,7 +289,8 @@ __global__ void plan_bwd_init_kernel(PlanArgs a) {
 
 // F: scatter forward entries into the reverse lists.
 __global__ void plan_bwd_scatter_kernel(PlanArgs a) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  // one warp per forward item, lanes over its entries
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (i >= a.cap_items) return;
   const TileItem it = reinterpret_cast<const TileItem*>(a.plan + a.off_fwd_items)[i];
   if (it.entry_len <= 0 || it.entry_off + it.entry_len > a.cap_entries) return;
@@ -301,7 +302,7 @@ __global__ void plan_bwd_scatter_kernel(PlanArgs a) {
   const TileItem* bitems = reinterpret_cast<const TileItem*>(a.plan + a.off_bwd_items);
   int* cursor = a.plan + a.off_bwd_cursor;
   int* bent = a.plan + a.off_bwd_entries;
-  for (int e = 0; e < it.entry_len; ++e) {
+  for (int e = lane; e < it.entry_len; e += 32) {
     const int kt = ent[e] >> 1, partial = ent[e] & 1;
     const int b = kh * a.cap_tiles + tile_base[s] + kt;
     const int pos = bitems[b].entry_off + atomicAdd(&cursor[b], 1);
@@ -387,6 +388,20 @@ __global__ void plan_bwd_sort_kernel(PlanArgs a) {
   const TileItem it = reinterpret_cast<const TileItem*>(a.plan + a.off_bwd_items)[i];
   if (it.entry_len <= 1 || it.entry_off + it.entry_len > a.cap_entries) return;
   int* e = a.plan + a.off_bwd_entries + it.entry_off;
+  constexpr int kLocal = 64;
+  if (it.entry_len <= kLocal) {
+    // short list: sort a private copy (L1-resident), then write it back once
+    int w[kLocal];
+    for (int x = 0; x < it.entry_len; ++x) w[x] = e[x];
+    for (int x = 1; x < it.entry_len; ++x) {
+      const int v = w[x];
+      int p = x;
+      while (p > 0 && w[p - 1] < v) { w[p] = w[p - 1]; --p; }
+      w[p] = v;
+    }
+    for (int x = 0; x < it.entry_len; ++x) e[x] = w[x];
+    return;
+  }
   for (int x = 1; x < it.entry_len; ++x) {
     const int v = e[x];
     int p = x;
@@ -461,7 +476,7 @@ int launch_plan(const PlanLaunch& L, cudaStream_t stream) {
   plan_fwd_fill_kernel<<<nb, 256, 0, stream>>>(a);
   plan_offsets_kernel<<<1, kScanThreads, 0, stream>>>(a, 1);
   plan_zero_kernel<<<nb, 256, 0, stream>>>(a.plan + a.off_bwd_cursor, z.cap_items);
-  plan_bwd_scatter_kernel<<<nb, 256, 0, stream>>>(a);
+  plan_bwd_scatter_kernel<<<(unsigned)(((long long)z.cap_items * 32 + 255) / 256), 256, 0, stream>>>(a);
   plan_bwd_sort_kernel<<<nb, 256, 0, stream>>>(a);
   plan_units_scan_kernel<<<1, kScanThreads, 0, stream>>>(a);
   plan_units_fill_kernel<<<nb, 256, 0, stream>>>(a);
