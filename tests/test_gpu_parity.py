@@ -250,6 +250,21 @@ def test_decode_partial_fill_and_splits(splits):
     _compare_decode(d, *_run_decode(d, splits), TOL[torch.bfloat16])
 
 
+@pytest.mark.parametrize("G,D,splits", [(8, 128, 0), (8, 64, 5), (1, 128, 40), (2, 64, 97)])
+def test_decode_heads_and_many_splits(G, D, splits):
+    # 40 and 97 splits put several rounds of split partials in the merge
+    # (32 per warp pass); 8 query heads per KV head use the 8-row pieces
+    d = W.decode(B=5, n_sink=4, window=1500, Hq=2 * G, Hkv=2, D=D, seqlen_range=(0, 3000))
+    _compare_decode(d, *_run_decode(d, splits), TOL[torch.bfloat16])
+
+
+def test_decode_many_sequences():
+    # more sequences than the streaming kernel stages cache lengths for in
+    # shared memory (1024): the lengths are then read from global memory
+    d = W.decode(B=1100, n_sink=2, window=30, Hq=2, Hkv=1, D=64, seqlen_range=(0, 40))
+    _compare_decode(d, *_run_decode(d), TOL[torch.bfloat16])
+
+
 def test_decode_fp32_no_sink():
     d = W.decode(B=4, n_sink=2, window=40, Hq=4, Hkv=4, D=128, dtype=torch.float32,
                  seqlen_range=(1, 100), sink_std=None)
