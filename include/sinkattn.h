@@ -161,6 +161,18 @@ int sinkattn_fwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
                  void *out, float *lse_new, float *sink_s,
                  sinkattn_stream_t stream);
 
+/* ---- forward with the raw LSE ------------------------------------------------
+ * Same as sinkattn_fwd, plus lse_orig (float32 [T_tot, Hq], 16-byte aligned,
+ * or NULL): the log-sum-exp over the visible keys alone, before the sink joins
+ * the denominator -- page 1's L_orig (its source notes: the raw LSE is what
+ * goes to a teacher), from which page 4's gate sigma(LSE - sink) is formed.
+ * Rows with no visible key get -inf.  LSE_new = logaddexp(lse_orig, a_h) and
+ * sink_s = exp(lse_orig - lse_new) hold up to rounding. */
+int sinkattn_fwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                    const void *q, const void *k, const void *v, const float *learnable_sink,
+                    const sinkattn_mask *mask, const void *plan, size_t plan_bytes, void *out,
+                    float *lse_new, float *sink_s, float *lse_orig, sinkattn_stream_t stream);
+
 /* ---- backward -------------------------------------------------------------
  * Computes dQ, dK, dV and dsink (page 1 sections 7-8).
  *   out, lse_new  the forward's O and LSE_new (sink-inclusive).
@@ -211,6 +223,39 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
                     float *sink_s, int num_splits, void *workspace,
                     size_t workspace_bytes, sinkattn_stream_t stream);
 
+/* ---- ring-cache maintenance -------------------------------------------------
+ * Page "Attention Sink / StreamingLLM" (the core-idea section): the cache
+ * keeps a sequence's first n_sink tokens in fixed slots and its most recent
+ * `window` tokens in a circular segment, each new token overwriting the oldest
+ * non-sink one.  Slot rule, the same as sinkattn_decode's: position
+ * p < n_sink -> slot p, otherwise n_sink + (p - n_sink) % window.  Caches are
+ * [B, S, Hkv, D] of type dt, S = n_sink + window, updated in place.
+ *
+ * sinkattn_cache_append -- one new token per sequence.
+ *   k_new, v_new   [B, Hkv, D] of type dt: the token being appended.
+ *   cache_seqlens  device int32 [B]: tokens ever appended, this one included
+ *                  (the caller increments it first, as for decode), so the
+ *                  token sits at position cache_seqlens[b] - 1; entries <= 0,
+ *                  and positions past the sink segment when window = 0, write
+ *                  nothing.
+ * sinkattn_cache_fill -- a prefill's tokens into caches, one per sequence.
+ *   cu_seqlens     device int32 [n_seq + 1]: sequence s is tokens
+ *                  [cu_seqlens[s], cu_seqlens[s + 1]) of the packed
+ *                  k, v [T_tot, Hkv, D] (type dt).
+ *   Every token that survives in the ring -- one of the first n_sink, or one
+ *   of the last `window` past them -- is written to its slot of sequence s;
+ *   the other slots are left as they are.
+ *   cache_seqlens_out  device int32 [n_seq] or NULL: receives each length.
+ * Both: D in {64, 128}, dt BF16 or FP32, 16-byte aligned pointers (else
+ * SINKATTN_ERR_INVALID_ARG); launch failures return SINKATTN_ERR_CUDA. */
+int sinkattn_cache_append(sinkattn_dtype dt, int B, int Hkv, int D, int n_sink, int window,
+                          const void *k_new, const void *v_new, const int32_t *cache_seqlens,
+                          void *k_cache, void *v_cache, sinkattn_stream_t stream);
+int sinkattn_cache_fill(sinkattn_dtype dt, int n_seq, int T_tot, int Hkv, int D, int n_sink,
+                        int window, const int32_t *cu_seqlens, const void *k, const void *v,
+                        void *k_cache, void *v_cache, int32_t *cache_seqlens_out,
+                        sinkattn_stream_t stream);
+
 /* ---- ring-buffer decode without caller scratch ------------------------------
  * No counterpart on the pages: this is a service for callers of this library.
  * Same computation, arguments and results as sinkattn_decode, minus the
@@ -221,7 +266,8 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
  * input and output buffers.  The per-split partials go to a fixed 4 MiB array
  * in the library's device image (every GPU that loads the library keeps it
  * until the process exits); nothing is allocated.
- *   - Limit: B * Hq * num_splits * (D + 2) * 4 bytes must fit in 4 MiB.  With
+ *   - Limit: B * Hq * num_splits * (D + 2) * 4 bytes (rounded up to 256) plus
+ *     256 bytes for a work counter must fit in 4 MiB.  With
  *     num_splits = 0 the automatic split count is lowered until it fits;
  *     a problem that does not fit even with one split, or an explicit
  *     num_splits that does not fit, returns SINKATTN_ERR_WORKSPACE and

@@ -191,12 +191,22 @@ int sinkattn_fwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
                  const void* q, const void* k, const void* v, const float* learnable_sink,
                  const sinkattn_mask* mask, const void* plan, size_t plan_bytes, void* out,
                  float* lse_new, float* sink_s, sinkattn_stream_t stream) {
+  return sinkattn_fwd_ex(dt, T_tot, Hq, Hkv, D, scale, q, k, v, learnable_sink, mask, plan,
+                         plan_bytes, out, lse_new, sink_s, nullptr, stream);
+}
+
+int sinkattn_fwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                    const void* q, const void* k, const void* v, const float* learnable_sink,
+                    const sinkattn_mask* mask, const void* plan, size_t plan_bytes, void* out,
+                    float* lse_new, float* sink_s, float* lse_orig, sinkattn_stream_t stream) {
   AttnProblem p{};
   int rc = attn_common(dt, T_tot, Hq, Hkv, D, q, k, v, learnable_sink, mask, plan, plan_bytes, &p);
   if (rc != SINKATTN_OK) return rc;
-  if (!out || !lse_new || !aligned16(out) || !aligned16(lse_new) || (sink_s && !aligned16(sink_s)))
+  if (!out || !lse_new || !aligned16(out) || !aligned16(lse_new) || (sink_s && !aligned16(sink_s)) ||
+      (lse_orig && !aligned16(lse_orig)))
     return SINKATTN_ERR_INVALID_ARG;
   p.scale = scale;
+  p.lse_orig = lse_orig;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dt == SINKATTN_FP32) return launch_fwd_simt(p, out, lse_new, sink_s, s);
   return launch_fwd_tc(p, out, lse_new, sink_s, s);

@@ -73,6 +73,7 @@ struct FwdParams {
   __nv_bfloat16* out;
   float* lse;
   float* sink_s;
+  float* lse_orig;  // or nullptr
   int* status;
   int Hq, Hkv, G, causal, n_sink, window;
   int per_item, chunks;  // CTAs per plan item, head chunks per KV head
@@ -357,6 +358,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
       p.lse[row] = lse_v;
       if (p.sink_s) p.sink_s[row] = ss;
+      // the raw LSE over the visible keys (before the sink joins)
+      if (p.lse_orig) p.lse_orig[row] = (m != -INFINITY && l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
       uint4* dst = reinterpret_cast<uint4*>(p.out + row * D);
       if (!have_o) {
         const uint4 z = make_uint4(0, 0, 0, 0);
@@ -497,6 +500,7 @@ int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaS
   fp.out = static_cast<__nv_bfloat16*>(out);
   fp.lse = lse;
   fp.sink_s = sink_s;
+  fp.lse_orig = p.lse_orig;
   fp.status = p.status;
   fp.Hq = p.Hq;
   fp.Hkv = p.Hkv;

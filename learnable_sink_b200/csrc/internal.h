@@ -47,6 +47,7 @@ struct AttnProblem {
   const int* plan;    // device plan words
   PlanSizes ps;
   int* status;
+  float* lse_orig;    // forward: [T_tot, Hq] LSE over the visible keys only, or nullptr
 };
 
 bool make_tmap_3d(CUtensorMap* map, const void* base, int T, int H, int D, int box_h, int box_t);

@@ -28,6 +28,7 @@ struct SimtArgs {
   int Hq, Hkv, causal, n_sink, window, tile, T_tot;
   float scale_log2;  // alpha * log2(e)
   int* status;
+  float* lse_orig;   // or nullptr
 };
 
 template <int D>
@@ -93,6 +94,8 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_simt_kernel(SimtArgs a, float
     if (lane == 0) {
       lse[row] = lse_v;
       if (sink_s) sink_s[row] = ss;
+      // the raw LSE over the visible keys (before the sink joins)
+      if (a.lse_orig) a.lse_orig[row] = (m != -INFINITY && l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
   }
 }
@@ -233,6 +236,7 @@ SimtArgs make_args(const AttnProblem& p) {
   a.T_tot = p.T_tot;
   a.scale_log2 = p.scale * kLog2e;
   a.status = p.status;
+  a.lse_orig = p.lse_orig;
   return a;
 }
 

@@ -61,6 +61,8 @@ def lib():
         L.sinkattn_plan.argtypes = [_i, _i, _i, M, _vp, _sz, _vp]
         L.sinkattn_fwd.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, M, _vp, _sz,
                                    _vp, _vp, _vp, _vp]
+        L.sinkattn_fwd_ex.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, M, _vp,
+                                      _sz, _vp, _vp, _vp, _vp, _vp]
         L.sinkattn_bwd_workspace_bytes.restype = _sz
         L.sinkattn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, M]
         L.sinkattn_bwd.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -70,6 +72,9 @@ def lib():
         L.sinkattn_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
         L.sinkattn_decode.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _i, _i,
                                       _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
+        L.sinkattn_cache_append.argtypes = [_i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.sinkattn_cache_fill.argtypes = [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp]
         L.sinkattn_set_kernel_events.argtypes = [_i, _vp, _vp]
         L.sinkattn_selftest_timeout.argtypes = [_vp]
         L.sinkattn_get_status.argtypes = [_vp]
@@ -169,8 +174,10 @@ def _contig(*ts):
 
 
 def fwd(q, k, v, sink, mask: Mask, plan: Plan, scale: Optional[float] = None, stream=None,
-        out=None, lse=None, sink_s=None):
-    """Forward.  Returns (out [T,Hq,D], lse_new [T,Hq] fp32, sink_s [T,Hq] fp32)."""
+        out=None, lse=None, sink_s=None, lse_orig=None):
+    """Forward.  Returns (out [T,Hq,D], lse_new [T,Hq] fp32, sink_s [T,Hq] fp32).
+    With ``lse_orig`` (fp32 [T,Hq]) also writes the LSE over the visible keys
+    alone, before the sink joins (sinkattn_fwd_ex)."""
     _contig(q, k, v, sink)
     T, Hq, D = q.shape
     Hkv = k.shape[1]
@@ -179,9 +186,16 @@ def fwd(q, k, v, sink, mask: Mask, plan: Plan, scale: Optional[float] = None, st
     lse = torch.empty(T, Hq, dtype=torch.float32, device=q.device) if lse is None else lse
     sink_s = torch.empty(T, Hq, dtype=torch.float32, device=q.device) if sink_s is None else sink_s
     cm = mask.c()
-    _check("sinkattn_fwd", lib().sinkattn_fwd(
-        _dt(q), T, Hq, Hkv, D, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(sink), _c.byref(cm),
-        _ptr(plan.buf), plan.nbytes, _ptr(out), _ptr(lse), _ptr(sink_s), _stream(stream)))
+    if lse_orig is None:
+        _check("sinkattn_fwd", lib().sinkattn_fwd(
+            _dt(q), T, Hq, Hkv, D, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(sink), _c.byref(cm),
+            _ptr(plan.buf), plan.nbytes, _ptr(out), _ptr(lse), _ptr(sink_s), _stream(stream)))
+    else:
+        _contig(lse_orig)
+        _check("sinkattn_fwd_ex", lib().sinkattn_fwd_ex(
+            _dt(q), T, Hq, Hkv, D, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(sink), _c.byref(cm),
+            _ptr(plan.buf), plan.nbytes, _ptr(out), _ptr(lse), _ptr(sink_s), _ptr(lse_orig),
+            _stream(stream)))
     return out, lse, sink_s
 
 
@@ -243,6 +257,29 @@ def decode(q, k_cache, v_cache, cache_seqlens, n_sink: int, window: int, sink,
         int(n_sink), int(window), _ptr(sink), _ptr(out), _ptr(lse), _ptr(sink_s), int(num_splits),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return out, lse, sink_s
+
+
+def cache_append(k_new, v_new, cache_seqlens, k_cache, v_cache, n_sink: int, window: int,
+                 stream=None) -> None:
+    """Write one new token per sequence (k_new/v_new [B, Hkv, D]) into its ring
+    slot; cache_seqlens [B] int32 already counts the new token."""
+    _contig(k_new, v_new, cache_seqlens, k_cache, v_cache)
+    B, Hkv, D = k_new.shape
+    _check("sinkattn_cache_append", lib().sinkattn_cache_append(
+        _dt(k_new), B, Hkv, D, int(n_sink), int(window), _ptr(k_new), _ptr(v_new),
+        _ptr(cache_seqlens), _ptr(k_cache), _ptr(v_cache), _stream(stream)))
+
+
+def cache_fill(k, v, cu_seqlens, k_cache, v_cache, n_sink: int, window: int,
+               cache_seqlens_out=None, stream=None) -> None:
+    """Write a packed prefill (k/v [T_tot, Hkv, D], sequences by cu_seqlens)
+    into the ring caches [n_seq, S, Hkv, D]; optionally store the lengths."""
+    _contig(k, v, cu_seqlens, k_cache, v_cache, cache_seqlens_out)
+    T, Hkv, D = k.shape
+    n_seq = cu_seqlens.numel() - 1
+    _check("sinkattn_cache_fill", lib().sinkattn_cache_fill(
+        _dt(k), n_seq, T, Hkv, D, int(n_sink), int(window), _ptr(cu_seqlens), _ptr(k), _ptr(v),
+        _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens_out), _stream(stream)))
 
 
 KERNEL_FWD, KERNEL_BWD, KERNEL_DECODE = 0, 1, 2

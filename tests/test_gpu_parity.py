@@ -342,3 +342,39 @@ def test_bf16_block_sparse_empty_rows_and_unselected_keys():
             unseen = vis[g].sum(0) == 0
             assert torch.all(grads[1].cpu()[torch.from_numpy(unseen), g].float() == 0)
             assert torch.all(grads[2].cpu()[torch.from_numpy(unseen), g].float() == 0)
+
+
+# ------------------------------------------------------------ raw LSE (before the sink)
+
+@pytest.mark.parametrize("dtype,block", [(torch.bfloat16, None), (torch.float32, None),
+                                         (torch.bfloat16, 64)])
+def test_forward_raw_lse_matches_sink_free_oracle(dtype, block):
+    # the raw LSE is the sink-free forward's LSE: checked against the oracle
+    # run without a sink (an independent route), and against the identities
+    # LSE_new = logaddexp(LSE_orig, a) and sink_s = exp(LSE_orig - LSE_new)
+    if block is None:
+        ms = spec([0, 300, 555], n_sink=4, window=200)
+        Hq, Hkv = 8, 2
+    else:
+        cu = W.random_cu_seqlens(900, 100, 500, 21)
+        bi = W.random_block_indices(cu, 2, block, block, 3, 22)
+        bi[:, ::7, :] = -1  # some query blocks select nothing: their rows see no key
+        ms = W.MaskSpec(causal=True, cu_seqlens=cu, block_indices=bi, block_q=block, block_k=block)
+        Hq, Hkv = 4, 2
+    T = int(ms.cu_seqlens[-1])
+    inp = W.make_attn("raw_lse", T_tot=T, Hq=Hq, Hkv=Hkv, D=64, dtype=dtype, mask=ms, seed=23)
+    m = S.Mask.from_spec(inp.mask)
+    plan = S.Plan(T, Hq, Hkv, m)
+    lse_orig = torch.empty(T, Hq, dtype=torch.float32, device="cuda")
+    out, lse, ss = S.fwd(dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.sink), m, plan,
+                         scale=inp.scale, lse_orig=lse_orig)
+    torch.cuda.synchronize()
+    _, rl0, _ = oracle.fwd(inp.q, inp.k, inp.v, None, inp.scale, **inp.mask.oracle_kwargs())
+    check_lse(np64(lse_orig), rl0, TOL[dtype]["lse"])
+    lo = np64(lse_orig)
+    a = inp.sink.double().numpy()[None, :]
+    fin = np.isfinite(lo)
+    assert np.abs(np.logaddexp(lo, a)[fin] - np64(lse)[fin]).max() <= 2 * TOL[dtype]["lse"]
+    assert np.abs(np.exp(lo - np64(lse))[fin] - np64(ss)[fin]).max() <= 2 * TOL[dtype]["ss"]
+    if block is not None:
+        assert (~fin).any(), "the case should contain rows without visible keys"
