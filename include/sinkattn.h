@@ -195,6 +195,43 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
                  void *dq, void *dk, void *dv, float *dsink,
                  void *workspace, size_t workspace_bytes, sinkattn_stream_t stream);
 
+/* ---- backward with an upstream gate gradient ---------------------------------
+ * Same as sinkattn_bwd, plus d_sink_s: float32 [T_tot, Hq] (16-byte aligned)
+ * or NULL, the upstream gradient dL/d sink_s of a loss that reads the gate
+ * sink_s = sigma(L_orig - a_h) as well as O -- page "Attention Sink and the
+ * native MoE in attention layers" (lvdousha26.github.io), section 5: the
+ * sink-aware balance loss is a function of the gate, which is differentiable
+ * through LSE and the sink.  With g = d_sink_s[t, h] and p_sink = 1 - sink_s
+ * the Delta of every row becomes Delta - g * p_sink (the key-tile kernels are
+ * otherwise unchanged) and the row's dsink term becomes
+ * -p_sink * (Delta + g * sink_s).  Without a sink (learnable_sink == NULL)
+ * sink_s is 1 on every row that sees a key and d_sink_s has no effect.
+ * sinkattn_bwd(...) == sinkattn_bwd_ex(..., d_sink_s = NULL, ...). */
+int sinkattn_bwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                    const void *q, const void *k, const void *v, const void *out,
+                    const void *dout, const float *lse_new, const float *d_sink_s,
+                    const float *learnable_sink, const sinkattn_mask *mask,
+                    const void *plan, size_t plan_bytes,
+                    void *dq, void *dk, void *dv, float *dsink,
+                    void *workspace, size_t workspace_bytes, sinkattn_stream_t stream);
+
+/* ---- head importance ---------------------------------------------------------
+ * Imp[h] = (1 / T_tot) * sum_t sink_s[t, h]: a head's mean gate over every
+ * packed token (page "Attention Sink and the native MoE in attention layers",
+ * section 4; the gate G = sigma(LSE - sink) is sink_s, section 5).  Rows that
+ * see no key count with their gate 0.
+ *   sink_s     float32 [T_tot, Hq] as written by the forward (T_tot >= 1,
+ *              1 <= Hq <= 256; SINKATTN_ERR_UNSUPPORTED above that).
+ *   imp        float32 [Hq] (written).
+ *   workspace  device scratch of at least
+ *              sinkattn_gate_importance_workspace_bytes(T_tot, Hq) bytes
+ *              (0 is returned there for invalid sizes).
+ * Partial sums are float64 in a partition fixed by (T_tot, Hq): bitwise
+ * reproducible. */
+size_t sinkattn_gate_importance_workspace_bytes(int T_tot, int Hq);
+int sinkattn_gate_importance(int T_tot, int Hq, const float *sink_s, float *imp,
+                             void *workspace, size_t workspace_bytes, sinkattn_stream_t stream);
+
 /* ---- ring-buffer decode ---------------------------------------------------
  * One query token per sequence attends over a StreamingLLM KV cache: n_sink
  * fixed slots holding the first tokens plus a circular window of `window`

@@ -224,13 +224,25 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
                  const float* lse_new, const float* learnable_sink, const sinkattn_mask* mask,
                  const void* plan, size_t plan_bytes, void* dq, void* dk, void* dv, float* dsink,
                  void* workspace, size_t workspace_bytes, sinkattn_stream_t stream) {
+  return sinkattn_bwd_ex(dt, T_tot, Hq, Hkv, D, scale, q, k, v, out, dout, lse_new, nullptr,
+                         learnable_sink, mask, plan, plan_bytes, dq, dk, dv, dsink, workspace,
+                         workspace_bytes, stream);
+}
+
+int sinkattn_bwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                    const void* q, const void* k, const void* v, const void* out,
+                    const void* dout, const float* lse_new, const float* d_sink_s,
+                    const float* learnable_sink, const sinkattn_mask* mask, const void* plan,
+                    size_t plan_bytes, void* dq, void* dk, void* dv, float* dsink,
+                    void* workspace, size_t workspace_bytes, sinkattn_stream_t stream) {
   AttnProblem p{};
   int rc = attn_common(dt, T_tot, Hq, Hkv, D, q, k, v, learnable_sink, mask, plan, plan_bytes, &p);
   if (rc != SINKATTN_OK) return rc;
   if (!out || !dout || !lse_new || !dq || !dk || !dv || !workspace) return SINKATTN_ERR_INVALID_ARG;
   if (learnable_sink && !dsink) return SINKATTN_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(dout) || !aligned16(lse_new) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (dsink && !aligned16(dsink)))
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (dsink && !aligned16(dsink)) ||
+      (d_sink_s && !aligned16(d_sink_s)))
     return SINKATTN_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(dt, T_tot, Hq, Hkv, D);
   if (workspace_bytes < L.total) return SINKATTN_ERR_WORKSPACE;
@@ -244,6 +256,7 @@ int sinkattn_bwd(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float sca
   b.dk = dk;
   b.dv = dv;
   b.dsink = learnable_sink ? dsink : nullptr;
+  b.dss = d_sink_s;  // without a sink, sink_s is 1 on every row that sees a key: no gradient
   b.delta = reinterpret_cast<float*>(ws + L.delta);
   b.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   b.dsink_part = reinterpret_cast<float*>(ws + L.part);

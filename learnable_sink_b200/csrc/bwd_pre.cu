@@ -7,6 +7,16 @@
 // backward kernels read a query tile's values with coalesced loads; a row
 // with LSE = -inf (it sees no key and has no sink) gets +inf there, which
 // makes every recomputed probability of the row exactly 0.
+// An upstream gradient g_ih = dL/d sink_s,ih (page "Attention Sink and the
+// native MoE in attention layers", lvdousha26.github.io, sections 4-5: the
+// head-importance statistic and the auxiliary balance loss are functions of
+// the gate sink_s) adds g to dL/dPhat_j of every real key, since
+// sink_s = sum_j Phat_j.  The softmax backward then needs
+//   mu_ih    = Delta_ih + g_ih * sink_s,ih
+//   dx_j     = Phat_j (<dO, V_j> + g - mu) = Phat_j (<dO, V_j> - Delta'),
+//   Delta'   = Delta - g * p_sink                   (1 - sink_s = p_sink)
+//   dsink_h  = -sum_i p_sink (Delta + g * (1 - p_sink))
+// so the key-tile kernels are unchanged: they read Delta' in place of Delta.
 // Each CTA owns a fixed range of tokens and writes one partial per head; a
 // second kernel sums the partials in a fixed order, so dsink is bitwise
 // deterministic.  HBM-bound: it streams O and dO once.
@@ -53,8 +63,8 @@ struct RowFrag {
 // its head (fixed order, so dsink is bitwise deterministic).
 template <typename T, int D>
 __global__ void __launch_bounds__(kPreThreads) preprocess_kernel(
-    const T* out, const T* dout, const float* lse, const float* sink, float* delta,
-    float* lse2, float* part, int T_tot, int Hq) {
+    const T* out, const T* dout, const float* lse, const float* sink, const float* dss,
+    float* delta, float* lse2, float* part, int T_tot, int Hq) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kPreTokens;
   for (int h = warp; h < Hq; h += kPreThreads / 32) {
@@ -89,9 +99,19 @@ __global__ void __launch_bounds__(kPreThreads) preprocess_kernel(
       float contrib = 0.f;
       if (lane < kRows && t < T_tot) {
         const float l = __ldg(lse + (long long)t * Hq + h);
-        delta[(long long)h * T_tot + t] = mine;
+        float dl = mine;
+        if (sink) {
+          const float ps = __expf(a - l);  // p_sink
+          if (dss) {
+            const float g = __ldg(dss + (long long)t * Hq + h);
+            contrib = -ps * (mine + g * (1.f - ps));
+            dl = mine - g * ps;
+          } else {
+            contrib = -mine * ps;  // -Delta * p_sink
+          }
+        }
+        delta[(long long)h * T_tot + t] = dl;
         lse2[(long long)h * T_tot + t] = (l == -INFINITY) ? INFINITY : l * kLog2e;
-        if (sink) contrib = -mine * __expf(a - l);  // -Delta * p_sink
       }
       dsum += contrib;
     }
@@ -127,16 +147,16 @@ int launch_bwd_preprocess(const AttnProblem& p, const BwdBuffers& b, cudaStream_
     const auto* o = static_cast<const __nv_bfloat16*>(b.out);
     const auto* d = static_cast<const __nv_bfloat16*>(b.dout);
     if (p.D == 64)
-      preprocess_kernel<__nv_bfloat16, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<__nv_bfloat16, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
     else
-      preprocess_kernel<__nv_bfloat16, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<__nv_bfloat16, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   } else {
     const auto* o = static_cast<const float*>(b.out);
     const auto* d = static_cast<const float*>(b.dout);
     if (p.D == 64)
-      preprocess_kernel<float, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<float, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
     else
-      preprocess_kernel<float, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
+      preprocess_kernel<float, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   }
   if (p.sink && b.dsink)
     dsink_reduce_kernel<<<(p.Hq + 3) / 4, 128, 0, stream>>>(b.dsink_part, nb, p.Hq, b.dsink);

@@ -73,6 +73,7 @@ struct BwdBuffers {
   void* dk;
   void* dv;
   float* dsink;
+  const float* dss;     // [T_tot, Hq] upstream dL/d sink_s, or nullptr
   float* delta;         // [Hq, T_tot] workspace (head-major)
   float* lse2;          // [Hq, T_tot] workspace: LSE_new * log2(e), -inf -> +inf
   float* dsink_part;    // [n_part_blocks, Hq] workspace

@@ -67,6 +67,12 @@ def lib():
         L.sinkattn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, M]
         L.sinkattn_bwd.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp, _vp,
                                    _vp, M, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+        L.sinkattn_bwd_ex.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp,
+                                      _vp, _vp, _vp, M, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _sz,
+                                      _vp]
+        L.sinkattn_gate_importance_workspace_bytes.restype = _sz
+        L.sinkattn_gate_importance_workspace_bytes.argtypes = [_i, _i]
+        L.sinkattn_gate_importance.argtypes = [_i, _i, _vp, _vp, _vp, _sz, _vp]
         L.sinkattn_decode_workspace_bytes.restype = _sz
         L.sinkattn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
         L.sinkattn_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
@@ -206,9 +212,10 @@ def bwd_workspace_bytes(q, k, mask: Mask) -> int:
 
 
 def bwd(q, k, v, out, dout, lse, sink, mask: Mask, plan: Plan, scale: Optional[float] = None,
-        stream=None, workspace=None, dq=None, dk=None, dv=None, dsink=None):
-    """Backward.  Returns (dq, dk, dv, dsink or None)."""
-    _contig(q, k, v, out, dout, lse, sink)
+        stream=None, workspace=None, dq=None, dk=None, dv=None, dsink=None, d_sink_s=None):
+    """Backward.  Returns (dq, dk, dv, dsink or None).  ``d_sink_s`` [T, Hq]
+    float32 is an optional upstream gradient of the gate sink_s."""
+    _contig(q, k, v, out, dout, lse, sink, d_sink_s)
     T, Hq, D = q.shape
     Hkv = k.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
@@ -221,11 +228,24 @@ def bwd(q, k, v, out, dout, lse, sink, mask: Mask, plan: Plan, scale: Optional[f
     dv = torch.empty_like(v) if dv is None else dv
     if dsink is None and sink is not None:
         dsink = torch.empty(Hq, dtype=torch.float32, device=q.device)
-    _check("sinkattn_bwd", lib().sinkattn_bwd(
+    _check("sinkattn_bwd_ex", lib().sinkattn_bwd_ex(
         _dt(q), T, Hq, Hkv, D, scale, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
-        _ptr(sink), _c.byref(cm), _ptr(plan.buf), plan.nbytes, _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(d_sink_s), _ptr(sink), _c.byref(cm), _ptr(plan.buf), plan.nbytes, _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(dsink), _ptr(workspace), workspace.numel(), _stream(stream)))
     return dq, dk, dv, dsink
+
+
+def gate_importance(sink_s, stream=None, workspace=None, imp=None):
+    """Per-head mean gate Imp [Hq] of sink_s [T, Hq] float32."""
+    _contig(sink_s)
+    T, Hq = sink_s.shape
+    nws = int(lib().sinkattn_gate_importance_workspace_bytes(T, Hq))
+    if workspace is None:
+        workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=sink_s.device)
+    imp = torch.empty(Hq, dtype=torch.float32, device=sink_s.device) if imp is None else imp
+    _check("sinkattn_gate_importance", lib().sinkattn_gate_importance(
+        T, Hq, _ptr(sink_s), _ptr(imp), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return imp
 
 
 def decode_num_splits(B, Hq, Hkv, D, n_sink, window) -> int:

@@ -266,3 +266,13 @@ def visible_pairs(spec: MaskSpec, Hq: int, Hkv: int) -> int:
                         total += int(vis.sum())
                 r += 1
     return int(total) * G
+
+
+def gate_inputs(T_tot: int, Hq: int, seed: int):
+    """Seeded per-(token, head) float32 arrays for the gate statistics and the
+    gate-gradient backward: (values uniform in [0, 1) shaped like sink_s,
+    standard-normal upstream gradients of sink_s)."""
+    gen = _gen(seed)
+    vals = torch.rand(T_tot, Hq, generator=gen, dtype=torch.float32)
+    grads = torch.randn(T_tot, Hq, generator=gen, dtype=torch.float32)
+    return vals, grads

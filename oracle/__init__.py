@@ -9,7 +9,10 @@ rows), which follows the page "Attention Sink, Learnable Sink and dsink"
 (notes.kuangjux.top): the forward of section 4 with the sink as an explicit
 extra softmax column, the backward as the explicit Jacobian of that augmented
 softmax (sections 7-8), the visible set of section 2, and the StreamingLLM
-ring-buffer KV set (sink segment + sliding window).
+ring-buffer KV set (sink segment + sliding window).  The gate statistics of
+the page "Attention Sink and the native MoE in attention layers"
+(lvdousha26.github.io, sections 4-5: head importance and the sink-aware
+balance loss) are plain numpy on top of the forward's sink_s.
 
 Every function takes and returns numpy arrays; floating-point inputs are
 converted to float64 here (the caller passes the same rounded values the GPU
@@ -58,7 +61,7 @@ def _load():
             lib.oracle_fwd.argtypes = _PROBLEM + [_d, _d, _d, _d, _d, _d, _d]
             lib.oracle_fwd_rows.argtypes = _PROBLEM + [
                 _d, _d, _d, _d, ctypes.c_int, _i32, _d, _d, _d]
-            lib.oracle_bwd.argtypes = _PROBLEM + [_d, _d, _d, _d, _d, _d, _d, _d, _d]
+            lib.oracle_bwd.argtypes = _PROBLEM + [_d, _d, _d, _d, _d, _d, _d, _d, _d, _d]
             lib.oracle_bwd_sampled.argtypes = _PROBLEM + [
                 _d, _d, _d, _d, _d, ctypes.c_int, _i32, _d, ctypes.c_int, _i32, _d, _d]
             lib.oracle_decode.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [
@@ -143,15 +146,17 @@ def fwd_rows(q, k, v, sink, scale, rows, **mask):
     return out, lse, ss
 
 
-def bwd(q, k, v, sink, dout, scale, **mask):
-    """Returns (dq, dk, dv, dsink) in float64; dsink is None without a sink."""
-    q, k, v, sink, dout = _f64(q), _f64(k), _f64(v), _f64(sink), _f64(dout)
+def bwd(q, k, v, sink, dout, scale, dss=None, **mask):
+    """Returns (dq, dk, dv, dsink) in float64; dsink is None without a sink.
+    ``dss`` [T, Hq] is an optional upstream gradient of sink_s (the loss is
+    sum dout*O + sum dss*sink_s)."""
+    q, k, v, sink, dout, dss = _f64(q), _f64(k), _f64(v), _f64(sink), _f64(dout), _f64(dss)
     T, Hq, Hkv, D = _shapes(q, k)
     pr = _Problem(T, Hq, Hkv, D, scale, **mask)
     dq = np.zeros((T, Hq, D)); dk = np.zeros((T, Hkv, D)); dv = np.zeros((T, Hkv, D))
     dsink = np.zeros(Hq) if sink is not None else None
     rc = _load().oracle_bwd(*pr.args, _p(q, _d), _p(k, _d), _p(v, _d), _p(sink, _d),
-                            _p(dout, _d), _p(dq, _d), _p(dk, _d), _p(dv, _d),
+                            _p(dout, _d), _p(dss, _d), _p(dq, _d), _p(dk, _d), _p(dv, _d),
                             _p(dsink, _d))
     if rc != 0:
         raise MemoryError("oracle_bwd: allocation failed")
@@ -174,6 +179,38 @@ def bwd_sampled(q, k, v, sink, dout, scale, rows, keys, **mask):
     if rc != 0:
         raise MemoryError("oracle_bwd_sampled: allocation failed")
     return dq, dk, dv
+
+
+def gate_importance(sink_s):
+    """Imp_h: the mean gate of head h over every token (page "Attention Sink
+    and the native MoE in attention layers", section 4; the gate
+    sigma(LSE - sink) of its section 5 is sink_s).  sink_s [T, Hq] -> [Hq]."""
+    ss = _f64(sink_s)
+    return ss.sum(axis=0) / ss.shape[0]
+
+
+def gate_aux_loss(imp, lam=1.0, n_shared=0):
+    """Sink-aware balance loss of one layer and its gradient d loss / d Imp
+    (same page, section 5): lam * (N_h - m) * CV(Imp over routed heads)^2,
+    where the m = n_shared heads of largest Imp are shared heads and left out
+    (m = 0 is the from-scratch form lam * N_h * CV^2).  CV = std / mean with
+    the population standard deviation.  Shared heads get gradient 0 (their
+    selection is piecewise constant).  Returns (loss, d_imp [Hq])."""
+    imp = _f64(imp)
+    n = imp.shape[0]
+    order = np.argsort(-imp, kind="stable")
+    routed = np.ones(n, dtype=bool)
+    routed[order[:n_shared]] = False
+    x = imp[routed]
+    nr = x.shape[0]
+    mu = x.mean()
+    var = ((x - mu) ** 2).mean()
+    loss = lam * nr * var / mu ** 2
+    # d var / d x_i = 2 (x_i - mu) / nr ; d mu / d x_i = 1 / nr
+    dx = lam * nr * (2.0 * (x - mu) / nr / mu ** 2 - 2.0 * var / mu ** 3 / nr)
+    d_imp = np.zeros(n)
+    d_imp[routed] = dx
+    return float(loss), d_imp
 
 
 def decode(q, k_cache, v_cache, cache_seqlens, n_sink, window, sink, scale):

@@ -22,7 +22,10 @@
  *
  * Backward is the explicit Jacobian of the augmented softmax (independent of
  * the dsink closed form of section 7):
- *   dPhat_j = <dO_ih, V_j> ; dPhat_sink = 0 (zero value row)
+ *   dPhat_j = <dO_ih, V_j> (+ dss_ih, an optional upstream gradient of
+ *             sink_s = sum_j Phat_j; page "Attention Sink and the native MoE
+ *             in attention layers", section 5, trains through the gate)
+ *   dPhat_sink = 0 (zero value row)
  *   mu      = sum_{j and sink} Phat dPhat          (equals Delta of section 7)
  *   dx_j    = Phat_j (dPhat_j - mu)
  *   da_h   += p_sink (0 - mu)
@@ -259,13 +262,14 @@ int oracle_fwd_rows(OM_PROBLEM_ARGS, const double *q, const double *k,
 }
 
 /* Full backward: dq [T,Hq,D], dk/dv [T,Hkv,D], dsink [Hq] (if sink != NULL).
- * dout is the upstream gradient dL/dO.  Two plain phases:
+ * dout is the upstream gradient dL/dO; dss [T,Hq] (or NULL) that of sink_s.
+ * Two plain phases:
  *   1. per row (i, h): forward statistics, mu = sum Phat dPhat, and dQ;
  *   2. per key (j, g): dK, dV summed over every (row, head of group g) that
  *      sees the key, with the row's Phat recomputed from its statistics. */
 int oracle_bwd(OM_PROBLEM_ARGS, const double *q, const double *k,
                const double *v, const double *sink, const double *dout,
-               double *dq, double *dk, double *dv, double *dsink) {
+               const double *dss, double *dq, double *dk, double *dv, double *dsink) {
     om_problem p = make_problem(OM_PROBLEM_PASS);
     const int G = Hq / Hkv;
     const long R = (long)T_tot * Hq;
@@ -288,17 +292,20 @@ int oracle_bwd(OM_PROBLEM_ARGS, const double *q, const double *k,
             for (int d = 0; d < D; ++d) dqrow[d] = 0.0;
             mu[r] = 0.0;
             if (st[r].M == -INFINITY) continue;
-            /* mu = sum_j Phat_j <dO, V_j> + p_sink * 0 */
+            /* an upstream gradient of sink_s = sum_j Phat_j (the real-token
+             * mass) adds dss to every real key's dPhat */
+            const double gs = dss ? dss[r] : 0.0;
+            /* mu = sum_j Phat_j dPhat_j + p_sink * 0 */
             double m = 0.0;
             for (int t = 0; t < st[r].n_vis; ++t) {
                 double P = exp(xs[t] - st[r].M) / st[r].den;
-                m += P * dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D);
+                m += P * (dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D) + gs);
             }
             mu[r] = m;
             for (int t = 0; t < st[r].n_vis; ++t) {
                 const double *krow = k + ((size_t)js[t] * Hkv + g) * D;
                 double P = exp(xs[t] - st[r].M) / st[r].den;
-                double dx = P * (dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D) - m);
+                double dx = P * (dot(dorow, v + ((size_t)js[t] * Hkv + g) * D, D) + gs - m);
                 for (int d = 0; d < D; ++d) dqrow[d] += scale * dx * krow[d];
             }
         }
@@ -320,7 +327,7 @@ int oracle_bwd(OM_PROBLEM_ARGS, const double *q, const double *k,
                 const double *qrow = q + (size_t)r * D, *dorow = dout + (size_t)r * D;
                 double x = scale * dot(qrow, krow, D);
                 double P = exp(x - st[r].M) / st[r].den;
-                double dx = P * (dot(dorow, vrow, D) - mu[r]);
+                double dx = P * (dot(dorow, vrow, D) + (dss ? dss[r] : 0.0) - mu[r]);
                 for (int d = 0; d < D; ++d) {
                     dkrow[d] += scale * dx * qrow[d];
                     dvrow[d] += P * dorow[d];

@@ -70,3 +70,20 @@ def test_workspace_queries(lib):
     assert lib.sinkattn_bwd_workspace_bytes(0, 128, 4, 2, 96, ctypes.byref(m)) == 0
     assert lib.sinkattn_decode_workspace_bytes(32, 32, 128, 4) >= 32 * 32 * 4 * 130 * 4
     assert lib.sinkattn_decode_workspace_bytes(32, 32, 80, 4) == 0
+    lib.sinkattn_gate_importance_workspace_bytes.restype = ctypes.c_size_t
+    # one float64 partial per head per CTA of at least 32 tokens, at most 1024 CTAs
+    assert lib.sinkattn_gate_importance_workspace_bytes(100, 32) == 4 * 32 * 8
+    assert lib.sinkattn_gate_importance_workspace_bytes(10 ** 6, 8) == 1024 * 8 * 8
+    assert lib.sinkattn_gate_importance_workspace_bytes(0, 8) == 0
+    assert lib.sinkattn_gate_importance_workspace_bytes(64, 257) == 0
+
+
+def test_gate_importance_host_validation(lib):
+    """Argument checks that return before anything reaches a device."""
+    f = lib.sinkattn_gate_importance
+    f.argtypes = [ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 3 + [ctypes.c_size_t,
+                                                                        ctypes.c_void_p]
+    assert f(0, 8, None, None, None, 0, None) == 1      # T_tot < 1
+    assert f(16, 0, None, None, None, 0, None) == 1     # Hq < 1
+    assert f(16, 257, None, None, None, 0, None) == 2   # more heads than supported
+    assert f(16, 8, None, None, None, 0, None) == 1     # null pointers

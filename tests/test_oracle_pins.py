@@ -259,6 +259,118 @@ def test_gate_identities_and_dsink_closed_form():
     np.testing.assert_allclose(dsink, -(delta * np.exp(a[None, :] - l_new)).sum(0), atol=1e-12)
 
 
+# ------------------------------------------- gate gradient and gate statistics
+# Page "Attention Sink and the native MoE in attention layers"
+# (lvdousha26.github.io), sections 4-5: head importance is the mean gate, the
+# balance loss is lam * N_h * CV(Imp)^2, and training through it needs the
+# backward to accept an upstream gradient of the gate sink_s.
+
+@pytest.mark.parametrize("mname", ["causal", "varlen_band", "block_sparse"])
+def test_gate_gradient_matches_library_autograd(mname):
+    """oracle.bwd with dss equals float64 autograd of
+    sum(dout * O) + sum(dss * sink_s) through torch's softmax."""
+    T, Hq, Hkv, D = 37, 4, 2, 16
+    mask = MASKS[mname] if mname != "block_sparse" else _block_sparse_mask()
+    q, k, v, a, dout = _random_problem(T, Hq, Hkv, D, seed=21)
+    dss = np.random.default_rng(22).standard_normal((T, Hq))
+    scale = 1 / math.sqrt(D)
+    dq, dk, dv, dsink = oracle.bwd(q, k, v, a, dout, scale, dss=dss, **mask)
+    tq, tk, tv, ta = (torch.from_numpy(x).requires_grad_() for x in (q, k, v, a))
+    vis = _vis_all(T, Hq, Hkv, mask)
+    out, _, ss = _sdpa_forward(tq, tk, tv, ta, scale, vis)
+    ((out * torch.from_numpy(dout)).sum() + (ss * torch.from_numpy(dss)).sum()).backward()
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dsink, ta.grad.numpy(), atol=1e-11)
+
+
+def test_gate_gradient_central_differences():
+    T, Hq, Hkv, D = 12, 4, 2, 4
+    mask = dict(causal=True, n_sink=1, window=4, cu_seqlens=np.array([0, 5, 12], dtype=np.int32))
+    q, k, v, a, dout = _random_problem(T, Hq, Hkv, D, seed=23)
+    dss = np.random.default_rng(24).standard_normal((T, Hq)) * 3.0
+    scale = 1 / math.sqrt(D)
+    grads = oracle.bwd(q, k, v, a, dout, scale, dss=dss, **mask)
+
+    def loss(args):
+        o, _, s_ = oracle.fwd(args[0], args[1], args[2], args[3], scale, **mask)
+        return float((o * dout).sum() + (s_ * dss).sum())
+
+    eps = 1e-6
+    rng = np.random.default_rng(1)
+    base = [q, k, v, a]
+    for which, grad in enumerate(grads):
+        arr = base[which]
+        for f in rng.choice(arr.size, size=min(arr.size, 10), replace=False):
+            idx = np.unravel_index(int(f), arr.shape)
+            pl = [x.copy() for x in base]; mi = [x.copy() for x in base]
+            pl[which][idx] += eps
+            mi[which][idx] -= eps
+            fd = (loss(pl) - loss(mi)) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, np.abs(grad).max()), (which, idx, fd)
+
+
+def test_gate_gradient_sigmoid_closed_form():
+    """With dout = 0 and dss = 1 the loss is sum sink_s = sum sigma(L_orig - a),
+    so dsink_h = -sum_i s (1 - s) (the logistic derivative) and dV = 0."""
+    T, Hq, Hkv, D = 30, 4, 2, 8
+    mask = MASKS["varlen_band"] | dict(cu_seqlens=np.array([0, 13, 30], dtype=np.int32))
+    q, k, v, a, _ = _random_problem(T, Hq, Hkv, D, seed=25)
+    scale = 0.4
+    _, _, s = oracle.fwd(q, k, v, a, scale, **mask)
+    _, _, dv, dsink = oracle.bwd(q, k, v, a, np.zeros((T, Hq, D)), scale,
+                                 dss=np.ones((T, Hq)), **mask)
+    np.testing.assert_allclose(dsink, -(s * (1 - s)).sum(0), atol=1e-12)
+    assert np.all(dv == 0)
+
+
+def test_gate_gradient_zero_dss_is_plain_backward():
+    T, Hq, Hkv, D = 37, 4, 2, 16
+    q, k, v, a, dout = _random_problem(T, Hq, Hkv, D, seed=26)
+    ref = oracle.bwd(q, k, v, a, dout, 0.25, **MASKS["band"])
+    got = oracle.bwd(q, k, v, a, dout, 0.25, dss=np.zeros((T, Hq)), **MASKS["band"])
+    for x, y in zip(ref, got):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_gate_importance_closed_forms():
+    """Imp is the per-head mean gate: rows of a constant gate give that
+    constant; for keys that all score 0 (q = 0) the gate of a row that sees n
+    keys is n / (n + e^a)."""
+    ss = np.tile(np.array([0.25, 0.5, 1.0]), (7, 1))
+    np.testing.assert_allclose(oracle.gate_importance(ss), [0.25, 0.5, 1.0], rtol=0, atol=0)
+    T, Hq, Hkv, D = 9, 2, 1, 4
+    q = np.zeros((T, Hq, D)); k = np.ones((T, Hkv, D)); v = np.ones((T, Hkv, D))
+    a = np.array([0.0, math.log(2.0)])
+    _, _, s = oracle.fwd(q, k, v, a, 1.0, **causal_mask(T))
+    n = np.arange(1, T + 1)
+    expect = [np.mean(n / (n + math.exp(ah))) for ah in a]
+    np.testing.assert_allclose(oracle.gate_importance(s), expect, atol=1e-15)
+
+
+def test_gate_aux_loss_closed_forms_and_gradient():
+    # Imp = (1, 3): mean 2, population std 1, CV = 1/2 -> lam * 2 * 1/4
+    loss, d = oracle.gate_aux_loss(np.array([1.0, 3.0]), lam=0.1)
+    assert abs(loss - 0.05) < 1e-15
+    # balanced heads: zero loss, zero gradient
+    loss, d = oracle.gate_aux_loss(np.full(8, 0.3), lam=1.0)
+    assert loss == 0.0 and np.all(np.abs(d) < 1e-15)
+    # shared/routed form: the top-1 head (5.0) is shared -> routed (1, 3)
+    loss, d = oracle.gate_aux_loss(np.array([1.0, 5.0, 3.0]), lam=0.1, n_shared=1)
+    assert abs(loss - 0.05) < 1e-15 and d[1] == 0.0
+    # gradient against central differences
+    rng = np.random.default_rng(27)
+    imp = rng.uniform(0.1, 1.0, 12)
+    for m in (0, 3):
+        _, d = oracle.gate_aux_loss(imp, lam=0.7, n_shared=m)
+        for h in range(12):
+            e = np.zeros(12); e[h] = 1e-7
+            fd = (oracle.gate_aux_loss(imp + e, 0.7, m)[0] -
+                  oracle.gate_aux_loss(imp - e, 0.7, m)[0]) / 2e-7
+            assert abs(fd - d[h]) < 1e-6, (m, h, fd, d[h])
+
+
 def test_relative_probabilities_unchanged_by_sink():
     T, Hq, Hkv = 9, 2, 1
     rng = np.random.default_rng(7)
