@@ -195,77 +195,77 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(DecodeProblem
 // next pieces, and for the first pieces of its next item, are in flight while
 // it computes), and writes one partial (m, l, acc) per query head and item.
 // No warp ever waits for another, so nothing couples the warps of an SM
-// beyond sharing its load bandwidth.  A group of D/8 lanes holds one row's
-// 8-element slices; the warp's groups split each piece's rows (PR each) and
-// merge their online-softmax states, max-rescaled, once per item.  Dot
-// products of a group's PR x G (row, head) pairs are reduced by a butterfly
-// that splits the values across the group's lanes.  bf16 is widened with
-// integer ops, products use the packed fp32x2 FMA, and the running maximum
-// moves only when a score exceeds it by more than 2^8 (so the output rescale
-// is rare; O = acc / l does not depend on which reference maximum was used).
+// beyond sharing its load bandwidth.
+//
+// The kernel is bound by HBM, so its arithmetic only has to stay off the
+// critical path; it runs on the warp-level tensor-core MMA (m16n8k16, bf16
+// in, fp32 accumulate), which spends a few instructions where CUDA-core
+// dot products spend hundreds.  The G query heads of the KV head are the 16
+// M rows (zero-padded; G <= 8, so rows 8-15 are always padding):
+//   S^T-free form   S[h][r] = Q[h] . K[r]  : A = Q (registers, once per item),
+//                                            B = K rows via ldmatrix
+//                   O[h][:] += P[h][r] V[r] : A = P (the S accumulators,
+//                                            rounded to bf16), B = V via
+//                                            ldmatrix.trans
+// A lane quad (lane / 4 = head) holds four scores of a 16-row piece, so the
+// online softmax needs two shuffles per piece.  K and V land in 64-column
+// (128-byte) TMA boxes with the 128-byte swizzle, which keeps the ldmatrix
+// row reads free of bank conflicts.  The running maximum moves only when a
+// score exceeds it by more than 2^8 (the output rescale is rare; O = acc / l
+// does not depend on which reference maximum was used); l is summed from the
+// fp32 probabilities.
 constexpr int kDecWarps = 8;      // warps per CTA (one CTA per SM)
 constexpr int kDecStages = 3;     // ring stages per warp
-constexpr int kLenSlots = 1024;   // sequences whose cache lengths are staged in shared memory
+// per-block shared-memory limit, less room for the kernel's static shared memory
+constexpr int kDecSmemMax = 232448 - 256;
 
 template <int D, int G>
 struct WarpGeom {
-  static constexpr int LPR = D / 8;                          // lanes per row
-  static constexpr int NGW = 32 / LPR;                       // row groups per warp
-  static constexpr int PR0 = 16 / NGW;
-  static constexpr int PR = PR0 * G <= 32 ? PR0 : 32 / G;    // rows per group per piece
-  static constexpr int R = NGW * PR;                         // rows per piece
-  static constexpr int V = PR * G;                           // values per lane before reduce
-  static constexpr int ROW_BYTES = D * 2;                    // one row of one head
-  static constexpr int PIECE_BYTES = R * ROW_BYTES;          // K or V piece [R][D]
+  static constexpr int R = 16;                               // rows per piece
+  static constexpr int HALVES = D / 64;                      // 64-column TMA boxes per row
+  static constexpr int HALF_BYTES = R * 128;                 // one box: R rows x 128 bytes
+  static constexpr int PIECE_BYTES = HALVES * HALF_BYTES;    // K or V piece [R][D]
   static constexpr int STAGE_BYTES = 2 * PIECE_BYTES;
+  static constexpr int KSTEPS = D / 16;                      // MMA k-steps of Q K^T
+  static constexpr int NT = D / 8;                           // MMA n-tiles of P V
   static constexpr int Q_BYTES = G * D * 2;                  // an item's query heads (bf16)
   static constexpr int OFF_Q = kDecStages * STAGE_BYTES;     // 2 q slots (this item, next)
-  static constexpr int OFF_SC = OFF_Q + 2 * Q_BYTES;         // float [2][NGW][V] scores, probabilities
-  static constexpr int WARP_BYTES = (OFF_SC + 2 * NGW * V * 4 + 127) / 128 * 128;
+  // stages start on 1024-byte boundaries (the swizzle pattern's period)
+  static constexpr int WARP_BYTES = (OFF_Q + 2 * Q_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = kDecWarps * WARP_BYTES;
-  static constexpr int OFF_LEN = OFF_BAR + kDecWarps * kDecStages * 8;  // int [kLenSlots]
-  // + 128: the kernel rounds the dynamic shared-memory base up to 128 bytes
-  static constexpr int SMEM = OFF_LEN + kLenSlots * 4 + 128;
-  static constexpr int LOG_LPR = LPR == 16 ? 4 : 3;
-  static constexpr int LOG_V = V >= 32 ? 5 : V >= 16 ? 4 : V >= 8 ? 3 : V >= 4 ? 2 : V >= 2 ? 1 : 0;
-  static constexpr int KS = LOG_V < LOG_LPR ? LOG_V : LOG_LPR;  // splitting steps
-  static constexpr int KEEP = V >> KS;                        // values a lane ends with
-  static_assert(PR >= 1 && (1 << LOG_V) == V, "power-of-two rows x heads");
-  static_assert(SMEM <= 232448, "shared memory");
+  static constexpr int OFF_LEN = OFF_BAR + kDecWarps * kDecStages * 8;
+  // cache lengths staged in shared memory (sequences past this read global)
+  static constexpr int LEN_FIT = (kDecSmemMax - 1024 - OFF_LEN) / 4;
+  static constexpr int LEN_SLOTS = LEN_FIT < 1024 ? LEN_FIT : 1024;
+  // + 1024: the kernel rounds the dynamic shared-memory base up to 1024 bytes
+  static constexpr int SMEM = OFF_LEN + LEN_SLOTS * 4 + 1024;
+  static_assert(G >= 1 && G <= 8, "query heads per KV head");
+  static_assert(D % 64 == 0 && HALF_BYTES % 1024 == 0, "swizzled boxes");
+  static_assert(LEN_SLOTS >= 64 && SMEM <= kDecSmemMax, "shared memory");
 };
 
-// Sum each of the V values over the LPR lanes of a group; afterwards lane gl
-// holds KEEP totals, value index decode_value_index(gl, j).
-template <int V, int LPR>
-__device__ __forceinline__ void butterfly_reduce(float (&v)[V], int gl) {
-  int c = V;
-#pragma unroll
-  for (int o = LPR / 2; o >= 1; o >>= 1) {
-    if (c > 1) {
-      const int half = c / 2;
-      const bool upper = (gl & o) != 0;
-#pragma unroll
-      for (int i = 0; i < V / 2; ++i) {
-        if (i < half) {
-          const float send = upper ? v[i] : v[i + half];
-          const float keep = upper ? v[i + half] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      c = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    }
-  }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
-
-template <int LOG_V, int LOG_LPR, int KS>
-__device__ __forceinline__ int decode_value_index(int gl, int j) {
-  int idx = 0;
-#pragma unroll
-  for (int k = 0; k < KS; ++k)
-    idx |= ((gl >> (LOG_LPR - 1 - k)) & 1) << (LOG_V - 1 - k);
-  return idx | j;
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// (c0, c1) += A B for one m16n8k16 tile whose A rows 8-15 are zero: a_lo / a_hi
+// hold row lane/4 at k = 2(lane%4) + {0, 1} and + 8; c0, c1 are that row's
+// outputs at n = 2(lane%4) + {0, 1}.  The accumulators of rows 8-15 are dropped.
+__device__ __forceinline__ void mma_top_rows(float& c0, float& c1, uint32_t a_lo, uint32_t a_hi,
+                                             uint32_t b0, uint32_t b1) {
+  float x2, x3;
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %10, %10};"
+      : "+f"(c0), "+f"(c1), "=f"(x2), "=f"(x3)
+      : "r"(a_lo), "r"(0u), "r"(a_hi), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
 }
 
 // Merge the splits of query head h of sequence b with the sink column (page
@@ -355,10 +355,9 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     DecodeProblem p, int chunk, int n_items) {
   using Geo = WarpGeom<D, G>;
-  constexpr int LPR = Geo::LPR, PR = Geo::PR, V = Geo::V, R = Geo::R;
-  constexpr int RS = kDecStages;
+  constexpr int R = Geo::R, RS = kDecStages;
   extern __shared__ uint8_t dsm_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) & ~uintptr_t(127));
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   __shared__ int abort_s;
   const int S = p.n_sink + p.window;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -366,7 +365,7 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Geo::OFF_BAR) + warp * RS;
   // cache_seqlens of every sequence, staged once per CTA when they fit
   int* s_len = reinterpret_cast<int*>(sm + Geo::OFF_LEN);
-  const bool len_in_smem = p.B <= kLenSlots;
+  const bool len_in_smem = p.B <= Geo::LEN_SLOTS;
   if (len_in_smem)
     for (int i = threadIdx.x; i < p.B; i += blockDim.x) s_len[i] = __ldg(p.cache_seqlens + i);
   if (threadIdx.x == 0) abort_s = 0;
@@ -434,32 +433,29 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
                     static_cast<const __nv_bfloat16*>(p.q) + ((long long)I.b * p.Hq + I.kvh * G) * D,
                     Geo::Q_BYTES, full + st);
         const int row0 = I.row0 + p_r0;  // rows past the split are unused
-        tma_load_3d(base, &tmap_k, full + st, 0, I.kvh, row0);
-        tma_load_3d(base + Geo::PIECE_BYTES, &tmap_v, full + st, 0, I.kvh, row0);
+#pragma unroll
+        for (int hf = 0; hf < Geo::HALVES; ++hf) {
+          tma_load_3d(base + hf * Geo::HALF_BYTES, &tmap_k, full + st, hf * 64, I.kvh, row0);
+          tma_load_3d(base + Geo::PIECE_BYTES + hf * Geo::HALF_BYTES, &tmap_v, full + st, hf * 64,
+                      I.kvh, row0);
+        }
       }
       p_r0 += R;
       ++pc_issue;
     }
   };
 
-  const int grp = lane / LPR, gl = lane % LPR;
-  const int c0 = gl * 8;
-  float* sc_s = reinterpret_cast<float*>(wsm + Geo::OFF_SC) + grp * V;                // scores
-  float* sc_p = reinterpret_cast<float*>(wsm + Geo::OFF_SC) + (Geo::NGW + grp) * V;   // probabilities
+  const int g = lane >> 2, t = lane & 3;  // fragment row (query head) and column pair
+  const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix and row this lane addresses
   const float scale_log2 = p.scale * kLog2e;
   bool ok = true;
   while (cur.it < n_items && ok) {
     const int split = cur.split, kvh = cur.kvh, b = cur.b, n_cur = cur.n;
-    float2 qv[G][4];
-    float2 acc[G][4];
-    float m_run[G], l_run[G];
+    uint32_t qa[Geo::KSTEPS][2];  // A fragments of Q (row g; zero for padding heads)
+    float oc[Geo::NT][2];         // O[g][8 j + 2 t + {0, 1}]
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_run[h] = -INFINITY;
-      l_run[h] = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[h][i] = make_float2(0.f, 0.f);
-    }
+    for (int j = 0; j < Geo::NT; ++j) oc[j][0] = oc[j][1] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // head g; l_run sums this lane's probabilities
     issue();
     for (int r0 = 0; r0 < n_cur; r0 += R) {
       const int st = pc_cons % RS;
@@ -467,123 +463,100 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
       if (!ok) break;
       const int rows = min(R, n_cur - r0);
       if (r0 == 0) {
-        const __nv_bfloat16* qs =
-            reinterpret_cast<const __nv_bfloat16*>(wsm + Geo::OFF_Q + (kc & 1) * Geo::Q_BYTES);
+        // padding heads read head 0's row (inside the slot) and drop it
+        const uint8_t* qs =
+            wsm + Geo::OFF_Q + (kc & 1) * Geo::Q_BYTES + (g < G ? g : 0) * D * 2 + t * 4;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float2 t[4];
-          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(qs + h * D + c0), t);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) qv[h][i] = make_float2(t[i].x * scale_log2, t[i].y * scale_log2);
+        for (int kk = 0; kk < Geo::KSTEPS; ++kk) {
+          const uint32_t lo = *reinterpret_cast<const uint32_t*>(qs + kk * 32);
+          const uint32_t hi = *reinterpret_cast<const uint32_t*>(qs + kk * 32 + 16);
+          qa[kk][0] = g < G ? lo : 0u;
+          qa[kk][1] = g < G ? hi : 0u;
         }
       }
-      const uint8_t* kbuf = wsm + st * Geo::STAGE_BYTES;
-      const uint8_t* vbuf = kbuf + Geo::PIECE_BYTES;
-      // scores of this group's PR rows for all G heads
-      float v[V];
-#pragma unroll
-      for (int rr = 0; rr < PR; ++rr) {
-        const int r = grp * PR + rr;
-        float2 kf[4];
-        bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(kbuf + r * Geo::ROW_BYTES + c0 * 2), kf);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float2 a = __fmul2_rn(qv[h][0], kf[0]);
-#pragma unroll
-          for (int i = 1; i < 4; ++i) a = __ffma2_rn(qv[h][i], kf[i], a);
-          v[rr * G + h] = a.x + a.y;
+      uint8_t* kbuf = wsm + st * Geo::STAGE_BYTES;
+      uint8_t* vbuf = kbuf + Geo::PIECE_BYTES;
+      // Rows past the valid range hold whatever the cache holds there; their
+      // scores are masked below, and their V rows are zeroed so that a stale
+      // NaN cannot reach the P V products (only an item's last piece).
+      if (rows < R) {
+        const int nz = Geo::HALVES * (R - rows) * 8;  // 16-byte chunks
+        for (int i = lane; i < nz; i += 32) {
+          const int hf = i / ((R - rows) * 8), rem = i % ((R - rows) * 8);
+          *reinterpret_cast<uint4*>(vbuf + hf * Geo::HALF_BYTES + (rows + rem / 8) * 128 +
+                                    (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
+        // order these generic writes before the stage's next asynchronous refill
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
       }
-      butterfly_reduce<V, LPR>(v, gl);
+      // S = Q K^T for rows 0-7 (sa) and 8-15 (sb) of the piece
+      const uint32_t kb = smem_u32(kbuf), vb = smem_u32(vbuf);
+      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < Geo::KEEP; ++j) {
-        const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
-        sc_s[idx] = (grp * PR + idx / G < rows) ? v[j] : -INFINITY;
+      for (int kk = 0; kk < Geo::KSTEPS; ++kk) {
+        // matrices: rows (mi >> 1) * 8 + mr, columns 16 kk + (mi & 1) * 8
+        const int row = (mi >> 1) * 8 + mr, chunk = ((2 * kk) & 7) + (mi & 1);
+        uint32_t r[4];
+        ldsm_x4(kb + (kk >> 2) * Geo::HALF_BYTES + row * 128 + ((chunk ^ mr) << 4), r);
+        mma_top_rows(sa0, sa1, qa[kk][0], qa[kk][1], r[0], r[1]);
+        mma_top_rows(sb0, sb1, qa[kk][0], qa[kk][1], r[2], r[3]);
       }
-      __syncwarp();
-      // Running maximum per head over the group's rows; it moves (and the
-      // group's sum and output are rescaled) only when a score exceeds it by
-      // more than 2^kLazyLog2.  From -inf any finite score moves it; an
-      // all-masked piece leaves it alone.
+      // scores of head g at rows 2t, 2t + 1, 8 + 2t, 9 + 2t (log2 units)
+      const int ra = 2 * t;
+      const float x0 = ra < rows ? sa0 * scale_log2 : -INFINITY;
+      const float x1 = ra + 1 < rows ? sa1 * scale_log2 : -INFINITY;
+      const float x2 = ra + 8 < rows ? sb0 * scale_log2 : -INFINITY;
+      const float x3 = ra + 9 < rows ? sb1 * scale_log2 : -INFINITY;
+      float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      // From -inf any finite score moves the maximum; an all-masked piece
+      // leaves it alone.
+      if (mx > m_run + kLazyLog2) {
+        const float corr = fast_exp2(m_run - mx);  // 0 when m_run was -inf
+        l_run *= corr;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int rr = 0; rr < PR; ++rr) mx = fmaxf(mx, sc_s[rr * G + h]);
-        if (mx > m_run[h] + kLazyLog2) {
-          const float corr = fast_exp2(m_run[h] - mx);  // 0 when m_run was -inf
-          l_run[h] *= corr;
-          const float2 c2 = make_float2(corr, corr);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[h][i] = __fmul2_rn(acc[h][i], c2);
-          m_run[h] = mx;
+        for (int j = 0; j < Geo::NT; ++j) {
+          oc[j][0] *= corr;
+          oc[j][1] *= corr;
         }
+        m_run = mx;
       }
+      const float p0 = x0 == -INFINITY ? 0.f : fast_exp2(x0 - m_run);
+      const float p1 = x1 == -INFINITY ? 0.f : fast_exp2(x1 - m_run);
+      const float p2 = x2 == -INFINITY ? 0.f : fast_exp2(x2 - m_run);
+      const float p3 = x3 == -INFINITY ? 0.f : fast_exp2(x3 - m_run);
+      l_run += (p0 + p1) + (p2 + p3);
+      const uint32_t pa_lo = pack_bf16x2(p0, p1), pa_hi = pack_bf16x2(p2, p3);
+      // O += P V, two n-tiles (16 columns) per ldmatrix
 #pragma unroll
-      for (int j = 0; j < Geo::KEEP; ++j) {
-        const int idx = decode_value_index<Geo::LOG_V, Geo::LOG_LPR, Geo::KS>(gl, j);
-        const int hj = idx % G;
-        float mh = m_run[0];
-#pragma unroll
-        for (int h = 1; h < G; ++h) mh = hj == h ? m_run[h] : mh;
-        sc_p[idx] = (grp * PR + idx / G < rows) ? fast_exp2(v[j] - mh) : 0.f;
+      for (int jp = 0; jp < Geo::NT / 2; ++jp) {
+        // matrices: rows (mi & 1) * 8 + mr, columns 16 jp + (mi >> 1) * 8
+        const int row = (mi & 1) * 8 + mr, chunk = ((2 * jp) & 7) + (mi >> 1);
+        uint32_t r[4];
+        ldsm_x4_trans(vb + (jp >> 2) * Geo::HALF_BYTES + row * 128 + ((chunk ^ mr) << 4), r);
+        mma_top_rows(oc[2 * jp][0], oc[2 * jp][1], pa_lo, pa_hi, r[0], r[1]);
+        mma_top_rows(oc[2 * jp + 1][0], oc[2 * jp + 1][1], pa_lo, pa_hi, r[2], r[3]);
       }
-      __syncwarp();
-      // P V over the group's rows (rows past the valid range may hold any
-      // bits, so they are skipped rather than weighted by zero)
-#pragma unroll
-      for (int rr = 0; rr < PR; ++rr) {
-        const int r = grp * PR + rr;
-        if (r < rows) {
-          float2 vf[4];
-          bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(vbuf + r * Geo::ROW_BYTES + c0 * 2), vf);
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pr = sc_p[rr * G + h];
-            l_run[h] += pr;
-            const float2 p2 = make_float2(pr, pr);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[h][i] = __ffma2_rn(p2, vf[i], acc[h][i]);
-          }
-        }
-      }
-      __syncwarp();  // every lane is done with the stage and the scratch
+      __syncwarp();  // every lane is done with the stage
       ++pc_cons;
       issue();       // refill the freed stage
     }
     if (!ok) break;
-    // merge the warp's groups (lanes gl, gl + LPR, ...) with max rescaling
-#pragma unroll
-    for (int o = 16; o >= LPR; o >>= 1) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m_run[h], o);
-        const float lo = __shfl_xor_sync(0xffffffffu, l_run[h], o);
-        const float mm = fmaxf(m_run[h], mo);
-        const float fa = (m_run[h] == -INFINITY) ? 0.f : fast_exp2(m_run[h] - mm);
-        const float fb = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mm);
-        l_run[h] = l_run[h] * fa + lo * fb;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float ax = __shfl_xor_sync(0xffffffffu, acc[h][i].x, o);
-          const float ay = __shfl_xor_sync(0xffffffffu, acc[h][i].y, o);
-          acc[h][i] = make_float2(acc[h][i].x * fa + ax * fb, acc[h][i].y * fa + ay * fb);
-        }
-        m_run[h] = mm;
-      }
-    }
+    // l of head g: the quad's lanes hold disjoint rows
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     // the split's partial of every query head: [b][kvh G + h][split][D + 2]
-    if (lane < LPR) {
+    if (g < G) {
+      // rows of D + 2 floats are only 8-byte aligned: float2 stores
+      float* part = p.part + (((long long)b * p.Hq + kvh * G + g) * p.num_splits + split) * (D + 2);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        // rows of D + 2 floats are only 8-byte aligned: float2 stores
-        float* part = p.part + (((long long)b * p.Hq + kvh * G + h) * p.num_splits + split) * (D + 2);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<float2*>(part + c0 + 2 * i) = acc[h][i];
-        if (gl == 0) {
-          part[D] = n_cur > 0 ? m_run[h] : -INFINITY;
-          part[D + 1] = n_cur > 0 ? l_run[h] : 0.f;
-        }
+      for (int j = 0; j < Geo::NT; ++j)
+        *reinterpret_cast<float2*>(part + 8 * j + 2 * t) = make_float2(oc[j][0], oc[j][1]);
+      if (t == 0) {
+        part[D] = n_cur > 0 ? m_run : -INFINITY;
+        part[D + 1] = n_cur > 0 ? l_run : 0.f;
       }
     }
     // next item; the producer side may already be streaming it
@@ -629,8 +602,8 @@ int launch_tma(const DecodeProblem& p, int chunk, cudaStream_t stream) {
   using Geo = WarpGeom<D, G>;
   const int S = p.n_sink + p.window;
   CUtensorMap mk, mv;
-  if (!make_tmap_3d_rows(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, Geo::R) ||
-      !make_tmap_3d_rows(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, Geo::R))
+  if (!make_tmap_3d(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, Geo::R) ||
+      !make_tmap_3d(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, Geo::R))
     return SINKATTN_ERR_CUDA;
   auto kern = decode_warp_kernel<D, G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM) !=

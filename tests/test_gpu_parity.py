@@ -253,7 +253,8 @@ def test_decode_partial_fill_and_splits(splits):
 @pytest.mark.parametrize("G,D,splits", [(8, 128, 0), (8, 64, 5), (1, 128, 40), (2, 64, 97)])
 def test_decode_heads_and_many_splits(G, D, splits):
     # 40 and 97 splits put several rounds of split partials in the merge
-    # (32 per warp pass); 8 query heads per KV head use the 8-row pieces
+    # (32 per warp pass); 8 query heads per KV head fill the whole shared
+    # memory and stage fewer cache lengths
     d = W.decode(B=5, n_sink=4, window=1500, Hq=2 * G, Hkv=2, D=D, seqlen_range=(0, 3000))
     _compare_decode(d, *_run_decode(d, splits), TOL[torch.bfloat16])
 
@@ -263,6 +264,22 @@ def test_decode_many_sequences():
     # shared memory (1024): the lengths are then read from global memory
     d = W.decode(B=1100, n_sink=2, window=30, Hq=2, Hkv=1, D=64, seqlen_range=(0, 40))
     _compare_decode(d, *_run_decode(d), TOL[torch.bfloat16])
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_ignores_nan_in_unfilled_slots(D):
+    # slots past a sequence's fill hold whatever the cache held; a NaN or inf
+    # there must not reach the output (the streaming kernel reads those rows
+    # as part of a whole piece)
+    d = W.decode(B=6, n_sink=4, window=60, Hq=8, Hkv=2, D=D, seqlen_range=(0, 70))
+    d.cache_seqlens = torch.tensor([0, 1, 5, 17, 33, 47], dtype=torch.int32)
+    S_ = d.n_sink + d.window
+    for b, n in enumerate(d.cache_seqlens.tolist()):
+        if n < S_:
+            d.k_cache[b, n:] = float("nan")
+            d.v_cache[b, n:] = float("inf") if b % 2 else float("nan")
+    for splits in (1, 3):
+        _compare_decode(d, *_run_decode(d, splits), TOL[torch.bfloat16])
 
 
 def test_decode_fp32_no_sink():
