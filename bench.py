@@ -244,6 +244,43 @@ def measure_config(S, inp, dev, steps=10, warmup=3):
             "bwd_kernel_ms": b_ms, "bwd_kernel_tflops": 10 * D * pairs / (b_ms * 1e-3) / 1e12}
 
 
+def measure_gates(S, q, k, lse, sink_s, mask, scale, flush, flush_rd, hbm_gbs, reps=10):
+    """Gate rows on the prefill's tensors: the sink-free model's gate (reads Q
+    once; Q is larger than L2) and the head importance (reads sink_s once;
+    L2 flushed before each call).  CUDA events around each call."""
+    T, Hq, D = q.shape
+    gate = torch.empty(T, Hq, dtype=torch.float32, device=q.device)
+    imp = torch.empty(Hq, dtype=torch.float32, device=q.device)
+    iws = torch.empty(max(16, S.lib().sinkattn_gate_importance_workspace_bytes(T, Hq)),
+                      dtype=torch.uint8, device=q.device)
+    n_seq = mask.cu_seqlens.numel() - 1
+    res = {}
+    for name, call, nbytes, cold in (
+            ("gate_vanilla", lambda: S.gate_vanilla(q, k, lse, mask, scale=scale, gate=gate),
+             q.numel() * q.element_size() + 8 * T * Hq + n_seq * k.shape[1] * D * k.element_size(),
+             False),
+            ("gate_importance", lambda: S.gate_importance(sink_s, workspace=iws, imp=imp),
+             4 * T * Hq, True)):
+        for _ in range(3):
+            call()
+        ts = []
+        for _ in range(reps):
+            if cold:
+                flush.zero_()
+                flush_rd.sum()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = sorted(ts)[len(ts) // 2]
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": ms, "bytes": nbytes, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm_gbs}
+    return res
+
+
 def run_ours(args, world, rank, local):
     from learnable_sink_b200 import sinkattn as S
     dev = torch.device("cuda", local)
@@ -418,6 +455,8 @@ def run_ours(args, world, rank, local):
 
     if rank != 0:
         return
+    gates = measure_gates(S, q, k, lse, sink_s, mask, inp.scale, flush, flush_rd,
+                          peaks["hbm_gbs"])
     clocks = clk.summary()
     peak_tf = peaks["bf16_tflops_sustained"]
     bwd_ach = flop_bwd / (kb_ms * 1e-3) / 1e12
@@ -461,6 +500,9 @@ def run_ours(args, world, rank, local):
             "decode_warp_kernel": {"ms": kd_ms, "achieved_gbs": dec_ach,
                                     "frac_of_hbm": dec_ach / peaks["hbm_gbs"]},
         },
+        # gate rows, timed after the main region on the prefill's tensors
+        # (median of 10 calls): not part of the step
+        "gates": gates,
     }
     if args.configs:
         extra = []

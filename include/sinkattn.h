@@ -232,6 +232,27 @@ size_t sinkattn_gate_importance_workspace_bytes(int T_tot, int Hq);
 int sinkattn_gate_importance(int T_tot, int Hq, const float *sink_s, float *imp,
                              void *workspace, size_t workspace_bytes, sinkattn_stream_t stream);
 
+/* ---- gate of a sink-free model ------------------------------------------------
+ * For a model without a learnable sink whose attention sink is the first
+ * token k_0 of each sequence, page "Attention Sink and the native MoE in
+ * attention layers" (section 5) forms the gate from the LSE the attention
+ * forward returns: G = sigma(LSE_not0 - q.k_0 * scale), LSE_not0 the
+ * log-sum-exp over the visible keys other than k_0.  With L the sink-free
+ * LSE over all visible keys, G = 1 - exp(x_0 - L), x_0 = scale <q, k_0>.
+ *   q, k      the forward's inputs (type dt, layouts above, D = 64 or 128).
+ *   lse       float32 [T_tot, Hq]: lse_new of sinkattn_fwd run with
+ *             learnable_sink = NULL, or lse_orig of sinkattn_fwd_ex, over the
+ *             same mask.
+ *   mask      the forward's mask (k_0 is visible to query qi unless a window
+ *             without sink tokens has passed it, qi >= window with n_sink = 0,
+ *             or the block lists leave out key block 0).
+ *   gate      float32 [T_tot, Hq] (written): 1 for a row that does not see
+ *             k_0, 0 for a row that sees no key (lse = -inf).
+ * Reads Q once; no workspace. */
+int sinkattn_gate_vanilla(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                          const void *q, const void *k, const float *lse,
+                          const sinkattn_mask *mask, float *gate, sinkattn_stream_t stream);
+
 /* ---- ring-buffer decode ---------------------------------------------------
  * One query token per sequence attends over a StreamingLLM KV cache: n_sink
  * fixed slots holding the first tokens plus a circular window of `window`

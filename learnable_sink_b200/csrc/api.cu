@@ -271,6 +271,36 @@ int sinkattn_bwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float 
   return launch_bwd_tc(p, b, s);
 }
 
+int sinkattn_gate_vanilla(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
+                          const void* q, const void* k, const float* lse,
+                          const sinkattn_mask* mask, float* gate, sinkattn_stream_t stream) {
+  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SINKATTN_ERR_INVALID_ARG;
+  if (!mask_ok(T_tot, Hq, Hkv, mask)) return SINKATTN_ERR_INVALID_ARG;
+  if (!q || !k || !lse || !gate) return SINKATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(lse) || !aligned16(gate))
+    return SINKATTN_ERR_INVALID_ARG;
+  if (mask->n_seq > 65535) return SINKATTN_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return SINKATTN_ERR_UNSUPPORTED;
+  GateVanillaArgs a{};
+  a.q = q;
+  a.k = k;
+  a.lse = lse;
+  a.gate = gate;
+  a.cu = mask->cu_seqlens;
+  a.bi = mask->block_indices;
+  a.n_seq = mask->n_seq;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.n_sink = mask->n_sink;
+  a.window = mask->window;
+  a.n_qblk = mask->block_indices ? mask->n_qblk : 0;
+  a.block_q = mask->block_q;
+  a.max_blocks = mask->block_indices ? mask->max_blocks : 0;
+  a.scale = scale;
+  return launch_gate_vanilla(a, dt, D, mask->max_seqlen, reinterpret_cast<cudaStream_t>(stream));
+}
+
 // the split merge handles up to this many splits
 constexpr int kMaxDecodeSplits = 128;
 

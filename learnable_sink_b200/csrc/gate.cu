@@ -70,7 +70,136 @@ __global__ void gate_reduce_kernel(const double* part, int n_blocks, int Hq, int
   if (lane == 0) imp[h] = (float)(s / (double)T_tot);
 }
 
+// Gate of a sink-free model whose attention sink is the first token k_0 of
+// each sequence (same page, section 5): G = sigma(LSE_not0 - x_0), x_0 =
+// scale <q, k_0>.  With L = the sink-free forward's LSE over the visible set,
+// L = logaddexp(LSE_not0, x_0), so G = 1 - e^(x_0 - L) = -expm1(x_0 - L): one
+// dot product per (token, head) and the LSE the forward already wrote.  A row
+// that does not see k_0 gets 1, a row that sees no key (L = -inf) gets 0.
+// One warp per token, eight heads' Q rows in flight at once; HBM-bound
+// (reads Q once).  CTA = kGvRows tokens of one sequence.
+constexpr int kGvRows = 32;
+constexpr int kGvHeads = 8;
+
+template <typename T, int D>
+struct QFrag {
+  static constexpr int E = D / 32;  // elements per lane
+  float v[E];
+  __device__ __forceinline__ void load(const T* row, int lane) {
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(row) + lane * E;
+      if constexpr (E == 4) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+      } else {
+        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(p));
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+        v[0] = a.x; v[1] = a.y;
+      }
+    } else {
+      if constexpr (E == 4) {
+        const float4 u = __ldg(reinterpret_cast<const float4*>(row) + lane);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+      } else {
+        const float2 u = __ldg(reinterpret_cast<const float2*>(row) + lane);
+        v[0] = u.x; v[1] = u.y;
+      }
+    }
+  }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
+  const int s = blockIdx.y;
+  const int start = __ldg(a.cu + s), len = __ldg(a.cu + s + 1) - start;
+  const int i0 = blockIdx.x * kGvRows;
+  if (i0 >= len) return;  // uniform over the CTA
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // block-sparse lists are indexed by query blocks numbered over all
+  // sequences: count the blocks of the sequences before s
+  __shared__ int red[8];
+  int qb_base = 0;
+  if (a.bi) {
+    int acc = 0;
+    for (int j = threadIdx.x; j < s; j += blockDim.x) {
+      const int l = __ldg(a.cu + j + 1) - __ldg(a.cu + j);
+      acc += (l + a.block_q - 1) / a.block_q;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) red[warp] = acc;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < 8; ++w) qb_base += red[w];
+  }
+  const int G = a.Hq / a.Hkv;
+  const T* k0 = static_cast<const T*>(a.k) + (long long)start * a.Hkv * D;
+  for (int i = i0 + warp; i < min(len, i0 + kGvRows); i += 8) {
+    const long long t = start + i;
+    const T* qrow = static_cast<const T*>(a.q) + t * a.Hq * D;
+    // is k_0 visible to query i (sequence-local)?  causal: always (0 <= i)
+    bool vis_band = a.window == 0 || a.n_sink > 0 || i < a.window;
+    for (int h0 = 0; h0 < a.Hq; h0 += kGvHeads) {
+      QFrag<T, D> qf[kGvHeads], kf[kGvHeads];
+#pragma unroll
+      for (int u = 0; u < kGvHeads; ++u) {
+        const int h = min(h0 + u, a.Hq - 1);
+        qf[u].load(qrow + (long long)h * D, lane);
+        kf[u].load(k0 + (long long)(h / G) * D, lane);
+      }
+      float dot[kGvHeads];
+#pragma unroll
+      for (int u = 0; u < kGvHeads; ++u) {
+        dot[u] = 0.f;
+#pragma unroll
+        for (int e = 0; e < QFrag<T, D>::E; ++e) dot[u] = fmaf(qf[u].v[e], kf[u].v[e], dot[u]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < kGvHeads; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+      // lane u writes head h0 + u
+      float mine = 0.f;
+#pragma unroll
+      for (int u = 0; u < kGvHeads; ++u) mine = lane == u ? dot[u] : mine;
+      const int h = h0 + lane;
+      if (lane < kGvHeads && h < a.Hq) {
+        bool vis = vis_band;
+        if (a.bi && vis) {
+          const int qb = qb_base + i / a.block_q;
+          vis = false;
+          if (qb < a.n_qblk) {
+            const int32_t* lst = a.bi + ((long long)(h / G) * a.n_qblk + qb) * a.max_blocks;
+            for (int e = 0; e < a.max_blocks; ++e) vis |= __ldg(lst + e) == 0;
+          }
+        }
+        const float l = __ldg(a.lse + t * a.Hq + h);
+        float gv;
+        if (l == -INFINITY) gv = 0.f;
+        else if (!vis) gv = 1.f;
+        else gv = fmaxf(0.f, -expm1f(mine * a.scale - l));
+        a.gate[t * a.Hq + h] = gv;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+int launch_gate_vanilla(const GateVanillaArgs& a, int dt, int D, int max_seqlen,
+                        cudaStream_t stream) {
+  const dim3 grid((max_seqlen + kGvRows - 1) / kGvRows, a.n_seq);
+  if (dt == SINKATTN_BF16) {
+    if (D == 64) gate_vanilla_kernel<__nv_bfloat16, 64><<<grid, 256, 0, stream>>>(a);
+    else gate_vanilla_kernel<__nv_bfloat16, 128><<<grid, 256, 0, stream>>>(a);
+  } else {
+    if (D == 64) gate_vanilla_kernel<float, 64><<<grid, 256, 0, stream>>>(a);
+    else gate_vanilla_kernel<float, 128><<<grid, 256, 0, stream>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
 
 }  // namespace sk
 

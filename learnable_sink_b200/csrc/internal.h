@@ -88,6 +88,20 @@ int launch_bwd_simt(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stre
 int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream);
 size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int Hkv, int D);
 
+// gate of a sink-free model (sink = first token of each sequence)
+struct GateVanillaArgs {
+  const void* q;
+  const void* k;
+  const float* lse;
+  float* gate;
+  const int32_t* cu;
+  const int32_t* bi;
+  int n_seq, Hq, Hkv, n_sink, window, n_qblk, block_q, max_blocks;
+  float scale;
+};
+int launch_gate_vanilla(const GateVanillaArgs& a, int dt, int D, int max_seqlen,
+                        cudaStream_t stream);
+
 // decode
 struct DecodeProblem {
   int dt, B, Hq, Hkv, D, n_sink, window, num_splits;

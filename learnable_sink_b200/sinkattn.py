@@ -73,6 +73,8 @@ def lib():
         L.sinkattn_gate_importance_workspace_bytes.restype = _sz
         L.sinkattn_gate_importance_workspace_bytes.argtypes = [_i, _i]
         L.sinkattn_gate_importance.argtypes = [_i, _i, _vp, _vp, _vp, _sz, _vp]
+        L.sinkattn_gate_vanilla.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, M,
+                                            _vp, _vp]
         L.sinkattn_decode_workspace_bytes.restype = _sz
         L.sinkattn_decode_workspace_bytes.argtypes = [_i, _i, _i, _i]
         L.sinkattn_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
@@ -246,6 +248,20 @@ def gate_importance(sink_s, stream=None, workspace=None, imp=None):
     _check("sinkattn_gate_importance", lib().sinkattn_gate_importance(
         T, Hq, _ptr(sink_s), _ptr(imp), _ptr(workspace), workspace.numel(), _stream(stream)))
     return imp
+
+
+def gate_vanilla(q, k, lse, mask: Mask, scale: Optional[float] = None, stream=None, gate=None):
+    """Gate sigma(LSE_not0 - q.k_0 scale) [T, Hq] of a sink-free model whose
+    sink is each sequence's first token; ``lse`` is the sink-free LSE."""
+    _contig(q, k, lse, gate)
+    T, Hq, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    cm = mask.c()
+    gate = torch.empty(T, Hq, dtype=torch.float32, device=q.device) if gate is None else gate
+    _check("sinkattn_gate_vanilla", lib().sinkattn_gate_vanilla(
+        _dt(q), T, Hq, k.shape[1], D, scale, _ptr(q), _ptr(k), _ptr(lse), _c.byref(cm),
+        _ptr(gate), _stream(stream)))
+    return gate
 
 
 def decode_num_splits(B, Hq, Hkv, D, n_sink, window) -> int:

@@ -213,6 +213,41 @@ def gate_aux_loss(imp, lam=1.0, n_shared=0):
     return float(loss), d_imp
 
 
+def gate_vanilla(q, k, scale, **mask):
+    """Gate of a sink-free model whose sink is the first token of each
+    sequence (page "Attention Sink and the native MoE in attention layers",
+    section 5): G = sigma(LSE_not0 - x_0) with x_0 = scale <q, k_0> and LSE_not0
+    the log-sum-exp of the visible keys other than k_0.  Readings: a row that
+    does not see k_0 puts no mass on it (G = 1); a row that sees no key gets
+    G = 0.  Brute force over the visible set.  Returns [T, Hq] float64."""
+    q, k = _f64(q), _f64(k)
+    T, Hq, Hkv, D = _shapes(q, k)
+    G = Hq // Hkv
+    cu = _Problem(T, Hq, Hkv, D, scale, **mask).cu
+    vis = [visible_dense(T, Hq, Hkv, g, **mask) for g in range(Hkv)]
+    out = np.zeros((T, Hq))
+    with np.errstate(over="ignore"):
+        for s in range(len(cu) - 1):
+            j0 = int(cu[s])
+            for i in range(int(cu[s]), int(cu[s + 1])):
+                for h in range(Hq):
+                    keys = np.nonzero(vis[h // G][i])[0]
+                    if keys.size == 0:
+                        continue
+                    if j0 not in keys:
+                        out[i, h] = 1.0
+                        continue
+                    x = scale * (k[keys, h // G] @ q[i, h])
+                    x0 = x[keys == j0][0]
+                    rest = x[keys != j0]
+                    if rest.size == 0:
+                        continue  # only k_0 is seen: all mass on it
+                    m = rest.max()
+                    lse_not0 = m + np.log(np.exp(rest - m).sum())
+                    out[i, h] = 1.0 / (1.0 + np.exp(-(lse_not0 - x0)))
+    return out
+
+
 def decode(q, k_cache, v_cache, cache_seqlens, n_sink, window, sink, scale):
     """Ring-buffer decode. q [B,Hq,D], caches [B,S,Hkv,D] (S = n_sink+window).
     Returns (out [B,Hq,D], lse_new [B,Hq], sink_s [B,Hq])."""

@@ -133,3 +133,50 @@ def test_balance_loss_gradient_through_backward(n_shared):
     grads = _bwd_with_gate_grad(inp, dss, out, lse, m, plan)
     _check(inp, dss, grads)
     assert float(grads[2].abs().max()) == 0.0
+
+
+# ------------------------------------------------------ gate of a sink-free model
+
+VANILLA_CASES = {
+    "bf16_causal_ragged_D128": dict(cu=[0, 300, 555], Hq=8, Hkv=2, D=128, dtype=torch.bfloat16),
+    "bf16_band_no_sink_tokens": dict(cu=[0, 200, 333], Hq=4, Hkv=2, D=64, dtype=torch.bfloat16,
+                                     window=37),
+    "bf16_band_with_sink_tokens": dict(cu=[0, 260], Hq=8, Hkv=1, D=128, dtype=torch.bfloat16,
+                                       n_sink=4, window=50),
+    "fp32_causal_D64": dict(cu=[0, 1, 130, 300], Hq=4, Hkv=4, D=64, dtype=torch.float32),
+    "bf16_block_sparse": dict(cu=None, Hq=8, Hkv=2, D=64, dtype=torch.bfloat16),
+}
+
+
+def _vanilla_inputs(name):
+    kw = dict(VANILLA_CASES[name])
+    cu = kw.pop("cu")
+    if cu is None:
+        cu_t = torch.tensor([0, 200, 450, 700], dtype=torch.int32)
+        bi = W.random_block_indices(cu_t, kw["Hkv"], 64, 64, 2, 51)
+        bi[:, 1, :] = torch.where(bi[:, 1, :] == 0, -1, bi[:, 1, :])  # a block that skips k_0
+        mask = W.MaskSpec(causal=True, cu_seqlens=cu_t, block_indices=bi, block_q=64, block_k=64)
+        T = 700
+    else:
+        mask = spec(cu, kw.pop("n_sink", 0), kw.pop("window", 0))
+        T = cu[-1]
+    return W.make_attn(name, T_tot=T, mask=mask, seed=52, sink_std=None, **kw)
+
+
+@pytest.mark.parametrize("name", list(VANILLA_CASES))
+def test_vanilla_gate(name):
+    inp = _vanilla_inputs(name)
+    ref = oracle.gate_vanilla(inp.q, inp.k, inp.scale, **inp.mask.oracle_kwargs())
+    m = S.Mask.from_spec(inp.mask)
+    # the gate kernel alone, on the oracle's sink-free LSE
+    _, rl, _ = oracle.fwd(inp.q, inp.k, inp.v, None, inp.scale, **inp.mask.oracle_kwargs())
+    lse = torch.from_numpy(rl).float().cuda()
+    got = S.gate_vanilla(dev(inp.q), dev(inp.k), lse, m, scale=inp.scale)
+    torch.cuda.synchronize()
+    assert np.abs(np64(got) - ref).max() <= 2e-5
+    # through the library's own sink-free forward
+    _, lse_f, _, m, _ = run_fwd(inp)
+    got = S.gate_vanilla(dev(inp.q), dev(inp.k), lse_f, m, scale=inp.scale)
+    torch.cuda.synchronize()
+    err = np.abs(np64(got) - ref).max()
+    assert err <= TOL[inp.q.dtype]["ss"], f"gate max abs {err:.3e}"

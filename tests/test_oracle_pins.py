@@ -371,6 +371,47 @@ def test_gate_aux_loss_closed_forms_and_gradient():
             assert abs(fd - d[h]) < 1e-6, (m, h, fd, d[h])
 
 
+@pytest.mark.parametrize("mname", ["causal", "band", "varlen_band", "block_sparse"])
+def test_vanilla_gate_is_one_minus_first_token_probability(mname):
+    """sigma(LSE_not0 - x_0) equals 1 - P(k_0) of the sink-free softmax; P(k_0)
+    is read from the oracle's forward with V one-hot on each sequence's first
+    token (an independent route through the attention forward)."""
+    T, Hq, Hkv, D = 37, 4, 2, 16
+    mask = MASKS[mname] if mname != "block_sparse" else _block_sparse_mask()
+    q, k, _, _, _ = _random_problem(T, Hq, Hkv, D, seed=31)
+    scale = 0.7
+    cu = mask["cu_seqlens"]
+    v = np.zeros((T, Hkv, D))
+    v[cu[:-1], :, 0] = 1.0
+    o, lse, _ = oracle.fwd(q, k, v, None, scale, **mask)
+    gate = oracle.gate_vanilla(q, k, scale, **mask)
+    seen = np.isfinite(lse)
+    np.testing.assert_allclose(gate[seen], 1.0 - o[..., 0][seen], atol=1e-12)
+    assert np.all(gate[~seen] == 0.0)
+
+
+def test_vanilla_gate_closed_forms():
+    """q = 0: every visible key scores 0, so the first token holds 1/n of the
+    mass and G = 1 - 1/n under a causal mask; the first token of a sequence
+    sees only itself (G = 0); a band without sink tokens hides k_0 from
+    queries past the window (G = 1)."""
+    T, Hq, Hkv, D = 20, 2, 1, 8
+    q = np.zeros((T, Hq, D)); k = np.random.default_rng(32).standard_normal((T, Hkv, D))
+    cu = np.array([0, 8, 20], dtype=np.int32)
+    gate = oracle.gate_vanilla(q, k, 1.0, causal=True, cu_seqlens=cu)
+    for s in range(2):
+        n = np.arange(1, cu[s + 1] - cu[s] + 1)
+        np.testing.assert_allclose(gate[cu[s]:cu[s + 1]], (1 - 1 / n)[:, None].repeat(Hq, 1),
+                                   atol=1e-15)
+    q = np.random.default_rng(33).standard_normal((T, Hq, D))
+    gate = oracle.gate_vanilla(q, k, 1.0, causal=True, window=3, cu_seqlens=cu)
+    assert np.all(gate[cu[:-1]] == 0.0)
+    for s in range(2):
+        for i in range(cu[s], cu[s + 1]):
+            if i - cu[s] >= 3:
+                assert np.all(gate[i] == 1.0)
+
+
 def test_relative_probabilities_unchanged_by_sink():
     T, Hq, Hkv = 9, 2, 1
     rng = np.random.default_rng(7)
