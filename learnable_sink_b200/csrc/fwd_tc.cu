@@ -30,6 +30,13 @@ namespace {
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows > 2^8
 
+// max of three floats in one instruction (sm_100 three-input max.f32)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int D_, int TQ_, int TK_, int NQT_>
 struct FwdCfg {
   static constexpr int D = D_, TQ = TQ_, TK = TK_, NQT = NQT_;
@@ -265,14 +272,20 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       if (!ok) break;
       tc_fence_after();
       // raw scores x = Q.K (the scale is folded into the exponent below)
+      // all TK / 32 loads in flight, one wait for them together
       float x[TK];
+      {
+        uint32_t rr[TK / 32][32];
 #pragma unroll
-      for (int c = 0; c < TK / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(s_addr + c * 32, rr);
+        for (int c = 0; c < TK / 32; ++c) tmem_ld32(s_addr + c * 32, rr[c]);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(rr[i]);
+        for (int c = 0; c < TK / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            asm volatile("" : "+r"(rr[c][i]));  // the values exist only after the wait
+            x[c * 32 + i] = __uint_as_float(rr[c][i]);
+          }
       }
       if (e & 1) {  // partial tile: element mask
 #pragma unroll
@@ -284,10 +297,14 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
 #pragma unroll
       for (int a = 0; a < 8; ++a) m8[a] = x[a];
 #pragma unroll
-      for (int c = 8; c < TK; ++c) m8[c & 7] = fmaxf(m8[c & 7], x[c]);
+      for (int k = 1; k < TK / 8; k += 2) {
 #pragma unroll
-      for (int a = 0; a < 4; ++a) m8[a] = fmaxf(m8[a], m8[a + 4]);
-      const float mraw = fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3]));
+        for (int a = 0; a < 8; ++a)
+          m8[a] = k + 1 < TK / 8 ? fmax3(m8[a], x[8 * k + a], x[8 * k + 8 + a])
+                                 : fmaxf(m8[a], x[8 * k + a]);
+      }
+      const float mraw = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
       const float mx = mraw * p.scale_log2;  // scale > 0: max commutes with it
       // Lazy rescale: the running reference max m only moves when the tile
       // max exceeds it by more than 2^8.  Per-row decision, but the TMEM
@@ -316,24 +333,28 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       }
       if (need) m = mx;
       const float mu = (m == -INFINITY) ? 0.f : m;
-      float rs8[8];
+      // p = 2^(x * alpha * log2(e) - m): the scaling FMA and the row sums run
+      // on element pairs (packed fp32x2 instructions), the exponentials one
+      // by one
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mu, -mu);
+      float2 rs4[4];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) rs8[a] = 0.f;
+      for (int a = 0; a < 4; ++a) rs4[a] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < TK / 64; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          // p = 2^(x * alpha * log2(e) - m): one FMA feeding the exponential
-          const float p0 = fast_exp2(fmaf(x[c * 64 + 2 * i], p.scale_log2, -mu));
-          const float p1 = fast_exp2(fmaf(x[c * 64 + 2 * i + 1], p.scale_log2, -mu));
-          rs8[(2 * i) & 7] += p0;
-          rs8[(2 * i + 1) & 7] += p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          const float2 y = __ffma2_rn(make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]), sc2, nm2);
+          const float2 pp = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          rs4[i & 3] = __fadd2_rn(rs4[i & 3], pp);
+          pk[i] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st32(s_addr + c * 32, pk);  // P over the first TK/2 columns of S_t
       }
-      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      const float2 r01 = __fadd2_rn(rs4[0], rs4[1]), r23 = __fadd2_rn(rs4[2], rs4[3]);
+      const float2 rsum = __fadd2_rn(r01, r23);
+      l += rsum.x + rsum.y;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p + t);

@@ -76,42 +76,35 @@ __global__ void gate_reduce_kernel(const double* part, int n_blocks, int Hq, int
 // L = logaddexp(LSE_not0, x_0), so G = 1 - e^(x_0 - L) = -expm1(x_0 - L): one
 // dot product per (token, head) and the LSE the forward already wrote.  A row
 // that does not see k_0 gets 1, a row that sees no key (L = -inf) gets 0.
-// One warp per token, eight heads' Q rows in flight at once; HBM-bound
-// (reads Q once).  CTA = kGvRows tokens of one sequence.
+// HBM-bound (reads Q once).  A warp streams one token's contiguous Q row
+// [Hq, D] as 16-byte chunks, kGvInFlight per lane in flight; the CPH chunks
+// of a head row sit in CPH adjacent lanes, which reduce its dot product.
+// CTA = kGvRows tokens of one sequence.
 constexpr int kGvRows = 32;
-constexpr int kGvHeads = 8;
+constexpr int kGvInFlight = 8;
 
-template <typename T, int D>
-struct QFrag {
-  static constexpr int E = D / 32;  // elements per lane
-  float v[E];
-  __device__ __forceinline__ void load(const T* row, int lane) {
-    if constexpr (sizeof(T) == 2) {
-      const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(row) + lane * E;
-      if constexpr (E == 4) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-      } else {
-        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(p));
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-        v[0] = a.x; v[1] = a.y;
-      }
-    } else {
-      if constexpr (E == 4) {
-        const float4 u = __ldg(reinterpret_cast<const float4*>(row) + lane);
-        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-      } else {
-        const float2 u = __ldg(reinterpret_cast<const float2*>(row) + lane);
-        v[0] = u.x; v[1] = u.y;
-      }
+template <typename T>
+__device__ __forceinline__ float dot16(const uint4& a, const uint4& b) {
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+      s = fmaf(u.x, v.x, s);
+      s = fmaf(u.y, v.y, s);
     }
+    return s;
+  } else {
+    return __uint_as_float(a.x) * __uint_as_float(b.x) + __uint_as_float(a.y) * __uint_as_float(b.y) +
+           __uint_as_float(a.z) * __uint_as_float(b.z) + __uint_as_float(a.w) * __uint_as_float(b.w);
   }
-};
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
+  constexpr int CPH = D * (int)sizeof(T) / 16;  // 16-byte chunks per head row: 8, 16 or 32
   const int s = blockIdx.y;
   const int start = __ldg(a.cu + s), len = __ldg(a.cu + s + 1) - start;
   const int i0 = blockIdx.x * kGvRows;
@@ -135,52 +128,52 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
     for (int w = 0; w < 8; ++w) qb_base += red[w];
   }
   const int G = a.Hq / a.Hkv;
-  const T* k0 = static_cast<const T*>(a.k) + (long long)start * a.Hkv * D;
+  const int n16 = a.Hq * CPH;  // chunks per token row
+  const uint4* k0 = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k) +
+                                                   (long long)start * a.Hkv * D);
   for (int i = i0 + warp; i < min(len, i0 + kGvRows); i += 8) {
     const long long t = start + i;
-    const T* qrow = static_cast<const T*>(a.q) + t * a.Hq * D;
+    const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + t * a.Hq * D);
     // is k_0 visible to query i (sequence-local)?  causal: always (0 <= i)
-    bool vis_band = a.window == 0 || a.n_sink > 0 || i < a.window;
-    for (int h0 = 0; h0 < a.Hq; h0 += kGvHeads) {
-      QFrag<T, D> qf[kGvHeads], kf[kGvHeads];
+    const bool vis_band = a.window == 0 || a.n_sink > 0 || i < a.window;
+    for (int c0 = 0; c0 < n16; c0 += 32 * kGvInFlight) {
+      uint4 qv[kGvInFlight], kv[kGvInFlight];
 #pragma unroll
-      for (int u = 0; u < kGvHeads; ++u) {
-        const int h = min(h0 + u, a.Hq - 1);
-        qf[u].load(qrow + (long long)h * D, lane);
-        kf[u].load(k0 + (long long)(h / G) * D, lane);
+      for (int u = 0; u < kGvInFlight; ++u) {
+        const int c = min(c0 + u * 32 + lane, n16 - 1);
+        const int h = c / CPH;
+        qv[u] = __ldg(qrow + c);
+        kv[u] = __ldg(k0 + (h / G) * CPH + (c - h * CPH));
       }
-      float dot[kGvHeads];
+      float dot[kGvInFlight];
 #pragma unroll
-      for (int u = 0; u < kGvHeads; ++u) {
-        dot[u] = 0.f;
+      for (int u = 0; u < kGvInFlight; ++u) dot[u] = dot16<T>(qv[u], kv[u]);
 #pragma unroll
-        for (int e = 0; e < QFrag<T, D>::E; ++e) dot[u] = fmaf(qf[u].v[e], kf[u].v[e], dot[u]);
-      }
+      for (int o = CPH / 2; o > 0; o >>= 1)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
+        for (int u = 0; u < kGvInFlight; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+      // the first lane of each head's group writes that head
 #pragma unroll
-        for (int u = 0; u < kGvHeads; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
-      // lane u writes head h0 + u
-      float mine = 0.f;
-#pragma unroll
-      for (int u = 0; u < kGvHeads; ++u) mine = lane == u ? dot[u] : mine;
-      const int h = h0 + lane;
-      if (lane < kGvHeads && h < a.Hq) {
-        bool vis = vis_band;
-        if (a.bi && vis) {
-          const int qb = qb_base + i / a.block_q;
-          vis = false;
-          if (qb < a.n_qblk) {
-            const int32_t* lst = a.bi + ((long long)(h / G) * a.n_qblk + qb) * a.max_blocks;
-            for (int e = 0; e < a.max_blocks; ++e) vis |= __ldg(lst + e) == 0;
+      for (int u = 0; u < kGvInFlight; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < n16 && (lane % CPH) == 0) {
+          const int h = c / CPH;
+          bool vis = vis_band;
+          if (a.bi && vis) {
+            const int qb = qb_base + i / a.block_q;
+            vis = false;
+            if (qb < a.n_qblk) {
+              const int32_t* lst = a.bi + ((long long)(h / G) * a.n_qblk + qb) * a.max_blocks;
+              for (int e = 0; e < a.max_blocks; ++e) vis |= __ldg(lst + e) == 0;
+            }
           }
+          const float l = __ldg(a.lse + t * a.Hq + h);
+          float gv;
+          if (l == -INFINITY) gv = 0.f;
+          else if (!vis) gv = 1.f;
+          else gv = fmaxf(0.f, -expm1f(dot[u] * a.scale - l));
+          a.gate[t * a.Hq + h] = gv;
         }
-        const float l = __ldg(a.lse + t * a.Hq + h);
-        float gv;
-        if (l == -INFINITY) gv = 0.f;
-        else if (!vis) gv = 1.f;
-        else gv = fmaxf(0.f, -expm1f(mine * a.scale - l));
-        a.gate[t * a.Hq + h] = gv;
       }
     }
   }
