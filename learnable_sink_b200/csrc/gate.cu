@@ -137,6 +137,11 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
     // is k_0 visible to query i (sequence-local)?  causal: always (0 <= i)
     const bool vis_band = a.window == 0 || a.n_sink > 0 || i < a.window;
     for (int c0 = 0; c0 < n16; c0 += 32 * kGvInFlight) {
+      // the batch covers heads hb0 .. hb0 + 32 kGvInFlight / CPH - 1 (at most
+      // 32): lane j loads head hb0 + j's LSE together with the Q chunks
+      const int hb0 = c0 / CPH;
+      const int hj = min(hb0 + lane, a.Hq - 1);
+      const float lse_b = __ldg(a.lse + t * a.Hq + hj);
       uint4 qv[kGvInFlight], kv[kGvInFlight];
 #pragma unroll
       for (int u = 0; u < kGvInFlight; ++u) {
@@ -156,6 +161,7 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
 #pragma unroll
       for (int u = 0; u < kGvInFlight; ++u) {
         const int c = c0 + u * 32 + lane;
+        const float l = __shfl_sync(0xffffffffu, lse_b, (min(c, n16 - 1) / CPH - hb0) & 31);
         if (c < n16 && (lane % CPH) == 0) {
           const int h = c / CPH;
           bool vis = vis_band;
@@ -167,7 +173,6 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
               for (int e = 0; e < a.max_blocks; ++e) vis |= __ldg(lst + e) == 0;
             }
           }
-          const float l = __ldg(a.lse + t * a.Hq + h);
           float gv;
           if (l == -INFINITY) gv = 0.f;
           else if (!vis) gv = 1.f;
