@@ -36,15 +36,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   }
 }
 
-// bf16 -> fp32 is exact and needs only the 16 bits moved up: integer ops,
-// no conversion unit.  Pair i holds elements 2i (low half) and 2i + 1.
-__device__ __forceinline__ void bf16x8_to_f32x2(const uint4& u, float2 (&f)[4]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-}
-
 // The streaming decode moves its running maximum only past this margin
 // (log2 units): probabilities stay below 2^8, far from fp32 overflow.
 constexpr float kLazyLog2 = 8.f;

@@ -475,21 +475,6 @@ bool make_tmap_3d_plain(CUtensorMap* map, const void* base, int T, int H, int D,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Whole rows, without swizzle: box {D, box_h, box_t} lands as plain rows of D
-// elements, so a row of one head (2 D bytes) is one request.
-bool make_tmap_3d_rows(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
-                       int box_t) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)box_h, (cuuint32_t)box_t};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // fp32 [T, H, D] map with 32-element (128-byte) boxes {32, box_h, box_t},
 // 128-byte swizzle: used to add dQ tiles into the fp32 accumulator.
 bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,

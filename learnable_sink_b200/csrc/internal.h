@@ -53,8 +53,6 @@ struct AttnProblem {
 bool make_tmap_3d(CUtensorMap* map, const void* base, int T, int H, int D, int box_h, int box_t);
 bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
                       int box_t);
-bool make_tmap_3d_rows(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
-                       int box_t);
 bool make_tmap_3d_plain(CUtensorMap* map, const void* base, int T, int H, int D, int box_h,
                         int box_t);
 
