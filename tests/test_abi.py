@@ -87,3 +87,23 @@ def test_gate_importance_host_validation(lib):
     assert f(16, 0, None, None, None, 0, None) == 1     # Hq < 1
     assert f(16, 257, None, None, None, 0, None) == 2   # more heads than supported
     assert f(16, 8, None, None, None, 0, None) == 1     # null pointers
+
+
+def test_gate_vanilla_and_bwd_ex_host_validation(lib):
+    """Invalid arguments are refused on the host, before any device query."""
+    m = _mask()
+    a16 = 256  # stand-in 16-byte-aligned device addresses: never dereferenced here
+    gv = lib.sinkattn_gate_vanilla
+    assert gv(0, 128, 4, 2, 96, 0.1, a16, a16, a16, ctypes.byref(m), a16, None) == 1  # D
+    assert gv(1, 128, 4, 2, 64, 0.1, a16, a16, a16, ctypes.byref(m), a16, None) == 1  # fp16
+    assert gv(0, 128, 4, 2, 64, 0.1, None, a16, a16, ctypes.byref(m), a16, None) == 1  # q
+    assert gv(0, 128, 4, 2, 64, 0.1, a16, a16, a16, ctypes.byref(m), None, None) == 1  # gate
+    assert gv(0, 128, 4, 2, 64, 0.1, a16 + 8, a16, a16, ctypes.byref(m), a16, None) == 1
+    assert gv(0, 128, 3, 2, 64, 0.1, a16, a16, a16, ctypes.byref(m), a16, None) == 1  # Hq % Hkv
+    bad = _mask(causal=0, window=8)                                                # window needs causal
+    assert gv(0, 128, 4, 2, 64, 0.1, a16, a16, a16, ctypes.byref(bad), a16, None) == 1
+    bx = lib.sinkattn_bwd_ex
+    args = [a16] * 5 + [a16, None, None]  # q k v out dout lse d_sink_s learnable_sink
+    tail = [a16, 1 << 20, a16, a16, a16, None, a16, 1 << 20, None]
+    assert bx(0, 128, 4, 2, 96, 0.1, *args, ctypes.byref(m), *tail) == 1   # D
+    assert bx(0, 128, 4, 2, 64, 0.1, None, *args[1:], ctypes.byref(m), *tail) == 1  # q
