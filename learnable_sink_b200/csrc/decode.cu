@@ -6,9 +6,11 @@
 // window has wrapped every slot is valid.  No positional encoding is applied
 // here, so the ring head's position does not matter.
 //
-// Stage 1 (one CTA per (split, KV head, sequence)): stream the split's K and
-// V rows once with 16-byte coalesced loads; the G = Hq/Hkv query heads of the
-// KV head share every loaded row.  Each CTA writes (m, l, acc[D]) per head.
+// Stage 1 streams each (sequence, KV head, split)'s K and V rows once; the
+// G = Hq/Hkv query heads of the KV head share every loaded row, and each split
+// writes (m, l, acc[D]) per query head.  bf16 runs the warp-streaming kernel
+// below (TMA rings, warp-level MMAs); fp32 runs one CTA per split with 16-byte
+// coalesced loads on the CUDA cores.
 // Stage 2: merge the splits with the sink column (page "Attention Sink,
 // Learnable Sink and dsink", section 4: e^{a_h} joins the denominator, the
 // sink value is zero) and write O, LSE_new and sink_s.
