@@ -634,3 +634,19 @@ def test_sampled_backward_equals_full_backward(mname):
     np.testing.assert_allclose(sq, dq[rows[:, 0], rows[:, 1]], atol=1e-13)
     np.testing.assert_allclose(sk, dk[keys[:, 0], keys[:, 1]], atol=1e-13)
     np.testing.assert_allclose(sv, dv[keys[:, 0], keys[:, 1]], atol=1e-13)
+
+
+@pytest.mark.parametrize("mname", ["varlen_band", "block_sparse"])
+def test_forward_rows_equal_full_forward_rows(mname):
+    """fwd_rows (the row-sampled forward used on full-size inputs) returns
+    exactly the full forward's values at the sampled (token, head) rows."""
+    T, Hq, Hkv, D = 37, 4, 2, 16
+    mask = MASKS[mname] if mname != "block_sparse" else _block_sparse_mask()
+    q, k, v, a, _ = _random_problem(T, Hq, Hkv, D, seed=41)
+    out, lse, ss = oracle.fwd(q, k, v, a, 0.3, **mask)
+    rng = np.random.default_rng(42)
+    rows = np.stack([rng.integers(0, T, 25), rng.integers(0, Hq, 25)], 1).astype(np.int32)
+    ro, rl, rs = oracle.fwd_rows(q, k, v, a, 0.3, rows, **mask)
+    np.testing.assert_array_equal(ro, out[rows[:, 0], rows[:, 1]])
+    np.testing.assert_array_equal(rl, lse[rows[:, 0], rows[:, 1]])
+    np.testing.assert_array_equal(rs, ss[rows[:, 0], rows[:, 1]])
