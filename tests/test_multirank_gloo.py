@@ -52,7 +52,7 @@ def _worker(rank, world, port, out):
 
 def test_dsink_allreduce_over_two_gloo_ranks_equals_full_batch():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     lens, x, a = _batch()
@@ -96,7 +96,7 @@ def _gate_worker(rank, world, port, out):
 
 def test_gate_statistics_and_gradient_over_two_gloo_ranks_equal_full_batch():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_gate_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     lens, x, a = _batch()
