@@ -1,0 +1,34 @@
+"""The C ABI from plain C: tests/c/abi_host.c is compiled with gcc against
+include/sinkattn.h, linked with libsinkattn.so and run (host-only entry
+points; no device is touched)."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+from learnable_sink_b200 import sinkattn as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not installed")
+def test_plain_c_program_uses_the_abi(tmp_path):
+    if not os.path.exists(S.LIB_PATH):
+        import learnable_sink_b200.build as B
+        B.build()
+    libdir = os.path.dirname(S.LIB_PATH)
+    exe = str(tmp_path / "abi_host")
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Werror",
+                           "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c", "abi_host.c"),
+                           "-L", libdir, "-lsinkattn", "-Wl,-rpath," + libdir, "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    kv = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    assert int(kv["version"]) >= 100
+    assert kv["ok"] == '"ok"'
+    assert int(kv["plan_bytes"]) > 0 and int(kv["plan_bytes_bad_heads"]) == 0
+    assert int(kv["bwd_ws"]) > 0
+    assert int(kv["decode_ws"]) >= 32 * 32 * 4 * 130 * 4
+    assert int(kv["imp_ws"]) == 4 * 32 * 8
+    assert int(kv["fwd_bad_d"]) == 1 and int(kv["gate_bad_t"]) == 1
