@@ -39,8 +39,9 @@ class CMask(_c.Structure):
 
 
 class SinkAttnError(RuntimeError):
-    def __init__(self, fn, code):
-        super().__init__(f"{fn} failed: {ERR_NAMES.get(code, code)} ({error_string(code)})")
+    def __init__(self, fn, code, detail=None):
+        msg = f"{fn} failed: {ERR_NAMES.get(code, code)} ({error_string(code)})"
+        super().__init__(msg if detail is None else f"{msg}: {detail}")
         self.code = code
 
 
@@ -175,6 +176,49 @@ class Plan:
         return self.buf.numel()
 
 
+def _want(fn, ok, detail):
+    """Metadata the C ABI cannot see through raw pointers (element types and
+    extents); a mismatch would make a kernel read or write outside a buffer,
+    so it is refused here as SINKATTN_ERR_INVALID_ARG before any launch."""
+    if not ok:
+        raise SinkAttnError(fn, 1, detail)
+
+
+def _same_type(fn, ref, **ts):
+    for name, t in ts.items():
+        if t is not None:
+            _want(fn, t.dtype == ref.dtype, f"{name} is {t.dtype}, expected {ref.dtype}")
+
+
+def _shape(fn, name, t, shape, dtype=None):
+    if t is None:
+        return
+    _want(fn, tuple(t.shape) == tuple(shape),
+          f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None:
+        _want(fn, t.dtype == dtype, f"{name} is {t.dtype}, expected {dtype}")
+
+
+def _attn_meta(fn, q, k, v, mask):
+    _want(fn, q.dim() == 3 and k.dim() == 3 and v.dim() == 3, "q, k, v must be [T, H, D]")
+    _same_type(fn, q, k=k, v=v)
+    _want(fn, tuple(k.shape) == tuple(v.shape), "k and v shapes differ")
+    _want(fn, q.shape[0] == k.shape[0] and q.shape[2] == k.shape[2],
+          f"q {tuple(q.shape)} and k {tuple(k.shape)} disagree on T or D")
+    _want(fn, mask.cu_seqlens.dtype == torch.int32, "cu_seqlens must be int32")
+    if mask.block_indices is not None:
+        _want(fn, mask.block_indices.dtype == torch.int32, "block_indices must be int32")
+
+
+def _ring_meta(fn, k_cache, v_cache, ref, B, D, n_sink, window):
+    _same_type(fn, ref, k_cache=k_cache, v_cache=v_cache)
+    _want(fn, tuple(k_cache.shape) == tuple(v_cache.shape), "k_cache and v_cache shapes differ")
+    S_ = int(n_sink) + int(window)
+    _want(fn, k_cache.shape[0] == B and k_cache.shape[1] == S_ and k_cache.shape[3] == D,
+          f"caches have shape {tuple(k_cache.shape)}, expected [{B}, n_sink + window = {S_}, "
+          f"Hkv, {D}]")
+
+
 def _contig(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -186,8 +230,13 @@ def fwd(q, k, v, sink, mask: Mask, plan: Plan, scale: Optional[float] = None, st
     """Forward.  Returns (out [T,Hq,D], lse_new [T,Hq] fp32, sink_s [T,Hq] fp32).
     With ``lse_orig`` (fp32 [T,Hq]) also writes the LSE over the visible keys
     alone, before the sink joins (sinkattn_fwd_ex)."""
-    _contig(q, k, v, sink)
+    _attn_meta("sinkattn_fwd", q, k, v, mask)
     T, Hq, D = q.shape
+    _shape("sinkattn_fwd", "learnable_sink", sink, (Hq,), torch.float32)
+    _shape("sinkattn_fwd", "out", out, q.shape, q.dtype)
+    for name, t in (("lse", lse), ("sink_s", sink_s), ("lse_orig", lse_orig)):
+        _shape("sinkattn_fwd", name, t, (T, Hq), torch.float32)
+    _contig(q, k, v, sink)
     Hkv = k.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     out = torch.empty_like(q) if out is None else out
@@ -217,8 +266,18 @@ def bwd(q, k, v, out, dout, lse, sink, mask: Mask, plan: Plan, scale: Optional[f
         stream=None, workspace=None, dq=None, dk=None, dv=None, dsink=None, d_sink_s=None):
     """Backward.  Returns (dq, dk, dv, dsink or None).  ``d_sink_s`` [T, Hq]
     float32 is an optional upstream gradient of the gate sink_s."""
-    _contig(q, k, v, out, dout, lse, sink, d_sink_s)
+    _attn_meta("sinkattn_bwd", q, k, v, mask)
     T, Hq, D = q.shape
+    _same_type("sinkattn_bwd", q, out=out, dout=dout, dq=dq, dk=dk, dv=dv)
+    for name, t in (("out", out), ("dout", dout), ("dq", dq)):
+        _shape("sinkattn_bwd", name, t, q.shape)
+    for name, t in (("dk", dk), ("dv", dv)):
+        _shape("sinkattn_bwd", name, t, k.shape)
+    for name, t in (("lse", lse), ("d_sink_s", d_sink_s)):
+        _shape("sinkattn_bwd", name, t, (T, Hq), torch.float32)
+    for name, t in (("learnable_sink", sink), ("dsink", dsink)):
+        _shape("sinkattn_bwd", name, t, (Hq,), torch.float32)
+    _contig(q, k, v, out, dout, lse, sink, d_sink_s)
     Hkv = k.shape[1]
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     cm = mask.c()
@@ -239,8 +298,11 @@ def bwd(q, k, v, out, dout, lse, sink, mask: Mask, plan: Plan, scale: Optional[f
 
 def gate_importance(sink_s, stream=None, workspace=None, imp=None):
     """Per-head mean gate Imp [Hq] of sink_s [T, Hq] float32."""
-    _contig(sink_s)
+    _want("sinkattn_gate_importance", sink_s.dim() == 2 and sink_s.dtype == torch.float32,
+          "sink_s must be float32 [T, Hq]")
     T, Hq = sink_s.shape
+    _shape("sinkattn_gate_importance", "imp", imp, (Hq,), torch.float32)
+    _contig(sink_s)
     nws = int(lib().sinkattn_gate_importance_workspace_bytes(T, Hq))
     if workspace is None:
         workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=sink_s.device)
@@ -253,8 +315,11 @@ def gate_importance(sink_s, stream=None, workspace=None, imp=None):
 def gate_vanilla(q, k, lse, mask: Mask, scale: Optional[float] = None, stream=None, gate=None):
     """Gate sigma(LSE_not0 - q.k_0 scale) [T, Hq] of a sink-free model whose
     sink is each sequence's first token; ``lse`` is the sink-free LSE."""
-    _contig(q, k, lse, gate)
+    _attn_meta("sinkattn_gate_vanilla", q, k, k, mask)
     T, Hq, D = q.shape
+    for name, t in (("lse", lse), ("gate", gate)):
+        _shape("sinkattn_gate_vanilla", name, t, (T, Hq), torch.float32)
+    _contig(q, k, lse, gate)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     cm = mask.c()
     gate = torch.empty(T, Hq, dtype=torch.float32, device=q.device) if gate is None else gate
@@ -276,8 +341,16 @@ def decode(q, k_cache, v_cache, cache_seqlens, n_sink: int, window: int, sink,
            scale: Optional[float] = None, num_splits: int = 0, stream=None, workspace=None,
            out=None, lse=None, sink_s=None):
     """Ring-buffer decode.  Returns (out [B,Hq,D], lse_new [B,Hq], sink_s [B,Hq])."""
-    _contig(q, k_cache, v_cache, cache_seqlens, sink)
+    fn = "sinkattn_decode"
+    _want(fn, q.dim() == 3 and k_cache.dim() == 4, "q must be [B, Hq, D], caches [B, S, Hkv, D]")
     B, Hq, D = q.shape
+    _ring_meta(fn, k_cache, v_cache, q, B, D, n_sink, window)
+    _shape(fn, "cache_seqlens", cache_seqlens, (B,), torch.int32)
+    _shape(fn, "learnable_sink", sink, (Hq,), torch.float32)
+    _shape(fn, "out", out, q.shape, q.dtype)
+    for name, t in (("lse", lse), ("sink_s", sink_s)):
+        _shape(fn, name, t, (B, Hq), torch.float32)
+    _contig(q, k_cache, v_cache, cache_seqlens, sink)
     Hkv = k_cache.shape[2]
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     if num_splits <= 0:
@@ -299,8 +372,14 @@ def cache_append(k_new, v_new, cache_seqlens, k_cache, v_cache, n_sink: int, win
                  stream=None) -> None:
     """Write one new token per sequence (k_new/v_new [B, Hkv, D]) into its ring
     slot; cache_seqlens [B] int32 already counts the new token."""
-    _contig(k_new, v_new, cache_seqlens, k_cache, v_cache)
+    fn = "sinkattn_cache_append"
+    _want(fn, k_new.dim() == 3 and k_cache.dim() == 4, "k_new must be [B, Hkv, D]")
     B, Hkv, D = k_new.shape
+    _shape(fn, "v_new", v_new, k_new.shape, k_new.dtype)
+    _ring_meta(fn, k_cache, v_cache, k_new, B, D, n_sink, window)
+    _want(fn, k_cache.shape[2] == Hkv, "k_new and the caches disagree on Hkv")
+    _shape(fn, "cache_seqlens", cache_seqlens, (B,), torch.int32)
+    _contig(k_new, v_new, cache_seqlens, k_cache, v_cache)
     _check("sinkattn_cache_append", lib().sinkattn_cache_append(
         _dt(k_new), B, Hkv, D, int(n_sink), int(window), _ptr(k_new), _ptr(v_new),
         _ptr(cache_seqlens), _ptr(k_cache), _ptr(v_cache), _stream(stream)))
@@ -310,8 +389,17 @@ def cache_fill(k, v, cu_seqlens, k_cache, v_cache, n_sink: int, window: int,
                cache_seqlens_out=None, stream=None) -> None:
     """Write a packed prefill (k/v [T_tot, Hkv, D], sequences by cu_seqlens)
     into the ring caches [n_seq, S, Hkv, D]; optionally store the lengths."""
-    _contig(k, v, cu_seqlens, k_cache, v_cache, cache_seqlens_out)
+    fn = "sinkattn_cache_fill"
+    _want(fn, k.dim() == 3 and k_cache.dim() == 4 and cu_seqlens.dim() == 1,
+          "k must be [T, Hkv, D], caches [n_seq, S, Hkv, D], cu_seqlens [n_seq + 1]")
     T, Hkv, D = k.shape
+    n_seq = cu_seqlens.numel() - 1
+    _shape(fn, "v", v, k.shape, k.dtype)
+    _want(fn, cu_seqlens.dtype == torch.int32, "cu_seqlens must be int32")
+    _ring_meta(fn, k_cache, v_cache, k, n_seq, D, n_sink, window)
+    _want(fn, k_cache.shape[2] == Hkv, "k and the caches disagree on Hkv")
+    _shape(fn, "cache_seqlens_out", cache_seqlens_out, (n_seq,), torch.int32)
+    _contig(k, v, cu_seqlens, k_cache, v_cache, cache_seqlens_out)
     n_seq = cu_seqlens.numel() - 1
     _check("sinkattn_cache_fill", lib().sinkattn_cache_fill(
         _dt(k), n_seq, T, Hkv, D, int(n_sink), int(window), _ptr(cu_seqlens), _ptr(k), _ptr(v),
