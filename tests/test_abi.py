@@ -107,3 +107,15 @@ def test_gate_vanilla_and_bwd_ex_host_validation(lib):
     tail = [a16, 1 << 20, a16, a16, a16, None, a16, 1 << 20, None]
     assert bx(0, 128, 4, 2, 96, 0.1, *args, ctypes.byref(m), *tail) == 1   # D
     assert bx(0, 128, 4, 2, 64, 0.1, None, *args[1:], ctypes.byref(m), *tail) == 1  # q
+
+
+def test_decode_split_heuristic(lib):
+    """About three (sequence, KV head, split) items per streaming warp (8 warps
+    on each of 148 SMs when no device is visible), no split under 16 slots,
+    at most 128 splits."""
+    f = lib.sinkattn_decode_num_splits
+    assert f(32, 32, 8, 128, 4, 1020) == 14                # ceil(148*8*3 / 256)
+    assert f(1, 32, 8, 128, 4, 1020) == 64                 # capped by 1024 slots / 16
+    assert f(1, 8, 1, 128, 4, 100000) == 128               # capped at 128 splits
+    assert f(4096, 64, 8, 128, 4, 1020) == 1               # enough items without splitting
+    assert f(0, 8, 1, 128, 4, 100) == 1                    # degenerate sizes
