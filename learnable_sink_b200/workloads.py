@@ -276,3 +276,22 @@ def gate_inputs(T_tot: int, Hq: int, seed: int):
     vals = torch.rand(T_tot, Hq, generator=gen, dtype=torch.float32)
     grads = torch.randn(T_tot, Hq, generator=gen, dtype=torch.float32)
     return vals, grads
+
+
+def fp8_window_cache(d: DecodeInputs, seed: int):
+    """A mixed-precision copy of a decode input's cache: the n_sink sink slots
+    as they are, the window slots as FP8 E4M3 codes (uint8) of the values
+    divided by a per-KV-head scale (float32 [Hkv], drawn so that the scaled
+    values use the format's range).  Returns (k_sink, v_sink, k_codes, v_codes,
+    k_scale, v_scale)."""
+    gen = _gen(seed)
+    Hkv = d.k_cache.shape[2]
+    k_scale = (torch.rand(Hkv, generator=gen) * 0.05 + 0.02).float()
+    v_scale = (torch.rand(Hkv, generator=gen) * 0.05 + 0.02).float()
+    ns = d.n_sink
+
+    def codes(x, sc):
+        return (x[:, ns:].float() / sc[None, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+
+    return (d.k_cache[:, :ns].clone(), d.v_cache[:, :ns].clone(), codes(d.k_cache, k_scale),
+            codes(d.v_cache, v_scale), k_scale, v_scale)

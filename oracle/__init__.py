@@ -262,6 +262,45 @@ def decode(q, k_cache, v_cache, cache_seqlens, n_sink, window, sink, scale):
     return out, lse, ss
 
 
+def fp8_e4m3_value(codes):
+    """Value of each FP8 E4M3 code (the OCP 8-bit format without infinities):
+    sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+    is subnormal (m / 8 * 2^-6); S.1111.111 is NaN.  uint8 codes -> float64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
+def decode_fp8_window(q, k_sink, v_sink, k_win, v_win, k_scale, v_scale, cache_seqlens,
+                      n_sink, window, sink, scale):
+    """Ring-buffer decode with a mixed-precision cache (page "Attention Sink /
+    StreamingLLM", on KV-cache quantisation: the first tokens carry much of
+    the attention weight, so they stay in high precision and the rest are
+    stored low).  k_sink/v_sink [B, n_sink, Hkv, D] hold the sink slots as
+    they are; k_win/v_win [B, window, Hkv, D] hold the window slots as FP8
+    E4M3 codes whose value is multiplied by a per-KV-head scale
+    (k_scale/v_scale [Hkv]).  The cache is dequantised and the float64 decode
+    above runs on it.  Returns (out, lse_new, sink_s)."""
+    k_scale, v_scale = _f64(k_scale), _f64(v_scale)
+    kw = fp8_e4m3_value(_u8arr(k_win)) * k_scale[None, None, :, None]
+    vw = fp8_e4m3_value(_u8arr(v_win)) * v_scale[None, None, :, None]
+    k = np.concatenate([_f64(k_sink), kw], axis=1)
+    v = np.concatenate([_f64(v_sink), vw], axis=1)
+    return decode(q, k, v, cache_seqlens, n_sink, window, sink, scale)
+
+
+def _u8arr(x):
+    """uint8 codes from a numpy array or a torch tensor of any 1-byte type."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().cpu().contiguous().view(torch.uint8).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.uint8))
+
+
 def visible_dense(T_tot, Hq, Hkv, g, **mask):
     """Dense visibility matrix [T, T] (uint8) of KV head g."""
     pr = _Problem(T_tot, Hq, Hkv, 1, 1.0, **mask)

@@ -650,3 +650,49 @@ def test_forward_rows_equal_full_forward_rows(mname):
     np.testing.assert_array_equal(ro, out[rows[:, 0], rows[:, 1]])
     np.testing.assert_array_equal(rl, lse[rows[:, 0], rows[:, 1]])
     np.testing.assert_array_equal(rs, ss[rows[:, 0], rows[:, 1]])
+
+
+# ------------------------------------------- mixed-precision (FP8 window) decode
+
+def test_fp8_e4m3_values_match_the_library_conversion():
+    """Every one of the 256 codes against torch's float8_e4m3fn conversion."""
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    got = oracle.fp8_e4m3_value(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    np.testing.assert_array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+
+
+def test_fp8_e4m3_closed_forms():
+    v = oracle.fp8_e4m3_value(np.array([0x38, 0x7E, 0x01, 0x08, 0xB8, 0x00, 0x80, 0x7F, 0xFF],
+                                        dtype=np.uint8))
+    np.testing.assert_array_equal(v[:7], [1.0, 448.0, 2.0 ** -9, 2.0 ** -6, -1.0, 0.0, -0.0])
+    assert np.isnan(v[7]) and np.isnan(v[8])
+
+
+def test_fp8_window_decode_is_the_decode_of_the_dequantised_cache():
+    """The sink slots stay as given and the window slots are code value x
+    per-KV-head scale: equal to the plain decode on that cache, and doubling
+    one head's scale equals doubling that head's window rows."""
+    d = W.decode(B=3, n_sink=4, window=28, Hq=8, Hkv=2, D=16, seqlen_range=(0, 90))
+    d.cache_seqlens = torch.tensor([2, 17, 90], dtype=torch.int32)
+    ks, vs, kc, vc, ksc, vsc = W.fp8_window_cache(d, 7)
+    got = oracle.decode_fp8_window(d.q, ks, vs, kc, vc, ksc, vsc, d.cache_seqlens, d.n_sink,
+                                   d.window, d.sink, d.scale)
+    kw = torch.from_numpy(kc.numpy()).view(torch.float8_e4m3fn).double() * ksc.double()[None, None, :, None]
+    vw = torch.from_numpy(vc.numpy()).view(torch.float8_e4m3fn).double() * vsc.double()[None, None, :, None]
+    k = torch.cat([ks.double(), kw], 1)
+    v = torch.cat([vs.double(), vw], 1)
+    ref = oracle.decode(d.q, k, v, d.cache_seqlens, d.n_sink, d.window, d.sink, d.scale)
+    for a, b in zip(got, ref):
+        np.testing.assert_array_equal(a, b)
+    ksc2 = ksc.clone()
+    ksc2[1] *= 2
+    got2 = oracle.decode_fp8_window(d.q, ks, vs, kc, vc, ksc2, vsc, d.cache_seqlens, d.n_sink,
+                                    d.window, d.sink, d.scale)
+    k2 = k.clone()
+    k2[:, d.n_sink:, 1] *= 2
+    ref2 = oracle.decode(d.q, k2, v, d.cache_seqlens, d.n_sink, d.window, d.sink, d.scale)
+    for a, b in zip(got2, ref2):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-15)
+    assert not np.allclose(got2[0], got[0])
