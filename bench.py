@@ -41,6 +41,10 @@ from learnable_sink_b200 import workloads as W  # noqa: E402
 
 METRIC = "sink-attn fwd+bwd TFLOP/s & decode KV GB/s on 1 B200, % of roofline"
 L2_BYTES = 126 * 1024 * 1024
+# launches of this library per step: plan 12, forward 1, backward 6
+# (preprocess, dsink reduce, split-tile zero/finish, tensor-core kernel, dQ
+# convert), decode 2
+GPU_LAUNCHES_PER_STEP = 12 + 1 + 6 + 2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -57,14 +61,15 @@ def file_hash(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def load_traffic(kernel):
-    """ncu-measured DRAM bytes per launch (profiles/traffic.json), valid only
-    while the kernel's source is unchanged since the capture."""
+def load_traffic(kernel, workload):
+    """ncu-measured DRAM bytes per launch (profiles/traffic.json, keyed
+    "kernel/workload"), valid only while the kernel's source is unchanged
+    since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        t = json.load(f).get(kernel)
+        t = json.load(f).get(f"{kernel}/{workload}")
     if not t:
         return None
     src = os.path.join(ROOT, t["source"])
@@ -74,68 +79,112 @@ def load_traffic(kernel):
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU
+    every 10 ms while running, through read-only NVML queries (nvidia-smi
+    polling as a fallback).  Settings are only read, never changed."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index, self.proc, self.lines = index, None, []
+    def __init__(self, device_index, period_s=0.01):
+        self.index, self.period = device_index, period_s
+        self.sm, self.mx, self.reasons = [], None, set()
+        self.proc = self.thread = None
+        self.stop = threading.Event()
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            bus = torch.cuda.get_device_properties(self.index).pci_bus_id
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode()
+                                                                  if isinstance(bus, str) else bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _nvml_loop(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                bits = int(get_reasons(h))
+                for b, n in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            self.stop.wait(self.period)
+
+    def _smi_read(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.proc.stdout:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                self.sm.append(float(parts[0]))
+                self.mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    self.reasons.add(n)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self.mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.source = "nvml"
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.SMI_FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.thread = threading.Thread(target=self._smi_read, daemon=True)
+                self.source = "nvidia-smi"
+            except OSError:
+                return self
+        self.thread.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = sorted(self.sm)
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": self.mx,
+                "sm_min_mhz": sm[0] if sm else None, "reasons": sorted(self.reasons),
+                "samples": len(sm), "source": self.source}
 
 
-def init_dist():
+def init_dist(backend="nccl"):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                             **kw)
     return world, rank, local
 
 
@@ -238,10 +287,29 @@ def measure_config(S, inp, dev, steps=10, warmup=3):
         return sum(x.elapsed_time(y) for x, y in zip(ev[a], ev[b])) / steps
 
     step_ms, f_ms, b_ms = mean("s0", "s1"), mean("f0", "f1"), mean("b0", "b1")
-    return {"workload": inp.name, "visible_pairs": pairs,
+    return {"workload": inp.name, "visible_pairs": pairs, "D": D,
             "plan_fwd_bwd_ms": step_ms, "tflops": 14 * D * pairs / (step_ms * 1e-3) / 1e12,
             "fwd_kernel_ms": f_ms, "fwd_kernel_tflops": 4 * D * pairs / (f_ms * 1e-3) / 1e12,
             "bwd_kernel_ms": b_ms, "bwd_kernel_tflops": 10 * D * pairs / (b_ms * 1e-3) / 1e12}
+
+
+def measure_decode_kernel(S, decode_step, flush, flush_rd, reps=20):
+    """Median CUDA-event time of the decode's streaming kernel, L2 flushed
+    before each call."""
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        flush_rd.sum()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e1.record()
+        S.set_kernel_events(S.KERNEL_DECODE, e0, e1)
+        decode_step()
+        S.set_kernel_events(S.KERNEL_DECODE, None, None)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return sorted(ts)[len(ts) // 2]
 
 
 def measure_gates(S, q, k, lse, sink_s, mask, scale, flush, flush_rd, hbm_gbs, reps=10):
@@ -355,17 +423,18 @@ def run_ours(args, world, rank, local):
 
     K = args.steps
     evs = {n: [ev() for _ in range(K)] for n in
-           ("p0", "p1", "d0", "d1", "kf0", "kf1", "kb0", "kb1", "kd0", "kd1")}
+           ("p0", "p1", "d0", "d1", "kf0", "kf1", "kb0", "kb1")}
+    host_t = [0.0, 0.0]
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        host_t[0] = time.perf_counter()
         r0 = ev()
         for i in range(K):
             S.set_kernel_events(S.KERNEL_FWD, evs["kf0"][i], evs["kf1"][i])
             S.set_kernel_events(S.KERNEL_BWD, evs["kb0"][i], evs["kb1"][i])
-            S.set_kernel_events(S.KERNEL_DECODE, evs["kd0"][i], evs["kd1"][i])
             evs["p0"][i].record()
             prefill_step()
             evs["p1"][i].record()
@@ -379,8 +448,9 @@ def run_ours(args, world, rank, local):
             decode_step()
             evs["d1"][i].record()
         r1 = ev()
+        host_t[1] = time.perf_counter()
         torch.cuda.synchronize()
-    for w in (S.KERNEL_FWD, S.KERNEL_BWD, S.KERNEL_DECODE):
+    for w in (S.KERNEL_FWD, S.KERNEL_BWD):
         S.set_kernel_events(w, None, None)
     if world > 1:
         torch.distributed.barrier()
@@ -397,7 +467,9 @@ def run_ours(args, world, rank, local):
     decode_ms = max_over_ranks(total("d0", "d1"), world)
     kf_ms = total("kf0", "kf1") / K
     kb_ms = total("kb0", "kb1") / K
-    kd_ms = total("kd0", "kd1") / K
+    # the streaming kernel alone (its own events; the step loop above times
+    # whole decode calls without events between their launches)
+    kd_ms = measure_decode_kernel(S, decode_step, flush, flush_rd)
     value = world * K * (flop_fwd + flop_bwd) / (prefill_ms * 1e-3) / 1e12
     dec_gbs = world * K * dec_bytes / (decode_ms * 1e-3) / 1e9
 
@@ -458,12 +530,50 @@ def run_ours(args, world, rank, local):
     gates = measure_gates(S, q, k, lse, sink_s, mask, inp.scale, flush, flush_rd,
                           peaks["hbm_gbs"])
     clocks = clk.summary()
-    peak_tf = peaks["bf16_tflops_sustained"]
-    bwd_ach = flop_bwd / (kb_ms * 1e-3) / 1e12
-    fwd_ach = flop_fwd / (kf_ms * 1e-3) / 1e12
+    burst, sustained, hbm = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"], peaks["hbm_gbs"]
+    # The timed region lasts well under the seconds-long loop the sustained
+    # figure was taken over; the clock sampled during it says which applies.
+    at_max = (clocks["sm_mhz"] is not None and clocks["sm_max_mhz"] is not None
+              and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"])
+    region_s = region_ms * 1e-3
+    tensor_peak = burst if (at_max or region_s < 2.0) else sustained
+    tensor_peak_name = "bf16_tflops (burst)" if tensor_peak == burst else "bf16_tflops_sustained"
     dec_kernel_bytes = 2 * valid * dHkv * dD * 2
-    dec_ach = dec_kernel_bytes / (kd_ms * 1e-3) / 1e9
-    traffic = load_traffic("bwd_tc_kernel")
+
+    def tensor_entry(kernel, workload, ms, flop):
+        ach = flop / (ms * 1e-3) / 1e12
+        return {"kernel": kernel, "workload": workload, "bound": "tensor", "achieved": ach,
+                "peak": tensor_peak, "unit": "TFLOP/s", "frac": ach / tensor_peak,
+                "frac_of_sustained": ach / sustained, "ms": ms,
+                "traffic": load_traffic(kernel, workload)}
+
+    def hbm_entry(kernel, workload, ms, nbytes):
+        ach = nbytes / (ms * 1e-3) / 1e9
+        return {"kernel": kernel, "workload": workload, "bound": "hbm", "achieved": ach,
+                "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "frac_of_8tbs": ach / 8000.0,
+                "ms": ms, "bytes": nbytes, "traffic": load_traffic(kernel, workload)}
+
+    rooflines = [
+        tensor_entry("fwd_tc_kernel", "training_prefill", kf_ms, flop_fwd),
+        tensor_entry("bwd_tc_kernel", "training_prefill", kb_ms, flop_bwd),
+        hbm_entry("decode_warp_kernel", "streamingllm_decode", kd_ms, dec_kernel_bytes),
+        hbm_entry("decode call (stream + merge)", "streamingllm_decode", decode_ms / K, dec_bytes),
+        hbm_entry("gate_vanilla_kernel", "training_prefill", gates["gate_vanilla"]["ms"],
+                  gates["gate_vanilla"]["bytes"]),
+    ]
+    extra = []
+    if args.configs:
+        for mk, wl in ((W.band, "streamingllm_band"), (W.varlen, "varlen_block_sparse")):
+            r = measure_config(S, mk(), dev)
+            r["frac"] = r["tflops"] / tensor_peak
+            extra.append(r)
+            D_ = r["D"]
+            rooflines.append(tensor_entry("fwd_tc_kernel", wl, r["fwd_kernel_ms"],
+                                          4 * D_ * r["visible_pairs"]))
+            rooflines.append(tensor_entry("bwd_tc_kernel", wl, r["bwd_kernel_ms"],
+                                          10 * D_ * r["visible_pairs"]))
+    dominant = rooflines[1]  # bwd_tc_kernel: the largest share of the prefill step
+    flush_ms = region_ms / K - prefill_ms / K - decode_ms / K
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": region_ms / K, "higher_is_better": True,
@@ -478,44 +588,89 @@ def run_ours(args, world, rank, local):
                   "the decode starts)",
         },
         "decode": {"value": dec_gbs, "unit": "GB/s", "ms_per_call": decode_ms / K,
-                   "bytes_per_call": dec_bytes, "num_splits": n_splits},
+                   "bytes_per_call": dec_bytes, "num_splits": n_splits,
+                   "frac": dec_gbs / hbm, "frac_of_8tbs": dec_gbs / 8000.0},
+        "step_breakdown_ms": {
+            "prefill": prefill_ms / K, "decode_call": decode_ms / K,
+            "l2_flush_and_gaps": flush_ms,
+            "host_issue_per_step": (host_t[1] - host_t[0]) * 1e3 / K,
+            "note": "device time per step; l2_flush_and_gaps = step - prefill - decode "
+                    "(the two flush kernels between prefill and decode, and any idle time)"},
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2,
                 "what": "pinned-host q,k,v,dO,sink -> device (step i+1's copies on a second stream "
                         "overlap step i's compute, double-buffered), plan+fwd+bwd, dsink -> host"},
-        # per step: plan 12, forward 1, backward 6 (preprocess, dsink reduce,
-        # split-tile zero/finish, tensor-core kernel, dQ convert), decode 2
-        "gpu_launches": K * (12 + 1 + 6 + 2),
-        "roofline": {"kernel": "bwd_tc_kernel (dK/dV/dQ)", "bound": "tensor",
-                     "achieved": bwd_ach, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": bwd_ach / peak_tf, "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained",
-                     "algorithmic": "10*D flop per visible pair x visible pairs per launch"},
-        "kernels": {
-            "fwd_tc_kernel": {"ms": kf_ms, "achieved_tflops": fwd_ach,
-                              "frac_of_sustained": fwd_ach / peak_tf},
-            "bwd_tc_kernel": {"ms": kb_ms, "achieved_tflops": bwd_ach,
-                              "frac_of_sustained": bwd_ach / peak_tf},
-            "decode_warp_kernel": {"ms": kd_ms, "achieved_gbs": dec_ach,
-                                    "frac_of_hbm": dec_ach / peaks["hbm_gbs"]},
-        },
+        "gpu_launches": K * GPU_LAUNCHES_PER_STEP,
+        "roofline": dict(dominant, peak_source=f"{peak_src} {tensor_peak_name}",
+                         algorithmic="10*D flop per visible (query, key, head) triple x visible "
+                                     "triples per launch"),
+        "rooflines": rooflines,
         # gate rows, timed after the main region on the prefill's tensors
         # (median of 10 calls): not part of the step
         "gates": gates,
     }
-    if args.configs:
-        extra = []
-        for mk in (W.band, W.varlen):
-            r = measure_config(S, mk(), dev)
-            r["frac_of_sustained"] = r["tflops"] / peak_tf
-            extra.append(r)
+    if extra:
         line["other_configs"] = extra
     if world == 1:
         dt, fl, desc, cores = cpu_oracle_sample(inp, 4096, 2)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "sample": desc, "seconds": dt}
     print(json.dumps(line), flush=True)
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(n: int, argv, skip_device_check: bool) -> int:
+    """``--gpus N`` without a launcher: start N processes of this script, one
+    per GPU, with the environment torch.distributed.run would give them
+    (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_ADDR/PORT on 127.0.0.1).  Only rank 0
+    prints.  Returns the first non-zero exit code of a rank, else 0."""
+    if not skip_device_check:
+        have = torch.cuda.device_count()
+        if n > have:
+            print(f"bench.py: --gpus {n} but only {have} CUDA device(s) are visible",
+                  file=sys.stderr)
+            return 2
+    port = free_port()
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n),
+                   LOCAL_WORLD_SIZE=str(n), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, os.path.abspath(__file__)] + list(argv),
+                                      env=env))
+    rc = 0
+    try:
+        for p in procs:
+            code = p.wait()
+            if code != 0 and rc == 0:
+                rc = code
+                for q in procs:  # a failed rank: stop the others (exact children only)
+                    if q.poll() is None:
+                        q.terminate()
+    finally:
+        for p in procs:
+            if p.poll() is None:
+                p.kill()
+                p.wait()
+    return rc
+
+
+def run_dry(args, world, rank):
+    """Launcher check without CUDA: every rank joins a gloo group, all-reduces
+    its rank number and meets a barrier; rank 0 prints one line."""
+    t = torch.tensor([float(rank + 1)])
+    torch.distributed.all_reduce(t)
+    torch.distributed.barrier()
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "rank_sum": float(t.item()),
+                          "master_addr": os.environ.get("MASTER_ADDR"),
+                          "local_rank": int(os.environ.get("LOCAL_RANK", "0"))}), flush=True)
 
 
 def main():
@@ -529,7 +684,20 @@ def main():
                          "(no timing, no JSON line)")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the band / varlen block-sparse measurements")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="launcher check on CPU: gloo ranks, no CUDA calls")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # the reference arm runs on the host cores: no GPU count to check
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:], args.dry_run or args.impl == "reference"))
+    if args.dry_run:
+        world, rank, _ = init_dist(backend="gloo")
+        try:
+            run_dry(args, world, rank)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+        return
     world, rank, local = init_dist() if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
     try:

@@ -268,8 +268,20 @@ int sinkattn_gate_vanilla(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, 
  *   learnable_sink float32 [Hq] or NULL.
  *   out [B, Hq, D] (type dt), lse_new / sink_s float32 [B, Hq] (sink_s may be
  *   NULL).
- *   num_splits     key splits per (sequence, KV head); 0 picks one.
- *   workspace      at least sinkattn_decode_workspace_bytes(B, Hq, D, splits).
+ *   num_splits     partial results per (sequence, KV head) that the
+ *                  workspace holds; 0 picks sinkattn_decode_num_splits.  A
+ *                  count above ceil(S / 16) or above 128 is lowered to it
+ *                  (same result).  bf16: the streaming kernel gives every warp
+ *                  an equal run of 16-row cache pieces and cuts no
+ *                  (sequence, KV head) into more than num_splits runs (1 =
+ *                  one warp per pair); fp32: num_splits equal key splits.
+ *   workspace      at least sinkattn_decode_workspace_bytes(B, Hq, D,
+ *                  num_splits) bytes, 16-byte aligned, any contents (every
+ *                  partial the merge reads is written by the same call).
+ * Launches two kernels: the streaming kernel, then the merge of the partials
+ * with the sink (a programmatic dependent launch that waits on the streaming
+ * kernel).  B * S must stay below 2^31.  After a call whose device status is
+ * SINKATTN_ERR_TIMEOUT, out, lse_new and sink_s are undefined.
  * Since no positional encoding is applied inside, the result depends only on
  * which tokens are in the cache, not on where the ring head is. */
 size_t sinkattn_decode_workspace_bytes(int B, int Hq, int D, int num_splits);
@@ -280,6 +292,44 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
                     const float *learnable_sink, void *out, float *lse_new,
                     float *sink_s, int num_splits, void *workspace,
                     size_t workspace_bytes, sinkattn_stream_t stream);
+
+/* ---- ring-buffer decode over a mixed-precision cache -------------------------
+ * Page "Attention Sink / StreamingLLM", on KV-cache quantisation: the first
+ * tokens carry much of the attention weight, so they are kept in high
+ * precision while the rest of the cache is stored low.  Here the n_sink sink
+ * slots stay bf16 and the window slots are FP8 E4M3 codes (the OCP 8-bit
+ * format: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities, S.1111.111 = NaN), each worth code value x a per-KV-head scale.
+ * Same computation and results as sinkattn_decode over the dequantised cache.
+ *   q              bf16 [B, Hq, D] (its elements must lie within the f16
+ *                  range: the window scores run on f16 tensor-core MMAs).
+ *   k_sink, v_sink bf16 [B, n_sink, Hkv, D]: slot s < n_sink of sequence b
+ *                  (may be NULL when n_sink = 0).
+ *   k_win, v_win   uint8 E4M3 codes [B, window, Hkv, D]: slot n_sink + j of
+ *                  sequence b is window row j (may be NULL when window = 0).
+ *   k_scale, v_scale  float32 [Hkv]: value = code value x scale of the row's
+ *                  KV head.
+ *   cache_seqlens, n_sink, window, learnable_sink, out (bf16), lse_new,
+ *   sink_s: as for sinkattn_decode (the same slot rule).
+ *   num_splits     partial results per (sequence, KV head) that the
+ *                  workspace holds; 0 picks sinkattn_decode_fp8_num_splits.
+ *                  A count above the pieces of one (sequence, KV head)
+ *                  (ceil(n_sink / 16) + ceil(window / 32)) or above 128 is
+ *                  lowered to it (same result).
+ *   workspace      at least sinkattn_decode_workspace_bytes(B, Hq, D,
+ *                  num_splits) bytes, any contents.
+ * D in {64, 128}, Hq / Hkv in {1, 2, 4, 8}, 16-byte aligned pointers, B and
+ * Hkv <= 65535, B * n_sink and B * window below 2^31 (else
+ * SINKATTN_ERR_INVALID_ARG / UNSUPPORTED); launch failures return
+ * SINKATTN_ERR_CUDA.  Launches the streaming kernel and the split merge. */
+int sinkattn_decode_fp8_num_splits(int B, int Hq, int Hkv, int D, int n_sink, int window);
+int sinkattn_decode_fp8(int B, int Hq, int Hkv, int D, float scale, const void *q,
+                        const void *k_sink, const void *v_sink, const void *k_win,
+                        const void *v_win, const float *k_scale, const float *v_scale,
+                        const int32_t *cache_seqlens, int n_sink, int window,
+                        const float *learnable_sink, void *out, float *lse_new, float *sink_s,
+                        int num_splits, void *workspace, size_t workspace_bytes,
+                        sinkattn_stream_t stream);
 
 /* ---- ring-cache maintenance -------------------------------------------------
  * Page "Attention Sink / StreamingLLM" (the core-idea section): the cache
@@ -324,19 +374,22 @@ int sinkattn_cache_fill(sinkattn_dtype dt, int n_seq, int T_tot, int Hkv, int D,
  * input and output buffers.  The per-split partials go to a fixed 4 MiB array
  * in the library's device image (every GPU that loads the library keeps it
  * until the process exits); nothing is allocated.
- *   - Limit: B * Hq * num_splits * (D + 2) * 4 bytes (rounded up to 256) plus
- *     256 bytes for a work counter must fit in 4 MiB.  With
- *     num_splits = 0 the automatic split count is lowered until it fits;
- *     a problem that does not fit even with one split, or an explicit
- *     num_splits that does not fit, returns SINKATTN_ERR_WORKSPACE and
- *     launches nothing.
+ *   - Limit: B * Hq * num_splits * (D + 2) * 4 bytes (rounded up to 256)
+ *     must fit in 4 MiB, num_splits counted after the same lowering
+ *     sinkattn_decode applies (to ceil(S / 16) and 128).  With num_splits = 0
+ *     the automatic count is lowered until it fits; a problem that does not
+ *     fit even with one split, or an explicit num_splits that does not fit,
+ *     returns SINKATTN_ERR_WORKSPACE and launches nothing.
  *   - The first call on each device looks up the array's device address
  *     (with that device current); make that first call before any stream
  *     capture.
  *   - Every call shares the one array and leaves its contents behind; each
  *     call writes every partial it reads, so nothing needs clearing, but calls
  *     that overlap on the GPU (different streams, or concurrent host threads)
- *     race on the array and must be serialised by the caller. */
+ *     race on the array and must be serialised by the caller.
+ *   - After a call whose device status is SINKATTN_ERR_TIMEOUT, some partials
+ *     were not written (the merge then read an earlier call's leftovers):
+ *     out, lse_new and sink_s are undefined. */
 int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scale,
                             const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *cache_seqlens, int n_sink, int window,

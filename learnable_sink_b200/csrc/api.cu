@@ -301,31 +301,27 @@ int sinkattn_gate_vanilla(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, 
   return launch_gate_vanilla(a, dt, D, mask->max_seqlen, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// the split merge handles up to this many splits
-constexpr int kMaxDecodeSplits = 128;
+namespace {
+int sm_count() {
+  int sms = 148, dev;
+  if (current_device(&dev)) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+}  // namespace
 
 int sinkattn_decode_num_splits(int B, int Hq, int Hkv, int D, int n_sink, int window) {
   (void)Hq; (void)D;
-  const int S = n_sink + window;
+  const long long S = (long long)n_sink + window;
   if (B < 1 || Hkv < 1 || S < 1) return 1;
-  int sms = 148, dev;
-  if (current_device(&dev)) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // enough (sequence, KV head, split) items for about three per warp of the
-  // streaming kernel (8 warps per SM take items from a shared counter), and
-  // no split shorter than 16 slots
-  const long long pairs = (long long)B * Hkv;
-  long long want = ((long long)sms * 8 * 3 + pairs - 1) / pairs;
-  long long max_split = (S + 15) / 16;
-  if (want > max_split) want = max_split;
-  if (want > kMaxDecodeSplits) want = kMaxDecodeSplits;
-  if (want < 1) want = 1;
-  return (int)want;
+  // the fewest partial slots per (sequence, KV head) that still let every
+  // warp of the streaming kernel (8 per SM) take an equal run of pieces
+  return decode_auto_splits(B, Hkv, (S + kDecodeRows - 1) / kDecodeRows, 8LL * sm_count());
 }
 
 size_t sinkattn_decode_workspace_bytes(int B, int Hq, int D, int num_splits) {
   if (B < 1 || Hq < 1 || num_splits < 1 || (D != 64 && D != 128)) return 0;
-  // per-split partials, then the streaming kernel's work-item counter
-  return round_up(sizeof(float) * (size_t)B * Hq * num_splits * (D + 2)) + kAlign;
+  // per-(sequence, query head) partial results: num_splits x (acc[D], m, l)
+  return round_up(sizeof(float) * (size_t)B * Hq * num_splits * (D + 2));
 }
 
 int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scale,
@@ -346,9 +342,9 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
       !aligned16(lse_new) || !aligned16(workspace) || (sink_s && !aligned16(sink_s)) ||
       (learnable_sink && !aligned16(learnable_sink)))
     return SINKATTN_ERR_INVALID_ARG;
+  if ((long long)B * (n_sink + (long long)window) > INT_MAX) return SINKATTN_ERR_INVALID_ARG;
   if (num_splits <= 0) num_splits = sinkattn_decode_num_splits(B, Hq, Hkv, D, n_sink, window);
-  if (num_splits > n_sink + window) num_splits = n_sink + window;
-  if (num_splits > kMaxDecodeSplits) num_splits = kMaxDecodeSplits;  // same result, fewer splits
+  num_splits = decode_clamp_splits(num_splits, n_sink, window);  // same result, fewer slots
   if (workspace_bytes < sinkattn_decode_workspace_bytes(B, Hq, D, num_splits))
     return SINKATTN_ERR_WORKSPACE;
   if (!device_is_sm100()) return SINKATTN_ERR_UNSUPPORTED;
@@ -371,10 +367,74 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
   p.lse = lse_new;
   p.sink_s = sink_s;
   p.part = static_cast<float*>(workspace);
-  p.counter = reinterpret_cast<int*>(static_cast<char*>(workspace) +
-                                     round_up(sizeof(float) * (size_t)B * Hq * num_splits * (D + 2)));
   p.status = status_word();
   return launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sinkattn_decode_fp8_num_splits(int B, int Hq, int Hkv, int D, int n_sink, int window) {
+  (void)Hq; (void)D;
+  if (B < 1 || Hkv < 1 || n_sink < 0 || window < 0 || n_sink + (long long)window < 1) return 1;
+  return decode_auto_splits(B, Hkv, fp8_pieces(n_sink, window), 8LL * sm_count());
+}
+
+int sinkattn_decode_fp8(int B, int Hq, int Hkv, int D, float scale, const void* q,
+                        const void* k_sink, const void* v_sink, const void* k_win,
+                        const void* v_win, const float* k_scale, const float* v_scale,
+                        const int32_t* cache_seqlens, int n_sink, int window,
+                        const float* learnable_sink, void* out, float* lse_new, float* sink_s,
+                        int num_splits, void* workspace, size_t workspace_bytes,
+                        sinkattn_stream_t stream) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128))
+    return SINKATTN_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SINKATTN_ERR_UNSUPPORTED;
+  if (n_sink < 0 || window < 0 || n_sink + (long long)window < 1) return SINKATTN_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535) return SINKATTN_ERR_INVALID_ARG;
+  if ((long long)B * n_sink > INT_MAX || (long long)B * window > INT_MAX)
+    return SINKATTN_ERR_INVALID_ARG;
+  if (!q || !cache_seqlens || !out || !lse_new || !workspace) return SINKATTN_ERR_INVALID_ARG;
+  if (n_sink > 0 && (!k_sink || !v_sink || !aligned16(k_sink) || !aligned16(v_sink)))
+    return SINKATTN_ERR_INVALID_ARG;
+  if (window > 0 && (!k_win || !v_win || !k_scale || !v_scale || !aligned16(k_win) ||
+                     !aligned16(v_win) || !aligned16(k_scale) || !aligned16(v_scale)))
+    return SINKATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse_new) || !aligned16(workspace) ||
+      (sink_s && !aligned16(sink_s)) || (learnable_sink && !aligned16(learnable_sink)))
+    return SINKATTN_ERR_INVALID_ARG;
+  if (num_splits <= 0) num_splits = sinkattn_decode_fp8_num_splits(B, Hq, Hkv, D, n_sink, window);
+  num_splits = decode_clamp_units(num_splits, fp8_pieces(n_sink, window));
+  if (workspace_bytes < sinkattn_decode_workspace_bytes(B, Hq, D, num_splits))
+    return SINKATTN_ERR_WORKSPACE;
+  if (!device_is_sm100()) return SINKATTN_ERR_UNSUPPORTED;
+  DecodeFp8Problem x{};
+  DecodeProblem& p = x.base;
+  p.dt = SINKATTN_BF16;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.n_sink = n_sink;
+  p.window = window;
+  p.num_splits = num_splits;
+  p.scale = scale;
+  p.q = q;
+  p.cache_seqlens = cache_seqlens;
+  p.sink = learnable_sink;
+  p.out = out;
+  p.lse = lse_new;
+  p.sink_s = sink_s;
+  p.part = static_cast<float*>(workspace);
+  p.status = status_word();
+  if (!p.status) return SINKATTN_ERR_CUDA;
+  x.k_sink = k_sink;
+  x.v_sink = v_sink;
+  x.k_win = k_win;
+  x.v_win = v_win;
+  // the kernel loads a KV head's scales for every segment, even without
+  // window slots (and then never uses them): keep the pointers valid
+  x.k_scale = window > 0 ? k_scale : lse_new;
+  x.v_scale = window > 0 ? v_scale : lse_new;
+  return launch_decode_fp8(x, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int sinkattn_set_kernel_events(int which, void* start, void* stop) {

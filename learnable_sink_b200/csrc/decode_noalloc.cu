@@ -14,7 +14,8 @@
 
 namespace {
 
-// Maximum scratch: B * Hq * num_splits * (D + 2) floats.  4 MiB per device.
+// Maximum scratch: B * Hq * num_splits * (D + 2) floats (rounded up to 256
+// bytes).  4 MiB per device.
 constexpr size_t kScratchFloats = size_t(1) << 20;
 static __device__ __align__(256) float g_decode_noalloc_scratch[kScratchFloats];
 
@@ -48,7 +49,6 @@ extern "C" int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv
   if (B < 1 || Hq < 1 || (D != 64 && D != 128) || n_sink < 0 || window < 0 ||
       n_sink + window < 1)
     return SINKATTN_ERR_INVALID_ARG;
-  const size_t per_split = sizeof(float) * (size_t)B * Hq * (D + 2);
   const size_t capacity = sizeof(float) * kScratchFloats;
   if (num_splits <= 0) {
     // automatic choice, reduced until the partials fit the fixed scratch
@@ -56,14 +56,17 @@ extern "C" int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv
     while (num_splits > 1 && sinkattn_decode_workspace_bytes(B, Hq, D, num_splits) > capacity)
       --num_splits;
   }
-  if (num_splits > n_sink + window) num_splits = n_sink + window;
-  if (per_split > capacity || sinkattn_decode_workspace_bytes(B, Hq, D, num_splits) > capacity)
+  // the same clamp sinkattn_decode applies, before the capacity check: an
+  // explicit count beyond it gives the same result with fewer slots
+  num_splits = sk::decode_clamp_splits(num_splits, n_sink, window);
+  if (sinkattn_decode_workspace_bytes(B, Hq, D, num_splits) > capacity)
     return SINKATTN_ERR_WORKSPACE;  // the problem needs more than the built-in scratch
   float* scratch = scratch_on_current_device();
   if (!scratch) return SINKATTN_ERR_CUDA;
-  // Every entry of the partials is written by the split kernel before the
-  // combine kernel reads it, and the decode resets its work counter itself,
-  // so nothing needs clearing between calls.
+  // The merge reads only the partial slots this call's streaming kernel
+  // writes, so nothing needs clearing between calls.  After a call whose
+  // device status is SINKATTN_ERR_TIMEOUT some slots were not written and the
+  // outputs are undefined.
   return sinkattn_decode(dt, B, Hq, Hkv, D, scale, q, k_cache, v_cache, cache_seqlens, n_sink,
                          window, learnable_sink, out, lse_new, sink_s, num_splits, scratch,
                          capacity, stream);

@@ -81,6 +81,10 @@ def lib():
         L.sinkattn_decode_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
         L.sinkattn_decode.argtypes = [_i, _i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _i, _i,
                                       _vp, _vp, _vp, _vp, _i, _vp, _sz, _vp]
+        L.sinkattn_decode_fp8_num_splits.argtypes = [_i, _i, _i, _i, _i, _i]
+        L.sinkattn_decode_fp8.argtypes = [_i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _i, _vp,
+                                          _sz, _vp]
         L.sinkattn_cache_append.argtypes = [_i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
         L.sinkattn_cache_fill.argtypes = [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp]
@@ -365,6 +369,53 @@ def decode(q, k_cache, v_cache, cache_seqlens, n_sink: int, window: int, sink,
         _dt(q), B, Hq, Hkv, D, scale, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens),
         int(n_sink), int(window), _ptr(sink), _ptr(out), _ptr(lse), _ptr(sink_s), int(num_splits),
         _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse, sink_s
+
+
+def decode_fp8_num_splits(B, Hq, Hkv, D, n_sink, window) -> int:
+    return int(lib().sinkattn_decode_fp8_num_splits(B, Hq, Hkv, D, n_sink, window))
+
+
+def decode_fp8(q, k_sink, v_sink, k_win, v_win, k_scale, v_scale, cache_seqlens, n_sink: int,
+               window: int, sink, scale: Optional[float] = None, num_splits: int = 0,
+               stream=None, workspace=None, out=None, lse=None, sink_s=None):
+    """Ring-buffer decode over a mixed-precision cache: bf16 sink slots
+    k_sink/v_sink [B, n_sink, Hkv, D], FP8 E4M3 window slots k_win/v_win
+    [B, window, Hkv, D] (uint8 codes, or torch.float8_e4m3fn) with per-KV-head
+    float32 scales k_scale/v_scale [Hkv].  Returns (out [B,Hq,D] bf16,
+    lse_new [B,Hq], sink_s [B,Hq])."""
+    fn = "sinkattn_decode_fp8"
+    _want(fn, q.dim() == 3 and q.dtype == torch.bfloat16, "q must be bfloat16 [B, Hq, D]")
+    B, Hq, D = q.shape
+    _want(fn, k_win.dim() == 4 and k_win.element_size() == 1 and v_win.element_size() == 1,
+          "k_win / v_win must be 1-byte [B, window, Hkv, D] E4M3 codes")
+    Hkv = k_win.shape[2]
+    _shape(fn, "k_win", k_win, (B, window, Hkv, D))
+    _shape(fn, "v_win", v_win, (B, window, Hkv, D))
+    for name, t in (("k_sink", k_sink), ("v_sink", v_sink)):
+        _shape(fn, name, t, (B, n_sink, Hkv, D), torch.bfloat16)
+    for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        _shape(fn, name, t, (Hkv,), torch.float32)
+    _shape(fn, "cache_seqlens", cache_seqlens, (B,), torch.int32)
+    _shape(fn, "learnable_sink", sink, (Hq,), torch.float32)
+    _shape(fn, "out", out, q.shape, q.dtype)
+    for name, t in (("lse", lse), ("sink_s", sink_s)):
+        _shape(fn, name, t, (B, Hq), torch.float32)
+    _contig(q, k_sink, v_sink, k_win, v_win, k_scale, v_scale, cache_seqlens, sink)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if num_splits <= 0:
+        num_splits = decode_fp8_num_splits(B, Hq, Hkv, D, n_sink, window)
+    nws = decode_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if lse is None else lse
+    sink_s = torch.empty(B, Hq, dtype=torch.float32, device=q.device) if sink_s is None else sink_s
+    _check(fn, lib().sinkattn_decode_fp8(
+        B, Hq, Hkv, D, scale, _ptr(q), _ptr(k_sink), _ptr(v_sink), _ptr(k_win), _ptr(v_win),
+        _ptr(k_scale), _ptr(v_scale), _ptr(cache_seqlens), int(n_sink), int(window), _ptr(sink),
+        _ptr(out), _ptr(lse), _ptr(sink_s), int(num_splits), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
     return out, lse, sink_s
 
 

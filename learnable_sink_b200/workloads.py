@@ -291,7 +291,12 @@ def fp8_window_cache(d: DecodeInputs, seed: int):
     ns = d.n_sink
 
     def codes(x, sc):
-        return (x[:, ns:].float() / sc[None, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        # torch's float8 cast does not saturate (|v| > 448 would become the
+        # NaN code), so the scaled values are clamped to the format's range
+        v = (x[:, ns:].float() / sc[None, None, :, None]).clamp(-448.0, 448.0)
+        c = v.to(torch.float8_e4m3fn).view(torch.uint8)
+        assert not bool(((c & 0x7F) == 0x7F).any()), "NaN code in the generated window cache"
+        return c
 
     return (d.k_cache[:, :ns].clone(), d.v_cache[:, :ns].clone(), codes(d.k_cache, k_scale),
             codes(d.v_cache, v_scale), k_scale, v_scale)

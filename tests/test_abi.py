@@ -110,12 +110,16 @@ def test_gate_vanilla_and_bwd_ex_host_validation(lib):
 
 
 def test_decode_split_heuristic(lib):
-    """About three (sequence, KV head, split) items per streaming warp (8 warps
-    on each of 148 SMs when no device is visible), no split under 16 slots,
-    at most 128 splits."""
+    """The fewest partial slots per (sequence, KV head) that still give each
+    streaming warp (8 on each of 148 SMs when no device is visible) an equal
+    run of 16-row pieces: runs of ppw = ceil(total pieces / warps), and a
+    pair of np pieces meets at most ceil((np - 1) / ppw) + 1 runs; never more
+    slots than pieces, never more than 128."""
     f = lib.sinkattn_decode_num_splits
-    assert f(32, 32, 8, 128, 4, 1020) == 14                # ceil(148*8*3 / 256)
-    assert f(1, 32, 8, 128, 4, 1020) == 64                 # capped by 1024 slots / 16
-    assert f(1, 8, 1, 128, 4, 100000) == 128               # capped at 128 splits
-    assert f(4096, 64, 8, 128, 4, 1020) == 1               # enough items without splitting
+    # 256 pairs x 64 pieces over 1184 warps: runs of 14 pieces
+    assert f(32, 32, 8, 128, 4, 1020) == 6                 # ceil(63 / 14) + 1
+    assert f(1, 32, 8, 128, 4, 1020) == 64                 # runs of 1 piece: one slot per piece
+    # 6251 pieces: runs of 50 keep the slots within 128
+    assert f(1, 8, 1, 128, 4, 100000) == 126               # ceil(6250 / 50) + 1
+    assert f(4096, 64, 8, 128, 4, 1020) == 2               # runs longer than a pair
     assert f(0, 8, 1, 128, 4, 100) == 1                    # degenerate sizes

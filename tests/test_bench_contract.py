@@ -38,3 +38,32 @@ def test_reference_arm_other_ranks_are_silent():
     r = _run({"WORLD_SIZE": "2", "RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_launcher_spawns_ranks_with_torchrun_environment():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself (the
+    environment torch.distributed.run would give them, rendezvous on
+    127.0.0.1); --dry-run makes them gloo ranks without CUDA calls.  Exactly
+    one line comes back, from rank 0, after an all-reduce over both ranks."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--dry-run"], cwd=ROOT,
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["dry_run"] is True and d["n_gpus"] == 2
+    assert d["rank_sum"] == 3.0  # ranks 0 and 1 each contributed rank + 1
+    assert d["master_addr"] == "127.0.0.1" and d["local_rank"] == 0
+
+
+def test_launcher_refuses_more_ranks_than_devices():
+    """Asking for more GPUs than are visible fails before any rank starts."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK")}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2
+    assert "CUDA device" in r.stderr
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]

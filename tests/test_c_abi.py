@@ -32,3 +32,17 @@ def test_plain_c_program_uses_the_abi(tmp_path):
     assert int(kv["decode_ws"]) >= 32 * 32 * 4 * 130 * 4
     assert int(kv["imp_ws"]) == 4 * 32 * 8
     assert int(kv["fwd_bad_d"]) == 1 and int(kv["gate_bad_t"]) == 1
+
+
+def test_decode_schedule_keeps_partials_inside_the_workspace(tmp_path):
+    """The streaming decode's static schedule (host code, compiled and run on
+    the CPU): over many shapes, warp runs stay within the launched warps and
+    no (sequence, KV head) pair meets more runs than its partial slots."""
+    from learnable_sink_b200 import build as B
+    exe = str(tmp_path / "decode_schedule_check")
+    subprocess.check_call([B.nvcc(), "-std=c++17", "-arch=sm_100a", "-I",
+                           os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c", "decode_schedule_check.cu"), "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout
+    assert out.stdout.startswith("ok ")
