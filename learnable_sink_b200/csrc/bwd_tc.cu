@@ -532,10 +532,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           P[32 * h2 + c] = fast_exp2(__uint_as_float(a[c]) * p.scale_log2 - lse_s[32 * h2 + c]);
       }
       if (partial) {
+        const KeySpan ks = key_span(kj, q0, it.seq_len, p.causal, p.n_sink, p.window);
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
           const int tok = (CW * cw + c) / HPT;
-          if (!visible_elem(q0 + tok, kj, it.seq_len, p.causal, p.n_sink, p.window)) P[c] = 0.f;
+          if (tok < ks.lo || tok > ks.hi) P[c] = 0.f;
         }
       }
       {

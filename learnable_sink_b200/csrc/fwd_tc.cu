@@ -37,9 +37,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-template <int D_, int TQ_, int TK_, int NQT_>
+// PAIR: the plan's key tiles are 64-key blocks and the kernel stages two of
+// them (consecutive entries of the list) as one 128-key tile, so the score MMA
+// has N = 128 (N = 64 runs at 2/3 of the tensor rate: its shared-memory
+// operand reads become the limit) and the softmax covers 128 columns per pass.
+template <int D_, int TQ_, int TK_, int NQT_, bool PAIR_ = false>
 struct FwdCfg {
   static constexpr int D = D_, TQ = TQ_, TK = TK_, NQT = NQT_;
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int PT = PAIR ? TK / 2 : TK;  // the plan's key tile
+  static_assert(!PAIR || TK == 128, "pairs of 64-key blocks");
   static constexpr int HPT = 128 / TQ;           // heads per query tile
   static constexpr int DH = D / 64;              // 64-column halves of a row
   static constexpr int Q_BYTES = 128 * D * 2;    // one query tile
@@ -49,6 +56,12 @@ struct FwdCfg {
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "not enough shared memory for a two-stage ring");
   static constexpr int MIN_BLOCKS = 1;
+  // Out of every 8 element pairs of a row, POLY8 take their exponentials on
+  // the FMA pipe (exp2_poly2) instead of the MUFU unit, whose 16 results per
+  // clock per SM would otherwise cap the tile rate: the exponentials of a
+  // 128 x 128 tile cost as many cycles as its two MMAs at D = 128, twice as
+  // many at D = 64.
+  static constexpr int POLY8 = D == 64 ? 3 : 2;
   // With two softmax warpgroups and one CTA per SM, registers are moved to the
   // softmax warpgroups: the producer and MMA warps then share a warpgroup with
   // two idle warps (setmaxnreg works on whole warpgroups), 12 warps in all,
@@ -125,7 +138,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
   const int chunk = rem % p.chunks;
   const int head0 = kvh * p.G + chunk * NQT * HPT;
   const int* ent = p.plan + hdr->off_fwd_entries + it.entry_off;
-  const int n = it.entry_len;
+  const int n = it.entry_len;                      // plan entries (key tiles)
+  const int nt = C::PAIR ? (n + 1) / 2 : n;        // staged key tiles
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -174,23 +188,32 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       int last_k[NS], last_v[NS];
       for (int s = 0; s < NS; ++s) last_k[s] = last_v[s] = -1;
       bool ok = true;
-      for (int j = 0; j < n && ok; ++j) {
+      for (int j = 0; j < nt && ok; ++j) {
         const int s = j % NS;
         const uint32_t par = ((j / NS) & 1) ^ 1;
-        const int krow = it.seq_start + (__ldg(ent + j) >> 1) * TK;
+        // a missing second block of a pair re-reads the first (its scores
+        // are masked; the values stay finite)
+        int krow[C::PAIR ? 2 : 1];
+        krow[0] = it.seq_start + (__ldg(ent + (C::PAIR ? 2 * j : j)) >> 1) * C::PT;
+        if constexpr (C::PAIR)
+          krow[1] = 2 * j + 1 < n ? it.seq_start + (__ldg(ent + 2 * j + 1) >> 1) * C::PT : krow[0];
         ok = mbar_wait(bar_ke + s, par, abort_flag, p.status);
         if (!ok) break;
         mbar_expect_tx(bar_kf + s, C::KV_BYTES);
         for (int h = 0; h < DH; ++h)
-          tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + h * (C::KV_BYTES / DH), &tmap_k,
-                      bar_kf + s, h * 64, kvh, krow);
+          for (int b2 = 0; b2 < (C::PAIR ? 2 : 1); ++b2)
+            tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + h * (C::KV_BYTES / DH) +
+                            b2 * C::PT * 128,
+                        &tmap_k, bar_kf + s, h * 64, kvh, krow[b2]);
         last_k[s] = j;
         ok = mbar_wait(bar_ve + s, par, abort_flag, p.status);
         if (!ok) break;
         mbar_expect_tx(bar_vf + s, C::KV_BYTES);
         for (int h = 0; h < DH; ++h)
-          tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + h * (C::KV_BYTES / DH), &tmap_v,
-                      bar_vf + s, h * 64, kvh, krow);
+          for (int b2 = 0; b2 < (C::PAIR ? 2 : 1); ++b2)
+            tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + h * (C::KV_BYTES / DH) +
+                            b2 * C::PT * 128,
+                        &tmap_v, bar_vf + s, h * 64, kvh, krow[b2]);
         last_v[s] = j;
       }
       if (!ok) {  // let copies already in flight land before the CTA exits
@@ -205,12 +228,19 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, TK, 0, 0);
+      constexpr uint32_t idesc_qk16 = idesc_bf16_f32(128, 16, 0, 0);
+      // staged tile j is a band's sink-only first tile: scores on its first
+      // 16 keys only, values from those 16 rows only
+      auto narrow = [&](int j) {
+        return !C::PAIR && sink_only_tile(__ldg(ent + j) >> 1, it.tile_start, TK, p.n_sink,
+                                          p.window);
+      };
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t sq = smem_u32(smem + C::OFF_Q), sk = smem_u32(smem + C::OFF_K),
                      sv = smem_u32(smem + C::OFF_V);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status);
-      for (int j = 0; j <= n && ok; ++j) {
-        if (j < n) ok = mbar_wait(bar_kf + j % NS, (j / NS) & 1, abort_flag, p.status);
+      for (int j = 0; j <= nt && ok; ++j) {
+        if (j < nt) ok = mbar_wait(bar_kf + j % NS, (j / NS) & 1, abort_flag, p.status);
         if (ok && j > 0) ok = mbar_wait(bar_vf + (j - 1) % NS, ((j - 1) / NS) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
@@ -220,30 +250,33 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
             if (!ok) break;
             tc_fence_after();
             const uint32_t vbase = sv + ((j - 1) % NS) * C::KV_BYTES;
+            const int kk_end = narrow(j - 1) ? 1 : TK / 16;
 #pragma unroll
             for (int kk = 0; kk < TK / 16; ++kk) {
+              if (kk >= kk_end) break;
               // B = V tile, MN-major: 64-column atoms TK*128 B apart, 8-row groups 1 KB apart
               const uint64_t bdesc = sdesc_sw128(vbase + kk * 16 * 128, TK * 128, 1024);
               mma_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * TK + kk * 8, bdesc, idesc_pv,
                      (j > 1 || kk > 0) ? 1u : 0u);
             }
           }
-          if (j < n) {
+          if (j < nt) {
             const uint32_t qbase = sq + t * C::Q_BYTES;
             const uint32_t kbase = sk + (j % NS) * C::KV_BYTES;
+            const uint32_t idq = narrow(j) ? idesc_qk16 : idesc_qk;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B inside the 128-B row
               const uint64_t adesc = sdesc_sw128(qbase + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024);
               const uint64_t bdesc = sdesc_sw128(kbase + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024);
-              mma_ss(tmem + C::S_COL + t * TK, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + C::S_COL + t * TK, adesc, bdesc, idq, kk > 0 ? 1u : 0u);
             }
             mma_commit(bar_s + t);
           }
         }
         if (!ok) break;
         if (j > 0) mma_commit(bar_ve + (j - 1) % NS);
-        if (j < n) mma_commit(bar_ke + j % NS);
+        if (j < nt) mma_commit(bar_ke + j % NS);
       }
       if (ok)
         for (int t = 0; t < NQT; ++t) mma_commit(bar_o + t);
@@ -265,12 +298,69 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
     const uint32_t o_addr = tmem + lane_off + C::O_COL + t * D;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int e = __ldg(ent + j);
-      const int k0 = (e >> 1) * TK;
+    for (int j = 0; j < nt; ++j) {
+      const int e = __ldg(ent + (C::PAIR ? 2 * j : j));
+      const int k0 = (e >> 1) * C::PT;
+      // second block of a pair: -1 when the list has no entry for it
+      const int e1 = C::PAIR ? (2 * j + 1 < n ? __ldg(ent + 2 * j + 1) : -1) : 0;
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s + t, j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      if (!C::PAIR && sink_only_tile(e >> 1, it.tile_start, TK, p.n_sink, p.window)) {
+        // a band's sink-only first tile: 16 score columns, keys [0, n_sink)
+        // visible (every row here is past them causally)
+        float x16[16];
+        {
+          uint32_t rr[16];
+          tmem_ld16(s_addr, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            asm volatile("" : "+r"(rr[c]));
+            x16[c] = c < p.n_sink ? __uint_as_float(rr[c]) : -INFINITY;
+          }
+        }
+        float mraw = x16[0];
+#pragma unroll
+        for (int c = 1; c < 16; c += 2) mraw = c + 1 < 16 ? fmax3(mraw, x16[c], x16[c + 1]) : fmaxf(mraw, x16[c]);
+        const float mx = mraw * p.scale_log2;
+        const bool need = mx > m + kRescaleThreshold;
+        float corr = 1.f;
+        if (need) {
+          corr = exp2f(m - mx);
+          l *= corr;
+        }
+        const bool touch_o = need && j > 0 && m != -INFINITY;
+        if (__any_sync(0xffffffffu, touch_o)) {
+          const float f = touch_o ? corr : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(o_addr + c * 32, rr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * f);
+            tmem_st32(o_addr + c * 32, rr);
+          }
+        }
+        if (need) m = mx;
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        uint32_t pk[8];
+        float rs = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p0 = fast_exp2(fmaf(x16[2 * i], p.scale_log2, -mu));
+          const float p1 = fast_exp2(fmaf(x16[2 * i + 1], p.scale_log2, -mu));
+          rs += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st8(s_addr, pk);
+        l += rs;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p + t);
+        continue;
+      }
       // raw scores x = Q.K (the scale is folded into the exponent below)
       // all TK / 32 loads in flight, one wait for them together
       float x[TK];
@@ -287,10 +377,29 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
             x[c * 32 + i] = __uint_as_float(rr[c][i]);
           }
       }
-      if (e & 1) {  // partial tile: element mask
+      // partial tiles: element mask from the row's visible span
+      if constexpr (C::PAIR) {
+        if (e & 1) {
+          const RowSpan sp = row_span(qi, k0, it.seq_len, p.causal, p.n_sink, p.window);
+#pragma unroll
+          for (int c = 0; c < C::PT; ++c)
+            if (!span_visible(sp, c)) x[c] = -INFINITY;
+        }
+        if (e1 < 0) {  // no second block
+#pragma unroll
+          for (int c = C::PT; c < TK; ++c) x[c] = -INFINITY;
+        } else if (e1 & 1) {
+          const RowSpan sp = row_span(qi, (e1 >> 1) * C::PT - C::PT, it.seq_len, p.causal,
+                                      p.n_sink, p.window);
+#pragma unroll
+          for (int c = C::PT; c < TK; ++c)
+            if (!span_visible(sp, c)) x[c] = -INFINITY;
+        }
+      } else if (e & 1) {
+        const RowSpan sp = row_span(qi, k0, it.seq_len, p.causal, p.n_sink, p.window);
 #pragma unroll
         for (int c = 0; c < TK; ++c)
-          if (!visible_elem(qi, k0 + c, it.seq_len, p.causal, p.n_sink, p.window)) x[c] = -INFINITY;
+          if (!span_visible(sp, c)) x[c] = -INFINITY;
       }
       // row max with eight independent accumulators (short dependency chains)
       float m8[8];
@@ -337,6 +446,13 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       // on element pairs (packed fp32x2 instructions), the exponentials one
       // by one
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mu, -mu);
+      // polynomial coefficients times `live` (0 for a row that has seen no
+      // key yet: its scores are all -inf and its probabilities must be 0)
+      const float live = (m == -INFINITY) ? 0.f : 1.f;
+      const float2 pc0 = make_float2(kExp2C0 * live, kExp2C0 * live);
+      const float2 pc1 = make_float2(kExp2C1 * live, kExp2C1 * live);
+      const float2 pc2 = make_float2(kExp2C2 * live, kExp2C2 * live);
+      const float2 pc3 = make_float2(kExp2C3 * live, kExp2C3 * live);
       float2 rs4[4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) rs4[a] = make_float2(0.f, 0.f);
@@ -346,7 +462,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float2 y = __ffma2_rn(make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]), sc2, nm2);
-          const float2 pp = make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          const float2 pp = (i % 8) < C::POLY8 ? exp2_poly2(y, pc0, pc1, pc2, pc3)
+                                               : make_float2(fast_exp2(y.x), fast_exp2(y.y));
           rs4[i & 3] = __fadd2_rn(rs4[i & 3], pp);
           pk[i] = pack_bf16x2(pp.x, pp.y);
         }
@@ -492,13 +609,13 @@ bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, i
 
 namespace {
 
-template <int D, int TQ, int TK, int NQT>
+template <int D, int TQ, int TK, int NQT, bool PAIR = false>
 int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
-  using C = FwdCfg<D, TQ, TK, NQT>;
+  using C = FwdCfg<D, TQ, TK, NQT, PAIR>;
   CUtensorMap mq, mk, mv;
   if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, TQ) ||
-      !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, TK) ||
-      !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, TK))
+      !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::PT) ||
+      !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::PT))
     return SINKATTN_ERR_CUDA;
   FwdParams fp{};
   fp.plan = p.plan;
@@ -549,13 +666,14 @@ int launch_fwd_tc(const AttnProblem& p, void* out, float* lse, float* sink_s, cu
     return two ? launch_cfg<64, 128, 128, 2>(p, out, lse, sink_s, stream)
                : launch_cfg<64, 128, 128, 1>(p, out, lse, sink_s, stream);
   }
-  // 64-token tiles need two heads per query tile
+  // 64-token tiles need two heads per query tile; key blocks are staged in
+  // pairs as 128-key tiles
   if (G % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;
   const bool two = (G % 4 == 0);
-  if (p.D == 128) return two ? launch_cfg<128, 64, 64, 2>(p, out, lse, sink_s, stream)
-                             : launch_cfg<128, 64, 64, 1>(p, out, lse, sink_s, stream);
-  return two ? launch_cfg<64, 64, 64, 2>(p, out, lse, sink_s, stream)
-             : launch_cfg<64, 64, 64, 1>(p, out, lse, sink_s, stream);
+  if (p.D == 128) return two ? launch_cfg<128, 64, 128, 2, true>(p, out, lse, sink_s, stream)
+                             : launch_cfg<128, 64, 128, 1, true>(p, out, lse, sink_s, stream);
+  return two ? launch_cfg<64, 64, 128, 2, true>(p, out, lse, sink_s, stream)
+             : launch_cfg<64, 64, 128, 1, true>(p, out, lse, sink_s, stream);
 }
 
 }  // namespace sk

@@ -77,6 +77,52 @@ __host__ __device__ __forceinline__ bool visible_elem(int qi, int kj, int seq_le
   return true;
 }
 
+// The visible columns c of one query row inside a tile that starts at key
+// k0 (sequence-local): c <= hi and (c >= lo or c < ns).  hi is the causal /
+// sequence-end bound, lo the window's lower bound (-1 without a window), ns
+// the end of the sink prefix (0 without a window).  Same set as visible_elem.
+struct RowSpan {
+  int lo, hi, ns;
+};
+__host__ __device__ __forceinline__ RowSpan row_span(int qi, int k0, int seq_len, int causal,
+                                                     int n_sink, int window) {
+  int last = seq_len - 1;
+  if (causal && qi < last) last = qi;
+  RowSpan s;
+  s.hi = last - k0;
+  s.lo = window > 0 ? qi - window + 1 - k0 : -1;
+  s.ns = window > 0 ? n_sink - k0 : 0;
+  return s;
+}
+__host__ __device__ __forceinline__ bool span_visible(const RowSpan& s, int c) {
+  return c <= s.hi && (c >= s.lo || c < s.ns);
+}
+
+// The query tokens t of a tile starting at q0 that see key kj: lo <= t <= hi
+// (qi >= kj when causal; past the sink prefix, qi <= kj + window - 1; a key
+// past the sequence is seen by none).  Same set as visible_elem.
+struct KeySpan {
+  int lo, hi;
+};
+__host__ __device__ __forceinline__ KeySpan key_span(int kj, int q0, int seq_len, int causal,
+                                                     int n_sink, int window) {
+  constexpr int kFar = 1 << 29;
+  KeySpan s;
+  s.lo = (causal ? kj : -kFar) - q0;
+  s.hi = kj >= seq_len ? -kFar
+       : (window > 0 && kj >= n_sink ? kj + window - 1 - q0 : kFar);
+  return s;
+}
+
+// A StreamingLLM band's first key tile, seen from a query tile whose every
+// row's window starts past that tile: only the n_sink <= 16 sink keys of it
+// are visible, so a 16-key slice of the tile carries all of its work.
+__host__ __device__ __forceinline__ bool sink_only_tile(int key_tile, int q_tile_start, int tile,
+                                                        int n_sink, int window) {
+  return key_tile == 0 && window > 0 && n_sink > 0 && n_sink <= 16 &&
+         q_tile_start - window + 1 >= tile;
+}
+
 // Tile classification from the interval bounds (no enumeration):
 // 0 = no visible pair, 1 = some, 2 = every (valid row, tile column) pair.
 // Rows are [q0, q0 + qlen); columns [k0, k0 + tile), keys past seq_len are

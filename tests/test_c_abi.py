@@ -46,3 +46,30 @@ def test_decode_schedule_keeps_partials_inside_the_workspace(tmp_path):
     out = subprocess.run([exe], capture_output=True, text=True)
     assert out.returncode == 0, out.stdout
     assert out.stdout.startswith("ok ")
+
+
+def test_mask_span_and_sink_only_tile_match_elementwise_visibility(tmp_path):
+    """The kernels' per-row mask (an interval plus the sink prefix) and the
+    band's sink-only tile rule agree with the element-wise visibility
+    predicate (host code, compiled and run on the CPU)."""
+    from learnable_sink_b200 import build as B
+    exe = str(tmp_path / "mask_span_check")
+    subprocess.check_call([B.nvcc(), "-std=c++17", "-arch=sm_100a",
+                           os.path.join(ROOT, "tests", "c", "mask_span_check.cu"), "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout
+    assert out.stdout.startswith("ok ")
+
+
+def test_fma_pipe_exp2_error_bound(tmp_path):
+    """The softmax's FMA-pipe exponential (Cody-Waite range reduction and a
+    fitted cubic) stays within 1e-4 relative error of 2^y on [-126, 8] and
+    returns exactly 0 for a row with no visible key (host evaluation of the
+    same fp32 operations)."""
+    from learnable_sink_b200 import build as B
+    exe = str(tmp_path / "exp2_poly_check")
+    subprocess.check_call([B.nvcc(), "-std=c++17", "-arch=sm_100a",
+                           os.path.join(ROOT, "tests", "c", "exp2_poly_check.cu"), "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout
+    assert out.stdout.startswith("ok ")
