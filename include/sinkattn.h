@@ -331,6 +331,24 @@ int sinkattn_decode_fp8(int B, int Hq, int Hkv, int D, float scale, const void *
                         int num_splits, void *workspace, size_t workspace_bytes,
                         sinkattn_stream_t stream);
 
+/* sinkattn_cache_append_fp8 -- one new token per sequence into the
+ * mixed-precision cache of sinkattn_decode_fp8 (same slot rule as
+ * sinkattn_cache_append).
+ *   k_new, v_new   bf16 [B, Hkv, D]: the token being appended.
+ *   cache_seqlens  device int32 [B], this token included (position
+ *                  cache_seqlens[b] - 1; entries <= 0 write nothing).
+ *   A position p < n_sink copies the token into k_sink / v_sink row p; a
+ *   later one writes window row (p - n_sink) % window of k_win / v_win as
+ *   the E4M3 codes of value / scale of the row's KV head (IEEE division in
+ *   float32, round to nearest even, magnitudes past 448 saturated to 448,
+ *   NaN stays NaN).
+ * D in {64, 128}, 16-byte aligned k_new, v_new and caches (else
+ * SINKATTN_ERR_INVALID_ARG); launch failures return SINKATTN_ERR_CUDA. */
+int sinkattn_cache_append_fp8(int B, int Hkv, int D, int n_sink, int window, const void *k_new,
+                              const void *v_new, const int32_t *cache_seqlens, void *k_sink,
+                              void *v_sink, void *k_win, void *v_win, const float *k_scale,
+                              const float *v_scale, sinkattn_stream_t stream);
+
 /* ---- ring-cache maintenance -------------------------------------------------
  * Page "Attention Sink / StreamingLLM" (the core-idea section): the cache
  * keeps a sequence's first n_sink tokens in fixed slots and its most recent

@@ -4,6 +4,8 @@
 // segment, each new token overwriting the oldest non-sink one.  Slot rule
 // (shared with the decode): position p < n_sink -> slot p, otherwise
 // n_sink + (p - n_sink) % window.  Both kernels are plain 16-byte copies.
+#include <cuda_fp8.h>
+
 #include "internal.h"
 
 namespace sk {
@@ -60,6 +62,60 @@ __global__ void cache_fill_kernel(const uint4* k, const uint4* v, const int32_t*
   }
 }
 
+// Mixed-precision cache (bf16 sink slots, FP8 E4M3 window rows with a scale
+// per KV head): one CTA per sequence, one thread per 8 elements of the
+// token's Hkv x D values.  A sink position copies its 16 bytes; a window
+// position stores the E4M3 codes of value / scale (IEEE division, round to
+// nearest even, saturating at +-448, NaN kept), 8 bytes per thread.
+__global__ void cache_append_fp8_kernel(const uint4* k_new, const uint4* v_new,
+                                        const int32_t* seqlens, uint4* k_sink, uint4* v_sink,
+                                        uint2* k_win, uint2* v_win, const float* k_scale,
+                                        const float* v_scale, int Hkv, int D, int n_sink,
+                                        int window) {
+  const int b = blockIdx.x;
+  const long long p = (long long)seqlens[b] - 1;
+  if (p < 0) return;
+  const int row8 = Hkv * D / 8;  // 8-element chunks of the token
+  if (p < n_sink) {
+    const long long dst = ((long long)b * n_sink + p) * row8, src = (long long)b * row8;
+    for (int i = threadIdx.x; i < row8; i += blockDim.x) {
+      k_sink[dst + i] = k_new[src + i];
+      v_sink[dst + i] = v_new[src + i];
+    }
+    return;
+  }
+  if (window <= 0) return;
+  const long long r = (p - n_sink) % window;
+  const long long dst = ((long long)b * window + r) * row8, src = (long long)b * row8;
+  for (int i = threadIdx.x; i < row8; i += blockDim.x) {
+    const int h = (i * 8) / D;
+    const float ks = k_scale[h], vs = v_scale[h];
+    const uint4 kk = k_new[src + i], vv = v_new[src + i];
+    const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kk);
+    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
+    uint32_t kc[2], vc[2];
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      uint32_t kb = 0, vb = 0;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float2 kf = __bfloat1622float2(k2[2 * w + u]);
+        const float2 vf = __bfloat1622float2(v2[2 * w + u]);
+        const uint32_t kq = __nv_cvt_float2_to_fp8x2(
+            make_float2(__fdiv_rn(kf.x, ks), __fdiv_rn(kf.y, ks)), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t vq = __nv_cvt_float2_to_fp8x2(
+            make_float2(__fdiv_rn(vf.x, vs), __fdiv_rn(vf.y, vs)), __NV_SATFINITE, __NV_E4M3);
+        kb |= (kq & 0xffffu) << (16 * u);
+        vb |= (vq & 0xffffu) << (16 * u);
+      }
+      kc[w] = kb;
+      vc[w] = vb;
+    }
+    k_win[dst + i] = make_uint2(kc[0], kc[1]);
+    v_win[dst + i] = make_uint2(vc[0], vc[1]);
+  }
+}
+
 bool cache_args_ok(sinkattn_dtype dt, int Hkv, int D, int n_sink, int window) {
   return (dt == SINKATTN_BF16 || dt == SINKATTN_FP32) && Hkv >= 1 && (D == 64 || D == 128) &&
          n_sink >= 0 && window >= 0 && n_sink + window >= 1;
@@ -106,5 +162,26 @@ extern "C" int sinkattn_cache_fill(sinkattn_dtype dt, int n_seq, int T_tot, int 
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), cu_seqlens, n_seq, T_tot,
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), cache_seqlens_out,
       n_sink + window, n_sink, window, row16);
+  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+extern "C" int sinkattn_cache_append_fp8(int B, int Hkv, int D, int n_sink, int window,
+                                         const void* k_new, const void* v_new,
+                                         const int32_t* cache_seqlens, void* k_sink,
+                                         void* v_sink, void* k_win, void* v_win,
+                                         const float* k_scale, const float* v_scale,
+                                         sinkattn_stream_t stream) {
+  if (!cache_args_ok(SINKATTN_BF16, Hkv, D, n_sink, window) || B < 1)
+    return SINKATTN_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !cache_seqlens || !a16(k_new) || !a16(v_new))
+    return SINKATTN_ERR_INVALID_ARG;
+  if (n_sink > 0 && (!k_sink || !v_sink || !a16(k_sink) || !a16(v_sink)))
+    return SINKATTN_ERR_INVALID_ARG;
+  if (window > 0 && (!k_win || !v_win || !k_scale || !v_scale || !a16(k_win) || !a16(v_win)))
+    return SINKATTN_ERR_INVALID_ARG;
+  cache_append_fp8_kernel<<<B, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), cache_seqlens,
+      static_cast<uint4*>(k_sink), static_cast<uint4*>(v_sink), static_cast<uint2*>(k_win),
+      static_cast<uint2*>(v_win), k_scale, v_scale, Hkv, D, n_sink, window);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }

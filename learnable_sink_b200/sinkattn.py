@@ -85,6 +85,7 @@ def lib():
         L.sinkattn_decode_fp8.argtypes = [_i, _i, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp, _i, _vp,
                                           _sz, _vp]
+        L.sinkattn_cache_append_fp8.argtypes = [_i, _i, _i, _i, _i] + [_vp] * 9 + [_vp]
         L.sinkattn_cache_append.argtypes = [_i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]
         L.sinkattn_cache_fill.argtypes = [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _vp]
@@ -434,6 +435,32 @@ def cache_append(k_new, v_new, cache_seqlens, k_cache, v_cache, n_sink: int, win
     _check("sinkattn_cache_append", lib().sinkattn_cache_append(
         _dt(k_new), B, Hkv, D, int(n_sink), int(window), _ptr(k_new), _ptr(v_new),
         _ptr(cache_seqlens), _ptr(k_cache), _ptr(v_cache), _stream(stream)))
+
+
+def cache_append_fp8(k_new, v_new, cache_seqlens, k_sink, v_sink, k_win, v_win, k_scale,
+                     v_scale, n_sink: int, window: int, stream=None) -> None:
+    """Write one new bf16 token per sequence (k_new/v_new [B, Hkv, D]) into
+    the mixed-precision cache of decode_fp8: a sink slot as it is, a window
+    row as E4M3 codes of value / scale; cache_seqlens [B] int32 already
+    counts the new token."""
+    fn = "sinkattn_cache_append_fp8"
+    _want(fn, k_new.dim() == 3 and k_new.dtype == torch.bfloat16, "k_new must be bf16 [B, Hkv, D]")
+    B, Hkv, D = k_new.shape
+    _shape(fn, "v_new", v_new, k_new.shape, k_new.dtype)
+    for name, t in (("k_sink", k_sink), ("v_sink", v_sink)):
+        _shape(fn, name, t, (B, n_sink, Hkv, D), torch.bfloat16)
+    for name, t in (("k_win", k_win), ("v_win", v_win)):
+        if t is not None:
+            _want(fn, t.element_size() == 1, f"{name} must hold 1-byte E4M3 codes")
+        _shape(fn, name, t, (B, window, Hkv, D))
+    for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        _shape(fn, name, t, (Hkv,), torch.float32)
+    _shape(fn, "cache_seqlens", cache_seqlens, (B,), torch.int32)
+    _contig(k_new, v_new, cache_seqlens, k_sink, v_sink, k_win, v_win, k_scale, v_scale)
+    _check(fn, lib().sinkattn_cache_append_fp8(
+        B, Hkv, D, int(n_sink), int(window), _ptr(k_new), _ptr(v_new), _ptr(cache_seqlens),
+        _ptr(k_sink), _ptr(v_sink), _ptr(k_win), _ptr(v_win), _ptr(k_scale), _ptr(v_scale),
+        _stream(stream)))
 
 
 def cache_fill(k, v, cu_seqlens, k_cache, v_cache, n_sink: int, window: int,

@@ -275,6 +275,57 @@ def fp8_e4m3_value(codes):
     return sign * val
 
 
+def fp8_e4m3_encode(x):
+    """E4M3 code of each value (float32 or float64 array): the nearest value
+    of the format's grid (fp8_e4m3_value), ties to the code with an even
+    mantissa, magnitudes beyond the largest finite value (448) saturated to
+    it, NaN -> the NaN code 0x7F; the sign bit carries the sign (-0.0 and
+    negative values that round to zero give 0x80).  Found by search over the
+    127 non-negative finite codes, whose values increase with the code."""
+    x = np.asarray(x, dtype=np.float64)
+    grid = fp8_e4m3_value(np.arange(0x7F, dtype=np.uint8))  # codes 0x00..0x7E, ascending
+    a = np.abs(x)
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 1, len(grid) - 1)  # grid[hi-1] < a <= grid[hi]
+    lo = hi - 1
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a <= 0.0, 0, code)
+    code = np.where(a >= grid[-1], 0x7E, code)  # saturate
+    code = code | np.where(np.signbit(x), 0x80, 0)
+    code = np.where(np.isnan(x), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def cache_append_fp8(k_new, v_new, cache_seqlens, k_sink, v_sink, k_win, v_win, k_scale,
+                     v_scale, n_sink, window):
+    """Mixed-precision ring-cache append (page "Attention Sink / StreamingLLM":
+    a fixed sink segment kept in high precision, the sliding window stored
+    low).  The token at position p = cache_seqlens[b] - 1 goes to sink slot p
+    (copied) if p < n_sink, else to window row (p - n_sink) mod window as E4M3
+    codes of value / scale (scale of its KV head; the division in float32, as
+    the values and scales are float32).  Returns new copies of the four
+    caches (k_sink, v_sink bf16-valued float64 arrays; k_win, v_win uint8)."""
+    ks, vs = _f64(k_sink).copy(), _f64(v_sink).copy()
+    kw, vw = _u8arr(k_win).copy(), _u8arr(v_win).copy()
+    kn, vn = np.asarray(_f64(k_new), dtype=np.float32), np.asarray(_f64(v_new), dtype=np.float32)
+    ksc = np.asarray(_f64(k_scale), dtype=np.float32)
+    vsc = np.asarray(_f64(v_scale), dtype=np.float32)
+    cs = np.asarray(cache_seqlens).astype(np.int64).reshape(-1)
+    for b, n in enumerate(cs):
+        pos = int(n) - 1
+        if pos < 0:
+            continue
+        if pos < n_sink:
+            ks[b, pos] = kn[b]
+            vs[b, pos] = vn[b]
+        elif window > 0:
+            r = (pos - n_sink) % window
+            kw[b, r] = fp8_e4m3_encode((kn[b] / ksc[:, None]).astype(np.float32))
+            vw[b, r] = fp8_e4m3_encode((vn[b] / vsc[:, None]).astype(np.float32))
+    return ks, vs, kw, vw
+
+
 def decode_fp8_window(q, k_sink, v_sink, k_win, v_win, k_scale, v_scale, cache_seqlens,
                       n_sink, window, sink, scale):
     """Ring-buffer decode with a mixed-precision cache (page "Attention Sink /

@@ -133,3 +133,41 @@ def test_fp8_decode_matches_bf16_decode_of_dequantised_cache():
     assert max_abs(np64(got[1]), np64(ref[1])) <= 1e-3
     assert max_abs(np64(got[2]), np64(ref[2])) <= 1e-3
     check_status()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp8_cache_append_bit_exact_then_decode(D):
+    """Appends into the mixed-precision cache are bit-exact against the
+    oracle's slot rule and E4M3 encoder (positions in the sink segment, in
+    the window, past a wrap, and an empty sequence); a decode over the
+    appended cache then matches the oracle."""
+    S.clear_status()
+    d = W.decode(B=6, n_sink=4, window=40, Hq=8, Hkv=2, D=D, seqlen_range=(0, 200),
+                 seed_offset=51)
+    ks, vs, kw, vw, ksc, vsc = W.fp8_window_cache(d, seed=W.SEED_BASE + 506)
+    gen = torch.Generator().manual_seed(W.SEED_BASE + 507)
+    B, Hkv = d.q.shape[0], d.k_cache.shape[2]
+    cs = torch.tensor([0, 1, 4, 5, 44, 173], dtype=torch.int32)  # positions -1, 0, 3, 4, 43, 172
+    kn = (torch.randn(B, Hkv, D, generator=gen) * 3).to(torch.bfloat16)
+    vn = (torch.randn(B, Hkv, D, generator=gen) * 3).to(torch.bfloat16)
+    kn[5, 0, :4] = torch.tensor([1e4, -1e4, 0.0, -0.0], dtype=torch.bfloat16)  # saturation, signed 0
+    ref = oracle.cache_append_fp8(kn, vn, cs, ks, vs, kw, vw, ksc, vsc, d.n_sink, d.window)
+    dev = [t.cuda().contiguous() for t in (ks, vs, kw, vw, ksc, vsc)]
+    S.cache_append_fp8(kn.cuda(), vn.cuda(), cs.cuda(), dev[0], dev[1], dev[2], dev[3], dev[4],
+                       dev[5], d.n_sink, d.window)
+    torch.cuda.synchronize()
+    assert np.array_equal(dev[0].float().cpu().double().numpy(), ref[0])
+    assert np.array_equal(dev[1].float().cpu().double().numpy(), ref[1])
+    assert np.array_equal(dev[2].cpu().numpy(), ref[2])
+    assert np.array_equal(dev[3].cpu().numpy(), ref[3])
+    # decode over the appended cache, every sequence at its new length
+    out, lse, ss = S.decode_fp8(d.q.cuda(), dev[0], dev[1], dev[2], dev[3], dev[4], dev[5],
+                                cs.cuda(), d.n_sink, d.window, d.sink.cuda(), scale=d.scale)
+    torch.cuda.synchronize()
+    ro, rl, rs = oracle.decode_fp8_window(d.q, ref[0], ref[1], ref[2], ref[3], ksc, vsc, cs,
+                                          d.n_sink, d.window, d.sink, d.scale)
+    tol = TOL[torch.bfloat16]
+    assert max_abs(np64(out), ro) <= tol["o"]
+    check_lse(np64(lse), rl, tol["lse"])
+    assert max_abs(np64(ss), rs) <= tol["ss"]
+    check_status()

@@ -696,3 +696,53 @@ def test_fp8_window_decode_is_the_decode_of_the_dequantised_cache():
     for a, b in zip(got2, ref2):
         np.testing.assert_allclose(a, b, rtol=0, atol=1e-15)
     assert not np.allclose(got2[0], got[0])
+
+
+def test_fp8_e4m3_encode_round_trips_every_code():
+    """Every finite code's value encodes back to that code (both signs)."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = oracle.fp8_e4m3_value(codes)
+    got = oracle.fp8_e4m3_encode(vals)
+    # +0 and -0 are distinct codes with the same value: the sign bit decides
+    assert np.array_equal(got, codes)
+
+
+def test_fp8_e4m3_encode_matches_the_library_conversion_in_range():
+    """Round to nearest, ties to even, against torch's float8_e4m3fn cast on
+    values inside the format's range (where the cast does not saturate)."""
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(0, 30, 20000), rng.uniform(-448, 448, 20000),
+                        rng.normal(0, 1e-2, 5000)]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.fp8_e4m3_encode(x), ref)
+
+
+def test_fp8_e4m3_encode_closed_forms():
+    """Ties go to the even mantissa, magnitudes past 448 saturate, NaN keeps
+    the NaN code, tiny values round to signed zero."""
+    x = np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 448.0, 464.0, 1e6, -1e6,
+                  float("nan"), -1e-30, 0.0, -0.0])
+    want = [0x38, 0x3A, 0x00, 0x02, 0x7E, 0x7E, 0x7E, 0xFE, 0x7F, 0x80, 0x00, 0x80]
+    assert oracle.fp8_e4m3_encode(x).tolist() == want
+
+
+def test_fp8_cache_append_slot_rule():
+    """Positions below n_sink land in the bf16 sink slots unchanged; later
+    positions land in window row (p - n_sink) mod window as codes of
+    value / scale; a sequence with no token writes nothing."""
+    B, Hkv, D, ns, win = 3, 2, 4, 2, 5
+    kn = np.arange(B * Hkv * D, dtype=np.float64).reshape(B, Hkv, D) / 8.0
+    vn = -kn
+    ks = np.zeros((B, ns, Hkv, D))
+    kw = np.zeros((B, win, Hkv, D), dtype=np.uint8)
+    sc = np.array([0.5, 0.25], dtype=np.float32)
+    cs = np.array([2, 0, 9], dtype=np.int32)  # positions 1, none, 8
+    k2, v2, kw2, vw2 = oracle.cache_append_fp8(kn, vn, cs, ks, ks, kw, kw, sc, sc, ns, win)
+    assert np.array_equal(k2[0, 1], kn[0]) and np.array_equal(v2[0, 1], vn[0])
+    assert not k2[1].any() and not kw2[1].any()
+    r = (8 - ns) % win
+    assert np.array_equal(kw2[2, r], oracle.fp8_e4m3_encode(kn[2] / sc[:, None]))
+    # within half a grid step (1/16 relative for normal values) of the value
+    back = oracle.fp8_e4m3_value(kw2[2, r]) * sc[:, None]
+    assert np.all(np.abs(back - kn[2]) <= np.abs(kn[2]) / 16 + 1e-12)
+    assert np.count_nonzero(kw2.reshape(B, win, -1).any(axis=2)) == 1
