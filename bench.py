@@ -312,6 +312,58 @@ def measure_decode_kernel(S, decode_step, flush, flush_rd, reps=20):
     return sorted(ts)[len(ts) // 2]
 
 
+def measure_fp8_decode(S, dec, dev, flush, flush_rd, reps=20):
+    """The FP8 window-cache decode on the StreamingLLM decode workload (the
+    same cache with its window slots as E4M3 codes): median CUDA-event time
+    of the whole call and of its streaming kernel, L2 flushed before each
+    call, and the call's algorithmic bytes (filled sink rows in bf16, filled
+    window rows as codes, Q/O bf16, LSE and sink_s)."""
+    cache = [t.to(dev) for t in W.fp8_window_cache(dec, seed=W.SEED_BASE + 501)]
+    q, cs, sink = dec.q.to(dev), dec.cache_seqlens.to(dev), dec.sink.to(dev)
+    B, Hq, D = dec.q.shape
+    Hkv = dec.k_cache.shape[2]
+    n = torch.clamp(dec.cache_seqlens.long(), min=0, max=dec.n_sink + dec.window)
+    sink_rows = int(torch.clamp(n, max=dec.n_sink).sum())
+    win_rows = int((n - torch.clamp(n, max=dec.n_sink)).sum())
+    kv_bytes = 2 * Hkv * D * (2 * sink_rows + win_rows)
+    nbytes = kv_bytes + 2 * B * Hq * D * 2 + 2 * B * Hq * 4 + B * 4 + 2 * Hkv * 4
+    splits = S.decode_fp8_num_splits(B, Hq, Hkv, D, dec.n_sink, dec.window)
+    ws = torch.empty(S.decode_workspace_bytes(B, Hq, D, splits), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ss = torch.empty_like(lse)
+
+    def call():
+        S.decode_fp8(q, *cache, cs, dec.n_sink, dec.window, sink, scale=dec.scale,
+                     num_splits=splits, workspace=ws, out=out, lse=lse, sink_s=ss)
+
+    for _ in range(3):
+        call()
+    res = {}
+    for mode in ("call", "kernel"):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            flush_rd.sum()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            if mode == "kernel":
+                e1.record()
+                S.set_kernel_events(S.KERNEL_DECODE, e0, e1)
+            call()
+            if mode == "kernel":
+                S.set_kernel_events(S.KERNEL_DECODE, None, None)
+            else:
+                e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        res[mode + "_ms"] = sorted(ts)[len(ts) // 2]
+    res.update(bytes=nbytes, kernel_bytes=kv_bytes, num_splits=splits,
+               call_gbs=nbytes / (res["call_ms"] * 1e-3) / 1e9)
+    return res
+
+
 def measure_gates(S, q, k, lse, sink_s, mask, scale, flush, flush_rd, hbm_gbs, reps=10):
     """Gate rows on the prefill's tensors: the sink-free model's gate (reads Q
     once; Q is larger than L2) and the head importance (reads sink_s once;
@@ -349,10 +401,46 @@ def measure_gates(S, q, k, lse, sink_s, mask, scale, flush, flush_rd, hbm_gbs, r
     return res
 
 
+def run_profile_workload(args, dev):
+    """Launches of one workload's kernels for an external profiler (warm-up +
+    steps, nothing timed, no JSON line): the band or varlen block-sparse
+    plan+fwd+bwd, or the FP8 window-cache decode."""
+    from learnable_sink_b200 import sinkattn as S
+    torch.cuda.set_device(dev)
+    if args.profile_workload in ("band", "varlen"):
+        inp = W.band() if args.profile_workload == "band" else W.varlen()
+        T, Hq, Hkv, D = inp.shape
+        q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+        sink, dout = inp.sink.to(dev), inp.dout.to(dev)
+        mask = S.Mask.from_spec(inp.mask, dev)
+        plan = S.Plan(T, Hq, Hkv, mask)
+        out = torch.empty_like(q)
+        lse = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+        ss = torch.empty_like(lse)
+        ws = torch.empty(S.bwd_workspace_bytes(q, k, mask), dtype=torch.uint8, device=dev)
+
+        def step():
+            plan.rebuild()
+            S.fwd(q, k, v, sink, mask, plan, scale=inp.scale, out=out, lse=lse, sink_s=ss)
+            S.bwd(q, k, v, out, dout, lse, sink, mask, plan, scale=inp.scale, workspace=ws)
+    else:  # fp8 decode
+        dec = W.decode()
+        cache = [t.to(dev) for t in W.fp8_window_cache(dec, seed=W.SEED_BASE + 501)]
+        qd, cs, dsk = dec.q.to(dev), dec.cache_seqlens.to(dev), dec.sink.to(dev)
+
+        def step():
+            S.decode_fp8(qd, *cache, cs, dec.n_sink, dec.window, dsk, scale=dec.scale)
+    for _ in range(args.warmup + args.steps):
+        step()
+    torch.cuda.synchronize()
+
+
 def run_ours(args, world, rank, local):
     from learnable_sink_b200 import sinkattn as S
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.profile_workload:
+        return run_profile_workload(args, dev)
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
 
@@ -553,11 +641,16 @@ def run_ours(args, world, rank, local):
                 "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "frac_of_8tbs": ach / 8000.0,
                 "ms": ms, "bytes": nbytes, "traffic": load_traffic(kernel, workload)}
 
+    fp8 = measure_fp8_decode(S, dec, dev, flush, flush_rd)
     rooflines = [
         tensor_entry("fwd_tc_kernel", "training_prefill", kf_ms, flop_fwd),
         tensor_entry("bwd_tc_kernel", "training_prefill", kb_ms, flop_bwd),
         hbm_entry("decode_warp_kernel", "streamingllm_decode", kd_ms, dec_kernel_bytes),
         hbm_entry("decode call (stream + merge)", "streamingllm_decode", decode_ms / K, dec_bytes),
+        hbm_entry("decode_fp8_kernel", "streamingllm_decode_fp8_window", fp8["kernel_ms"],
+                  fp8["kernel_bytes"]),
+        hbm_entry("decode_fp8 call (stream + merge)", "streamingllm_decode_fp8_window",
+                  fp8["call_ms"], fp8["bytes"]),
         hbm_entry("gate_vanilla_kernel", "training_prefill", gates["gate_vanilla"]["ms"],
                   gates["gate_vanilla"]["bytes"]),
     ]
@@ -590,6 +683,7 @@ def run_ours(args, world, rank, local):
         "decode": {"value": dec_gbs, "unit": "GB/s", "ms_per_call": decode_ms / K,
                    "bytes_per_call": dec_bytes, "num_splits": n_splits,
                    "frac": dec_gbs / hbm, "frac_of_8tbs": dec_gbs / 8000.0},
+        "decode_fp8_window": fp8,
         "step_breakdown_ms": {
             "prefill": prefill_ms / K, "decode_call": decode_ms / K,
             "l2_flush_and_gaps": flush_ms,
@@ -682,6 +776,8 @@ def main():
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps of the prefill and decode stages for a profiler "
                          "(no timing, no JSON line)")
+    ap.add_argument("--profile-workload", choices=["band", "varlen", "fp8"], default=None,
+                    help="like --profile, for one other workload's kernels")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the band / varlen block-sparse measurements")
     ap.add_argument("--dry-run", action="store_true",

@@ -187,9 +187,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   float* s_dl = reinterpret_cast<float*>(smem + C::OFF_DL);
 
   const PlanHdr* hdr = reinterpret_cast<const PlanHdr*>(p.plan);
-  const int rank = blockIdx.x / p.per_item;
+  // KV head slowest (lists shared by the KV heads): the CTAs of one
+  // (KV head, sequence) are launched together
+  const int rank = blockIdx.x % hdr->cap_units;
   if (rank >= min(hdr->n_bwd_units, hdr->cap_units)) return;
-  const int rem = blockIdx.x % p.per_item;
+  const int rem = blockIdx.x / hdr->cap_units;
   // work unit: a slice of one key tile's reverse list (long lists are split)
   const int4 unit = reinterpret_cast<const int4*>(p.plan + hdr->off_bwd_units)[
       p.plan[hdr->off_bwd_unit_order + rank]];

@@ -316,8 +316,8 @@ __global__ void plan_zero_kernel(int* p, int n) {
 }
 
 // H: backward work units.  One CTA scans the per-item unit counts (item
-// order), then every item writes its units, then the units are ordered
-// longest first (counting sort on the entry count, at most kBwdChunk).
+// order), then every item writes its units, then the launch order is set
+// (item order).
 __global__ void __launch_bounds__(kScanThreads) plan_units_scan_kernel(PlanArgs a) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
@@ -353,31 +353,20 @@ __global__ void plan_units_fill_kernel(PlanArgs a) {
   const int n = bwd_units_of(it.entry_len);
   const int b = a.plan[a.off_unit_base + i];
   int4* units = reinterpret_cast<int4*>(a.plan + a.off_bwd_units);
+  // near-equal parts: unit c takes entries [c len / n, (c + 1) len / n)
   for (int c = 0; c < n && b + c < a.cap_units; ++c) {
-    const int first = c * kBwdChunk;
-    const int cnt = min(kBwdChunk, it.entry_len - first);
-    units[b + c] = make_int4(i, first, max(cnt, 0), n);
+    const int first = (int)((long long)c * it.entry_len / n);
+    const int last = (int)((long long)(c + 1) * it.entry_len / n);
+    units[b + c] = make_int4(i, first, max(last - first, 0), n);
   }
 }
 
-__global__ void __launch_bounds__(kScanThreads) plan_units_order_kernel(PlanArgs a) {
-  __shared__ int cursor[kBwdChunk + 1];
-  __shared__ int hist[kBwdChunk + 1];
+__global__ void plan_units_order_kernel(PlanArgs a) {
+  // item order: units of one (KV-head slot, sequence) are consecutive
   const int n_units = min(hdr(a)->n_bwd_units, a.cap_units);
-  const int4* units = reinterpret_cast<const int4*>(a.plan + a.off_bwd_units);
   int* order = a.plan + a.off_bwd_unit_order;
-  if (threadIdx.x <= kBwdChunk) hist[threadIdx.x] = 0;
-  __syncthreads();
-  for (int u = threadIdx.x; u < n_units; u += kScanThreads)
-    atomicAdd(&hist[kBwdChunk - units[u].z], 1);  // bin 0 = longest
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int b = 0; b <= kBwdChunk; ++b) { cursor[b] = run; run += hist[b]; }
-  }
-  __syncthreads();
-  for (int u = threadIdx.x; u < n_units; u += kScanThreads)
-    order[atomicAdd(&cursor[kBwdChunk - units[u].z], 1)] = u;
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < n_units; u += gridDim.x * blockDim.x)
+    order[u] = u;
 }
 
 // G: sort every reverse list by query tile, latest first (insertion sort;
@@ -480,7 +469,7 @@ int launch_plan(const PlanLaunch& L, cudaStream_t stream) {
   plan_bwd_sort_kernel<<<nb, 256, 0, stream>>>(a);
   plan_units_scan_kernel<<<1, kScanThreads, 0, stream>>>(a);
   plan_units_fill_kernel<<<nb, 256, 0, stream>>>(a);
-  plan_units_order_kernel<<<1, kScanThreads, 0, stream>>>(a);
+  plan_units_order_kernel<<<(z.cap_units + 255) / 256, 256, 0, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

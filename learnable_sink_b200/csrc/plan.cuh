@@ -21,8 +21,14 @@
 //   bwd_units[cap_units][4] backward work units: (bwd item, first entry,
 //                        entry count, number of units of that item); a
 //                        reverse list longer than kBwdChunk entries is split
-//                        so no single CTA serialises a very popular key tile
-//   bwd_unit_order[cap_units] units, longest first
+//                        into near-equal parts, so no single CTA serialises a
+//                        very popular key tile and no unit is much longer
+//                        than the others
+//   bwd_unit_order[cap_units] units in item order: (KV-head slot, sequence,
+//                        key tile), so the units of one sequence and KV head
+//                        -- which reduce into the same dQ tiles and read the
+//                        same Q/dO tiles -- run at about the same time and
+//                        find those tiles in L2
 //   unit_base[cap_items] first unit of every bwd item
 // With no block_indices the lists do not depend on the KV head: one slot
 // (kvh = -1) serves every KV head.
@@ -33,7 +39,7 @@ namespace sk {
 
 constexpr int kPlanMagic = 0x534b4150;  // 'SKAP'
 constexpr int kHdrWords = 32;
-constexpr int kBwdChunk = 32;  // reverse-list entries per backward work unit
+constexpr int kBwdChunk = 16;  // most reverse-list entries per backward work unit
 
 struct PlanHdr {
   int magic;

@@ -315,7 +315,7 @@ BF16_BWD = {
     "extreme_sinks": dict(cu=[0, 260], Hq=4, Hkv=1, D=128, sink_values=[-80.0, -20.0, 20.0, 80.0]),
     "non_causal": dict(cu=[0, 100, 300], Hq=4, Hkv=2, D=128, causal=False),
     # key tile 0 is seen by 34 query tiles: its reverse list is split into
-    # two work units whose fp32 dK/dV are summed through the accumulator
+    # work units whose fp32 dK/dV are summed through the accumulator
     "causal_split_list_D64": dict(cu=[0, 4300], Hq=4, Hkv=2, D=64),
     "band_split_list_D128": dict(cu=[0, 4300], Hq=4, Hkv=1, D=128, n_sink=4, window=300),
 }
