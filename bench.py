@@ -97,15 +97,20 @@ class ClockSampler:
         self.stop = threading.Event()
         self.source = None
 
+    def _pci_bus_id(self) -> bytes:
+        """NVML's PCI bus id string ("domain:bus:device.0") of the CUDA device,
+        built from the integer fields torch reports (CUDA and NVML may number
+        devices differently)."""
+        pr = torch.cuda.get_device_properties(self.index)
+        dom, bus, dev = (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))
+        return f"{dom:08X}:{bus:02X}:{dev:02X}.0".encode()
+
     def _nvml_handle(self):
         import pynvml
         pynvml.nvmlInit()
-        try:
-            bus = torch.cuda.get_device_properties(self.index).pci_bus_id
-            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode()
-                                                                  if isinstance(bus, str) else bus)
-        except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        # the lookup takes a C string: pass bytes only (pynvml hands its
+        # argument to c_char_p, which treats an integer as an address)
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(self._pci_bus_id())
 
     def _nvml_loop(self, nv, h):
         get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
@@ -144,8 +149,12 @@ class ClockSampler:
             self.source = "nvml"
         except Exception:
             try:
+                try:
+                    which = self._pci_bus_id().decode()
+                except Exception:
+                    which = str(self.index)
                 self.proc = subprocess.Popen(
-                    ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.SMI_FIELDS}",
+                    ["nvidia-smi", "-i", which, f"--query-gpu={self.SMI_FIELDS}",
                      "--format=csv,noheader,nounits", "-lms", "50"],
                     stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
                 self.thread = threading.Thread(target=self._smi_read, daemon=True)

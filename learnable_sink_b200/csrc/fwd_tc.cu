@@ -3,7 +3,7 @@
 // Page "Attention Sink, Learnable Sink and dsink": scores and GQA map
 // (section 1), the sink logit folded into the softmax denominator with a zero
 // value (section 4), LSE_new and the gate sink_s (sections 4 and 9); page
-// "Attention Sink Forges Native MoE" (section 5) reads the same gate as
+// "Attention Sink and the native MoE in attention layers" (section 5) reads the same gate as
 // G = sigma(LSE - sink).
 //
 // One CTA = NQT query tiles of 128 rows that share a token range and a KV

@@ -86,6 +86,15 @@ def test_noalloc_decode_matches_oracle_and_workspace_decode_twice(case, num_spli
     ref = S.decode(t["q"], t["k"], t["v"], t["cs"], d.n_sink, d.window, t["sink"],
                    scale=d.scale)
     outs = [_outputs(d), _outputs(d)]
+    B, Hq, D = d.q.shape
+    if num_splits > 0:
+        # an explicit count is first lowered like the workspace decode's
+        # (to the 16-row pieces of one pair, at most 128); if the partials
+        # then exceed the 4 MiB array the call is refused before any launch
+        n = min(num_splits, -(-(d.n_sink + d.window) // 16), 128)
+        if -(-(4 * B * Hq * n * (D + 2)) // 256) * 256 > 4 << 20:
+            assert _call_noalloc(d, t, outs[0], num_splits) == 4  # SINKATTN_ERR_WORKSPACE
+            return
     # first call: looks up the array's address (and loads the kernels)
     assert _call_noalloc(d, t, outs[0], num_splits) == 0
     torch.cuda.synchronize()
