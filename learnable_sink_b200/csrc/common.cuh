@@ -7,7 +7,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
-#include <string.h>
 
 #include "../../include/sinkattn.h"
 
@@ -249,52 +248,6 @@ __device__ __forceinline__ void regs_to() {
   static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
   if constexpr (N > FROM) regs_inc<N>();
   else if constexpr (N < FROM) regs_dec<N>();
-}
-
-// ---------------------------------------------------------------- exp2 on the FMA pipe
-// 2^y for y <= 8 without the MUFU unit, to share the softmax's
-// exponentials between the two pipes (Cody-Waite range reduction plus a
-// polynomial): y is clamped to >= -126, n = round(y) by the 1.5 * 2^23
-// rounding constant, f = y - n in [-1/2, 1/2], 2^f from a cubic fitted to
-// 2^f on [-1/2, 1/2] by iteratively reweighted least squares toward the
-// minimax fit (Lawson's algorithm; max relative error 7.5e-5), and the
-// result is 2^f * 2^n with 2^n built from n's exponent bits.  `live` = 0
-// returns 0 (a row with no visible key so far).  The fp32 arithmetic is the
-// same per element in this scalar form and the packed form the kernels use.
-constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f,
-                kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.05517164617776871f;
-constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-__host__ __device__ __forceinline__ float exp2_poly(float y, float live) {
-  y = y > -126.f ? y : -126.f;
-  const float t = y + kRound;
-  const float n = t - kRound;
-  const float f = y - n;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  uint32_t tb;
-  memcpy(&tb, &t, 4);
-  const uint32_t sb = (tb + uint32_t(127 - 0x4B400000)) << 23;  // (n + 127) << 23
-  float sc;
-  memcpy(&sc, &sb, 4);
-  return p * (sc * live);
-}
-
-// Two exp2_poly evaluations on packed fp32x2 instructions; c0..c3 are the
-// polynomial's coefficients already multiplied by `live`.
-__device__ __forceinline__ float2 exp2_poly2(float2 y, float2 c0, float2 c1, float2 c2,
-                                             float2 c3) {
-  const float2 yc = make_float2(fmaxf(y.x, -126.f), fmaxf(y.y, -126.f));
-  const float2 t = __fadd2_rn(yc, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), yc);
-  float2 p = __ffma2_rn(c3, f, c2);
-  p = __ffma2_rn(p, f, c1);
-  p = __ffma2_rn(p, f, c0);
-  const float2 sc = make_float2(
-      __uint_as_float((__float_as_uint(t.x) << 23) + (uint32_t(127 - 0x4B400000) << 23)),
-      __uint_as_float((__float_as_uint(t.y) << 23) + (uint32_t(127 - 0x4B400000) << 23)));
-  return __fmul2_rn(p, sc);
 }
 
 // ---------------------------------------------------------------- misc

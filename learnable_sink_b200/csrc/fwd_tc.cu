@@ -56,12 +56,7 @@ struct FwdCfg {
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "not enough shared memory for a two-stage ring");
   static constexpr int MIN_BLOCKS = 1;
-  // Out of every 8 element pairs of a row, POLY8 take their exponentials on
-  // the FMA pipe (exp2_poly2) instead of the MUFU unit, whose 16 results per
-  // clock per SM would otherwise cap the tile rate: the exponentials of a
-  // 128 x 128 tile cost as many cycles as its two MMAs at D = 128, twice as
-  // many at D = 64.
-  static constexpr int POLY8 = D == 64 ? 3 : 2;
+
   // With two softmax warpgroups and one CTA per SM, registers are moved to the
   // softmax warpgroups: the producer and MMA warps then share a warpgroup with
   // two idle warps (setmaxnreg works on whole warpgroups), 12 warps in all,
@@ -446,13 +441,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       // on element pairs (packed fp32x2 instructions), the exponentials one
       // by one
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mu, -mu);
-      // polynomial coefficients times `live` (0 for a row that has seen no
-      // key yet: its scores are all -inf and its probabilities must be 0)
-      const float live = (m == -INFINITY) ? 0.f : 1.f;
-      const float2 pc0 = make_float2(kExp2C0 * live, kExp2C0 * live);
-      const float2 pc1 = make_float2(kExp2C1 * live, kExp2C1 * live);
-      const float2 pc2 = make_float2(kExp2C2 * live, kExp2C2 * live);
-      const float2 pc3 = make_float2(kExp2C3 * live, kExp2C3 * live);
       float2 rs4[4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) rs4[a] = make_float2(0.f, 0.f);
@@ -462,8 +450,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float2 y = __ffma2_rn(make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]), sc2, nm2);
-          const float2 pp = (i % 8) < C::POLY8 ? exp2_poly2(y, pc0, pc1, pc2, pc3)
-                                               : make_float2(fast_exp2(y.x), fast_exp2(y.y));
+          const float2 pp = make_float2(fast_exp2(y.x), fast_exp2(y.y));
           rs4[i & 3] = __fadd2_rn(rs4[i & 3], pp);
           pk[i] = pack_bf16x2(pp.x, pp.y);
         }
