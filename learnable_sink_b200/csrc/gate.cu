@@ -79,9 +79,12 @@ __global__ void gate_reduce_kernel(const double* part, int n_blocks, int Hq, int
 // HBM-bound (reads Q once).  A warp streams one token's contiguous Q row
 // [Hq, D] as 16-byte chunks, kGvInFlight per lane in flight; the CPH chunks
 // of a head row sit in CPH adjacent lanes, which reduce its dot product.
-// CTA = kGvRows tokens of one sequence.
-constexpr int kGvRows = 32;
-constexpr int kGvInFlight = 8;
+// CTA = kGvRows tokens of one sequence; the sequence's k_0 rows [Hkv, D] are
+// staged once in shared memory when they fit kGvK0Smem bytes (else read
+// through L1), so the loop's only global loads are Q's.
+constexpr int kGvRows = 64;
+constexpr int kGvInFlight = 16;
+constexpr int kGvK0Smem = 32 * 1024;
 
 template <typename T>
 __device__ __forceinline__ float dot16(const uint4& a, const uint4& b) {
@@ -131,6 +134,12 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
   const int n16 = a.Hq * CPH;  // chunks per token row
   const uint4* k0 = reinterpret_cast<const uint4*>(static_cast<const T*>(a.k) +
                                                    (long long)start * a.Hkv * D);
+  extern __shared__ uint4 k0s[];
+  const bool k0_in_smem = a.Hkv * CPH * 16 <= kGvK0Smem;
+  if (k0_in_smem) {
+    for (int j = threadIdx.x; j < a.Hkv * CPH; j += blockDim.x) k0s[j] = __ldg(k0 + j);
+    __syncthreads();
+  }
   for (int i = i0 + warp; i < min(len, i0 + kGvRows); i += 8) {
     const long long t = start + i;
     const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + t * a.Hq * D);
@@ -148,7 +157,8 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
         const int c = min(c0 + u * 32 + lane, n16 - 1);
         const int h = c / CPH;
         qv[u] = __ldg(qrow + c);
-        kv[u] = __ldg(k0 + (h / G) * CPH + (c - h * CPH));
+        const int kc = (h / G) * CPH + (c - h * CPH);
+        kv[u] = k0_in_smem ? k0s[kc] : __ldg(k0 + kc);
       }
       float dot[kGvInFlight];
 #pragma unroll
@@ -189,12 +199,14 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
 int launch_gate_vanilla(const GateVanillaArgs& a, int dt, int D, int max_seqlen,
                         cudaStream_t stream) {
   const dim3 grid((max_seqlen + kGvRows - 1) / kGvRows, a.n_seq);
+  const size_t k0_bytes = (size_t)a.Hkv * D * (dt == SINKATTN_BF16 ? 2 : 4);
+  const size_t smem = k0_bytes <= (size_t)kGvK0Smem ? k0_bytes : 0;
   if (dt == SINKATTN_BF16) {
-    if (D == 64) gate_vanilla_kernel<__nv_bfloat16, 64><<<grid, 256, 0, stream>>>(a);
-    else gate_vanilla_kernel<__nv_bfloat16, 128><<<grid, 256, 0, stream>>>(a);
+    if (D == 64) gate_vanilla_kernel<__nv_bfloat16, 64><<<grid, 256, smem, stream>>>(a);
+    else gate_vanilla_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(a);
   } else {
-    if (D == 64) gate_vanilla_kernel<float, 64><<<grid, 256, 0, stream>>>(a);
-    else gate_vanilla_kernel<float, 128><<<grid, 256, 0, stream>>>(a);
+    if (D == 64) gate_vanilla_kernel<float, 64><<<grid, 256, smem, stream>>>(a);
+    else gate_vanilla_kernel<float, 128><<<grid, 256, smem, stream>>>(a);
   }
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }

@@ -123,3 +123,33 @@ def test_decode_split_heuristic(lib):
     assert f(1, 8, 1, 128, 4, 100000) == 126               # ceil(6250 / 50) + 1
     assert f(4096, 64, 8, 128, 4, 1020) == 2               # runs longer than a pair
     assert f(0, 8, 1, 128, 4, 100) == 1                    # degenerate sizes
+
+
+def test_decode_fp8_host_validation_and_split_heuristic(lib):
+    """The mixed-precision decode's host checks refuse bad arguments before any
+    device query; its split count follows the same rule over its pieces
+    (16-row sink pieces, 32-row window pieces)."""
+    f = lib.sinkattn_decode_fp8
+    f.argtypes = [ctypes.c_int] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 8 + \
+        [ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_void_p,
+                                                                 ctypes.c_size_t, ctypes.c_void_p]
+    a = 256  # stand-in 16-byte-aligned device address: never dereferenced here
+    ok = [a] * 8  # q k_sink v_sink k_win v_win k_scale v_scale cache_seqlens
+
+    def call(B=2, Hq=8, Hkv=2, D=128, ptrs=ok, n_sink=4, window=60, out=a, ws=a, ws_bytes=1 << 20):
+        return f(B, Hq, Hkv, D, 0.1, *ptrs, n_sink, window, None, out, a, None, 0, ws, ws_bytes,
+                 None)
+
+    assert call(D=96) == 1                        # head dimension
+    assert call(Hq=6, Hkv=4) == 1                 # Hq % Hkv
+    assert call(Hq=32, Hkv=2) == 2                # 16 query heads per KV head: unsupported
+    assert call(n_sink=0, window=0) == 1          # empty cache
+    assert call(ptrs=[a, None] + ok[2:]) == 1     # sink slots without k_sink
+    assert call(ptrs=ok[:3] + [a + 8] + ok[4:]) == 1  # misaligned window codes
+    assert call(out=None) == 1
+    assert call(ws_bytes=16) == 4                 # workspace too small
+    ns = lib.sinkattn_decode_fp8_num_splits
+    # 32 x 8 pairs x (1 sink piece + 32 window pieces) over 1184 warps: runs
+    # of 8 pieces, so a pair meets ceil(32 / 8) + 1 runs
+    assert ns(32, 32, 8, 128, 4, 1020) == 5
+    assert ns(1, 8, 1, 128, 0, 32) == 1           # one piece per pair
