@@ -256,6 +256,17 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def executed_pairs(plan, Hq, Hkv):
+    """(query, key, head) triples of the tiles the plan lists (visible or
+    masked inside a partial tile): the work the kernels execute, read from the
+    plan header's entry count (int32 word 12) and tile size (word 4); a list
+    entry covers tile x tile pairs for every query head of its KV-head slot."""
+    h = plan.buf[:64].cpu().view(torch.int32).tolist()
+    tile, kh_slots, n_entries = h[4], h[5], h[12]
+    heads = Hq if kh_slots == 1 else Hq // Hkv
+    return n_entries * tile * tile * heads
+
+
 def measure_config(S, inp, dev, steps=10, warmup=3):
     """Plan+fwd+bwd of one workload: per-call and per-kernel times (CUDA events)."""
     T, Hq, Hkv, D = inp.shape
@@ -296,7 +307,10 @@ def measure_config(S, inp, dev, steps=10, warmup=3):
         return sum(x.elapsed_time(y) for x, y in zip(ev[a], ev[b])) / steps
 
     step_ms, f_ms, b_ms = mean("s0", "s1"), mean("f0", "f1"), mean("b0", "b1")
-    return {"workload": inp.name, "visible_pairs": pairs, "D": D,
+    ex = executed_pairs(plan, Hq, Hkv)
+    return {"workload": inp.name, "visible_pairs": pairs, "D": D, "executed_pairs": ex,
+            "executed_fwd_tflops": 4 * D * ex / (f_ms * 1e-3) / 1e12,
+            "executed_bwd_tflops": 10 * D * ex / (b_ms * 1e-3) / 1e12,
             "plan_fwd_bwd_ms": step_ms, "tflops": 14 * D * pairs / (step_ms * 1e-3) / 1e12,
             "fwd_kernel_ms": f_ms, "fwd_kernel_tflops": 4 * D * pairs / (f_ms * 1e-3) / 1e12,
             "bwd_kernel_ms": b_ms, "bwd_kernel_tflops": 10 * D * pairs / (b_ms * 1e-3) / 1e12}
@@ -685,6 +699,7 @@ def run_ours(args, world, rank, local):
                         "(+ StreamingLLM decode B32 cache 4+1020 Hq32 Hkv8 D128 per step)",
             "global_batch": 4 * world, "seq_len": 4096, "parallelism": f"dp{world}",
             "visible_pairs_per_rank": pairs,
+            "executed_pairs_per_rank": executed_pairs(plan, Hq, Hkv),
             "l2": "prefill inputs larger than L2; before each decode L2 is flushed by writing "
                   "252 MB and then reading another 252 MB (dirty lines written back before "
                   "the decode starts)",
