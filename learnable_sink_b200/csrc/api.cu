@@ -208,7 +208,7 @@ int sinkattn_fwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float 
   p.scale = scale;
   p.lse_orig = lse_orig;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dt == SINKATTN_FP32) return launch_fwd_simt(p, out, lse_new, sink_s, s);
+  if (dt == SINKATTN_FP32) return launch_fwd_tf32(p, out, lse_new, sink_s, s);
   return launch_fwd_tc(p, out, lse_new, sink_s, s);
 }
 

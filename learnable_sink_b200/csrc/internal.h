@@ -57,7 +57,8 @@ bool make_tmap_3d_plain(CUtensorMap* map, const void* base, int T, int H, int D,
                         int box_t);
 
 // forward
-int launch_fwd_simt(const AttnProblem& p, void* out, float* lse, float* sink_s,
+// fp32 inputs: 3xTF32 tensor-core forward
+int launch_fwd_tf32(const AttnProblem& p, void* out, float* lse, float* sink_s,
                     cudaStream_t stream);
 int launch_fwd_tc(const AttnProblem& p, void* out, float* lse, float* sink_s,
                   cudaStream_t stream);

@@ -1,10 +1,9 @@
-// Exact-fp32 CUDA-core path for fp32 inputs (tensor cores would round the
-// operands).  One warp owns one (row, head); lanes split the head dimension.
-// Forward: online softmax over the plan's key tiles, then the sink epilogue
-// (page "Attention Sink, Learnable Sink and dsink", section 4: the sink logit
-// a_h joins the denominator unscaled and carries a zero value).  Backward:
-// dQ per row and dK/dV per key from P = exp(x - L_new) and Delta (sections
-// 7-8), visiting only the tiles the plan lists.
+// fp32 backward on the CUDA cores (the fp32 forward runs on the tensor cores
+// with the 3xTF32 split, fwd_tf32.cu).  One warp owns one (row, head) for dQ
+// and one (key, KV head) for dK/dV; lanes split the head dimension.  dQ per
+// row and dK/dV per key from P = exp(x - L_new) and Delta (page "Attention
+// Sink, Learnable Sink and dsink", sections 7-8), visiting only the tiles the
+// plan lists.
 #include "internal.h"
 
 namespace sk {
@@ -31,76 +30,6 @@ struct SimtArgs {
   float* lse_orig;   // or nullptr
 };
 
-template <int D>
-__global__ void __launch_bounds__(kWarps * 32) fwd_simt_kernel(SimtArgs a, float* out, float* lse,
-                                                               float* sink_s) {
-  constexpr int E = D / 32;
-  const PlanHdr* h = reinterpret_cast<const PlanHdr*>(a.plan);
-  const int G = a.Hq / a.Hkv;
-  const int heads_per_item = h->kh_slots == 1 ? a.Hq : G;
-  const int rank = blockIdx.x / heads_per_item, hh = blockIdx.x % heads_per_item;
-  if (rank >= h->n_fwd_items) return;
-  const int idx = a.plan[h->off_fwd_order + rank];
-  const TileItem it = reinterpret_cast<const TileItem*>(a.plan + h->off_fwd_items)[idx];
-  const int head = it.kvh < 0 ? hh : it.kvh * G + hh;
-  const int kvh = head / G;
-  const int* ent = a.plan + h->off_fwd_entries + it.entry_off;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float a2 = a.sink ? a.sink[head] * kLog2e : -INFINITY;
-
-  for (int r = warp; r < it.tile_len; r += kWarps) {
-    const int qi = it.tile_start + r;
-    const long long row = (long long)(it.seq_start + qi) * a.Hq + head;
-    float qv[E], acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      qv[e] = a.q[row * D + lane + 32 * e] * a.scale_log2;
-      acc[e] = 0.f;
-    }
-    float m = -INFINITY, l = 0.f;
-    for (int t = 0; t < it.entry_len; ++t) {
-      const int kt = ent[t] >> 1, partial = ent[t] & 1;
-      const int k0 = kt * a.tile;
-      const int kend = min(k0 + a.tile, it.seq_len);
-      for (int kj = k0; kj < kend; ++kj) {
-        if (partial && !visible_elem(qi, kj, it.seq_len, a.causal, a.n_sink, a.window)) continue;
-        const long long krow = (long long)(it.seq_start + kj) * a.Hkv + kvh;
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) s += qv[e] * a.k[krow * D + lane + 32 * e];
-        s = warp_sum(s);
-        const float mn = fmaxf(m, s);
-        const float corr = exp2f(m - mn);  // m = -inf on the first key: 0
-        const float p = exp2f(s - mn);
-        l = l * corr + p;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = acc[e] * corr + p * a.v[krow * D + lane + 32 * e];
-        m = mn;
-      }
-    }
-    // sink epilogue in the log2 domain
-    const float mt = fmaxf(m, a2);
-    float o_scale = 0.f, lse_v = -INFINITY, ss = 0.f;
-    if (mt != -INFINITY) {
-      const float fr = (m == -INFINITY) ? 0.f : exp2f(m - mt);
-      const float lr = l * fr;
-      const float den = lr + (a.sink ? exp2f(a2 - mt) : 0.f);
-      o_scale = fr / den;
-      lse_v = (mt + log2f(den)) * kLn2;
-      ss = lr / den;
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) out[row * D + lane + 32 * e] = acc[e] * o_scale;
-    if (lane == 0) {
-      lse[row] = lse_v;
-      if (sink_s) sink_s[row] = ss;
-      // the raw LSE over the visible keys (before the sink joins)
-      if (a.lse_orig) a.lse_orig[row] = (m != -INFINITY && l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
-    }
-  }
-}
-
-// dQ: one warp per (row, head).
 template <int D>
 __global__ void __launch_bounds__(kWarps * 32) dq_simt_kernel(SimtArgs a, const float* dout,
                                                               const float* lse,
@@ -241,20 +170,6 @@ SimtArgs make_args(const AttnProblem& p) {
 }
 
 }  // namespace
-
-int launch_fwd_simt(const AttnProblem& p, void* out, float* lse, float* sink_s,
-                    cudaStream_t stream) {
-  const SimtArgs a = make_args(p);
-  const int G = p.Hq / p.Hkv;
-  const int per_item = p.ps.kh_slots == 1 ? p.Hq : G;
-  const long long grid = (long long)p.ps.cap_items * per_item;
-  if (grid <= 0 || grid > 0x7fffffffLL) return SINKATTN_ERR_INVALID_ARG;
-  if (p.D == 64)
-    fwd_simt_kernel<64><<<(unsigned)grid, kWarps * 32, 0, stream>>>(a, static_cast<float*>(out), lse, sink_s);
-  else
-    fwd_simt_kernel<128><<<(unsigned)grid, kWarps * 32, 0, stream>>>(a, static_cast<float*>(out), lse, sink_s);
-  return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
-}
 
 int launch_bwd_simt(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   const SimtArgs a = make_args(p);
