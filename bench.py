@@ -41,6 +41,9 @@ from learnable_sink_b200 import workloads as W  # noqa: E402
 
 METRIC = "sink-attn fwd+bwd TFLOP/s & decode KV GB/s on 1 B200, % of roofline"
 L2_BYTES = 126 * 1024 * 1024
+# a device-side wait (about 0.5 ms at 1.9 GHz) enqueued before a short timed
+# call, long enough for the host to issue that call behind it
+HOST_COVER_CYCLES = 1_000_000
 # launches of this library per step: plan 12, forward 1, backward 6
 # (preprocess, dsink reduce, split-tile zero/finish, tensor-core kernel, dQ
 # convert), decode 2
@@ -323,6 +326,7 @@ def measure_decode_kernel(S, decode_step, flush, flush_rd, reps=20):
     for _ in range(reps):
         flush.zero_()
         flush_rd.sum()
+        torch.cuda._sleep(HOST_COVER_CYCLES)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -368,6 +372,7 @@ def measure_fp8_decode(S, dec, dev, flush, flush_rd, reps=20):
         for _ in range(reps):
             flush.zero_()
             flush_rd.sum()
+            torch.cuda._sleep(HOST_COVER_CYCLES)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -389,8 +394,9 @@ def measure_fp8_decode(S, dec, dev, flush, flush_rd, reps=20):
 
 def measure_gates(S, q, k, lse, sink_s, mask, scale, flush, flush_rd, hbm_gbs, reps=10):
     """Gate rows on the prefill's tensors: the sink-free model's gate (reads Q
-    once; Q is larger than L2) and the head importance (reads sink_s once;
-    L2 flushed before each call).  CUDA events around each call."""
+    once) and the head importance (reads sink_s once).  L2 is flushed before
+    each call, then the device is kept busy (torch.cuda._sleep) while the host
+    issues the call, so the CUDA events around it see no host issue gap."""
     T, Hq, D = q.shape
     gate = torch.empty(T, Hq, dtype=torch.float32, device=q.device)
     imp = torch.empty(Hq, dtype=torch.float32, device=q.device)
@@ -398,19 +404,18 @@ def measure_gates(S, q, k, lse, sink_s, mask, scale, flush, flush_rd, hbm_gbs, r
                       dtype=torch.uint8, device=q.device)
     n_seq = mask.cu_seqlens.numel() - 1
     res = {}
-    for name, call, nbytes, cold in (
+    for name, call, nbytes in (
             ("gate_vanilla", lambda: S.gate_vanilla(q, k, lse, mask, scale=scale, gate=gate),
-             q.numel() * q.element_size() + 8 * T * Hq + n_seq * k.shape[1] * D * k.element_size(),
-             False),
+             q.numel() * q.element_size() + 8 * T * Hq + n_seq * k.shape[1] * D * k.element_size()),
             ("gate_importance", lambda: S.gate_importance(sink_s, workspace=iws, imp=imp),
-             4 * T * Hq, True)):
+             4 * T * Hq)):
         for _ in range(3):
             call()
         ts = []
         for _ in range(reps):
-            if cold:
-                flush.zero_()
-                flush_rd.sum()
+            flush.zero_()
+            flush_rd.sum()
+            torch.cuda._sleep(HOST_COVER_CYCLES)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -446,6 +451,16 @@ def run_profile_workload(args, dev):
             plan.rebuild()
             S.fwd(q, k, v, sink, mask, plan, scale=inp.scale, out=out, lse=lse, sink_s=ss)
             S.bwd(q, k, v, out, dout, lse, sink, mask, plan, scale=inp.scale, workspace=ws)
+    elif args.profile_workload == "gate":
+        inp = W.prefill()
+        T, Hq, Hkv, D = inp.shape
+        q, k = inp.q.to(dev), inp.k.to(dev)
+        mask = S.Mask.from_spec(inp.mask, dev)
+        lse = torch.randn(T, Hq, dtype=torch.float32, device=dev).abs_().add_(4.0)
+        gate = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+
+        def step():
+            S.gate_vanilla(q, k, lse, mask, scale=inp.scale, gate=gate)
     else:  # fp8 decode
         dec = W.decode()
         cache = [t.to(dev) for t in W.fp8_window_cache(dec, seed=W.SEED_BASE + 501)]
@@ -576,6 +591,10 @@ def run_ours(args, world, rank, local):
     region_ms = max_over_ranks(r0.elapsed_time(r1), world)
     prefill_ms = max_over_ranks(total("p0", "p1"), world)
     decode_ms = max_over_ranks(total("d0", "d1"), world)
+    # the rest of the step: the L2 flush between prefill and decode, and the
+    # device's idle time from one step's decode to the next step's prefill
+    flush_only_ms = total("p1", "d0") / K
+    between_ms = sum(evs["d1"][i].elapsed_time(evs["p0"][i + 1]) for i in range(K - 1)) / max(1, K - 1)
     kf_ms = total("kf0", "kf1") / K
     kb_ms = total("kb0", "kb1") / K
     # the streaming kernel alone (its own events; the step loop above times
@@ -710,10 +729,13 @@ def run_ours(args, world, rank, local):
         "decode_fp8_window": fp8,
         "step_breakdown_ms": {
             "prefill": prefill_ms / K, "decode_call": decode_ms / K,
-            "l2_flush_and_gaps": flush_ms,
+            "l2_flush_and_gaps": flush_ms, "l2_flush": flush_only_ms,
+            "decode_to_next_prefill": between_ms,
             "host_issue_per_step": (host_t[1] - host_t[0]) * 1e3 / K,
             "note": "device time per step; l2_flush_and_gaps = step - prefill - decode "
-                    "(the two flush kernels between prefill and decode, and any idle time)"},
+                    "(the two flush kernels between prefill and decode, and any idle time); "
+                    "l2_flush = prefill end to decode start; decode_to_next_prefill = decode "
+                    "end to the next step's prefill start"},
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2,
@@ -800,7 +822,7 @@ def main():
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps of the prefill and decode stages for a profiler "
                          "(no timing, no JSON line)")
-    ap.add_argument("--profile-workload", choices=["band", "varlen", "fp8"], default=None,
+    ap.add_argument("--profile-workload", choices=["band", "varlen", "fp8", "gate"], default=None,
                     help="like --profile, for one other workload's kernels")
     ap.add_argument("--no-configs", dest="configs", action="store_false",
                     help="skip the band / varlen block-sparse measurements")

@@ -420,7 +420,8 @@ int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, fl
  * other launches of the call stay outside the events).
  *   which   SINKATTN_KERNEL_FWD (the attention forward kernel),
  *           SINKATTN_KERNEL_BWD (the dK/dV/dQ kernel of sinkattn_bwd),
- *           SINKATTN_KERNEL_DECODE (the split-KV streaming kernel).
+ *           SINKATTN_KERNEL_DECODE (the split-KV streaming kernel),
+ *           SINKATTN_KERNEL_GATE (the kernel of sinkattn_gate_vanilla).
  *   start, stop  cudaEvent_t handles created by the caller, or both NULL to
  *           stop recording.  They are recorded by every later call of that
  *           kind on the calling host thread's current device until changed.
@@ -428,6 +429,7 @@ int sinkattn_decode_noalloc(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, fl
 #define SINKATTN_KERNEL_FWD 0
 #define SINKATTN_KERNEL_BWD 1
 #define SINKATTN_KERNEL_DECODE 2
+#define SINKATTN_KERNEL_GATE 3
 int sinkattn_set_kernel_events(int which, void *start, void *stop);
 
 /* ---- failure-detection self-test ---------------------------------------------

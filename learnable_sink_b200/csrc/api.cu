@@ -47,7 +47,7 @@ bool device_is_sm100() {
   return g_is_sm100[dev] == 1;
 }
 
-thread_local KernelEvents g_events[3];
+thread_local KernelEvents g_events[4];
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -112,7 +112,7 @@ BwdLayout bwd_layout(int dt, int T_tot, int Hq, int Hkv, int D) {
 }  // namespace
 
 KernelEvents kernel_events(int which) {
-  return (which >= 0 && which < 3) ? g_events[which] : KernelEvents{};
+  return (which >= 0 && which < 4) ? g_events[which] : KernelEvents{};
 }
 
 }  // namespace sk
@@ -438,7 +438,7 @@ int sinkattn_decode_fp8(int B, int Hq, int Hkv, int D, float scale, const void* 
 }
 
 int sinkattn_set_kernel_events(int which, void* start, void* stop) {
-  if (which < 0 || which > 2 || ((start == nullptr) != (stop == nullptr)))
+  if (which < 0 || which > 3 || ((start == nullptr) != (stop == nullptr)))
     return SINKATTN_ERR_INVALID_ARG;
   g_events[which].start = static_cast<cudaEvent_t>(start);
   g_events[which].stop = static_cast<cudaEvent_t>(stop);

@@ -56,7 +56,6 @@ struct FwdCfg {
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "not enough shared memory for a two-stage ring");
   static constexpr int MIN_BLOCKS = 1;
-
   // With two softmax warpgroups and one CTA per SM, registers are moved to the
   // softmax warpgroups: the producer and MMA warps then share a warpgroup with
   // two idle warps (setmaxnreg works on whole warpgroups), 12 warps in all,

@@ -201,6 +201,7 @@ int launch_gate_vanilla(const GateVanillaArgs& a, int dt, int D, int max_seqlen,
   const dim3 grid((max_seqlen + kGvRows - 1) / kGvRows, a.n_seq);
   const size_t k0_bytes = (size_t)a.Hkv * D * (dt == SINKATTN_BF16 ? 2 : 4);
   const size_t smem = k0_bytes <= (size_t)kGvK0Smem ? k0_bytes : 0;
+  record_start(SINKATTN_KERNEL_GATE, stream);
   if (dt == SINKATTN_BF16) {
     if (D == 64) gate_vanilla_kernel<__nv_bfloat16, 64><<<grid, 256, smem, stream>>>(a);
     else gate_vanilla_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(a);
@@ -208,6 +209,7 @@ int launch_gate_vanilla(const GateVanillaArgs& a, int dt, int D, int max_seqlen,
     if (D == 64) gate_vanilla_kernel<float, 64><<<grid, 256, smem, stream>>>(a);
     else gate_vanilla_kernel<float, 128><<<grid, 256, smem, stream>>>(a);
   }
+  record_stop(SINKATTN_KERNEL_GATE, stream);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

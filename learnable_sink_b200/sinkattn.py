@@ -484,7 +484,7 @@ def cache_fill(k, v, cu_seqlens, k_cache, v_cache, n_sink: int, window: int,
         _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens_out), _stream(stream)))
 
 
-KERNEL_FWD, KERNEL_BWD, KERNEL_DECODE = 0, 1, 2
+KERNEL_FWD, KERNEL_BWD, KERNEL_DECODE, KERNEL_GATE = 0, 1, 2, 3
 
 
 def set_kernel_events(which: int, start=None, stop=None) -> None:
