@@ -27,113 +27,125 @@ namespace sk {
 namespace {
 
 constexpr int kPreThreads = 256;
-constexpr int kPreTokens = 16;   // tokens per CTA
-constexpr int kRows = 8;         // rows in flight per warp
+constexpr int kPreTokens = 4;    // tokens per CTA
+constexpr int kPreSlots = 8;     // rows per lane group in flight (each of O and dO)
 constexpr int kMaxHeads = 256;
+constexpr int kRedThreads = 256;
 
-// D/32 elements of one row held by a lane, converted to fp32.
-template <typename T, int D>
-struct RowFrag {
-  static constexpr int E = D / 32;
-  float v[E];
-  __device__ __forceinline__ void load(const T* row, int lane) {
-    if constexpr (sizeof(T) == 2) {
-      const __nv_bfloat16* p = reinterpret_cast<const __nv_bfloat16*>(row) + lane * E;
-      if constexpr (E == 4) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-      } else {
-        const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(p));
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
-        v[0] = a.x; v[1] = a.y;
-      }
-    } else {
+// <a, b> over one 16-byte chunk of each row.
+template <typename T>
+__device__ __forceinline__ float chunk_dot(const uint4& a, const uint4& b) {
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+    float s = 0.f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = __ldg(row + lane * E + e);
+    for (int i = 0; i < 4; ++i) {
+      const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+      s = fmaf(u.x, v.x, s);
+      s = fmaf(u.y, v.y, s);
     }
+    return s;
+  } else {
+    float s = __uint_as_float(a.x) * __uint_as_float(b.x);
+    s = fmaf(__uint_as_float(a.y), __uint_as_float(b.y), s);
+    s = fmaf(__uint_as_float(a.z), __uint_as_float(b.z), s);
+    return fmaf(__uint_as_float(a.w), __uint_as_float(b.w), s);
   }
-};
+}
 
-// One warp owns one head of the CTA's tokens, kRows rows at a time: all loads
-// of a group are issued before any reduction, so each lane keeps 2 kRows loads
-// in flight.  Delta and LSE2 of consecutive tokens land in consecutive words
-// of the head-major arrays; the warp also writes the CTA's dsink partial for
-// its head (fixed order, so dsink is bitwise deterministic).
+// The CTA's rows (token, head) are contiguous in memory: row r of the CTA is
+// token t0 + r / Hq, head r % Hq.  A row is L = D sizeof(T) / 16 chunks of 16
+// bytes, so one warp load instruction covers 32 / L rows (one chunk a lane);
+// a warp phase issues kPreSlots such loads of O and of dO before any
+// arithmetic (8 KB in flight per warp), reduces each row over its L lanes,
+// and lane (row group, i < kPreSlots) finishes the row of slot i, whose LSE
+// (and upstream gate gradient) it loaded beside the chunks.
 template <typename T, int D>
 __global__ void __launch_bounds__(kPreThreads) preprocess_kernel(
     const T* out, const T* dout, const float* lse, const float* sink, const float* dss,
     float* delta, float* lse2, float* part, int T_tot, int Hq) {
+  constexpr int L = D * (int)sizeof(T) / 16;  // 8, 16 or 32
+  static_assert(L >= kPreSlots && L <= 32, "row layout");
+  constexpr int RPI = 32 / L;                 // rows per load instruction
+  constexpr int RPP = RPI * kPreSlots;        // rows per warp phase
+  __shared__ float contrib_s[kPreTokens * kMaxHeads];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / L, li = lane % L;
   const int t0 = blockIdx.x * kPreTokens;
-  for (int h = warp; h < Hq; h += kPreThreads / 32) {
-    const float a = sink ? __ldg(sink + h) : 0.f;
-    float dsum = 0.f;
+  const int nt = min(kPreTokens, T_tot - t0);
+  const int R = nt * Hq;
+  const long long row0 = (long long)t0 * Hq;
+  const uint4* O = reinterpret_cast<const uint4*>(out) + row0 * L;
+  const uint4* dO = reinterpret_cast<const uint4*>(dout) + row0 * L;
+  for (int ph = warp * RPP; ph < R; ph += (kPreThreads / 32) * RPP) {
+    uint4 o[kPreSlots], d[kPreSlots];
 #pragma unroll
-    for (int g = 0; g < kPreTokens; g += kRows) {
-      RowFrag<T, D> o[kRows], d[kRows];
+    for (int s = 0; s < kPreSlots; ++s) {
+      const int r = min(ph + s * RPI + sub, R - 1);
+      o[s] = __ldg(O + (long long)r * L + li);
+      d[s] = __ldg(dO + (long long)r * L + li);
+    }
+    // the row this lane finishes: slot li of its row group
+    const int my_r = ph + li * RPI + sub;
+    const bool mine_ok = li < kPreSlots && my_r < R;
+    const int rr = min(my_r, R - 1);
+    const float l = __ldg(lse + row0 + rr);
+    const float g = dss ? __ldg(dss + row0 + rr) : 0.f;
+    float acc[kPreSlots];
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        const int t = min(t0 + g + r, T_tot - 1);
-        const long long row = ((long long)t * Hq + h) * D;
-        o[r].load(out + row, lane);
-        d[r].load(dout + row, lane);
-      }
-      float acc[kRows];
+    for (int s = 0; s < kPreSlots; ++s) acc[s] = chunk_dot<T>(o[s], d[s]);
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        acc[r] = 0.f;
+    for (int off = L / 2; off > 0; off >>= 1)
 #pragma unroll
-        for (int e = 0; e < RowFrag<T, D>::E; ++e) acc[r] += o[r].v[e] * d[r].v[e];
-      }
+      for (int s = 0; s < kPreSlots; ++s) acc[s] += __shfl_xor_sync(0xffffffffu, acc[s], off);
+    float dot = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-        for (int r = 0; r < kRows; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
-      // lane r (< kRows) writes token t0 + g + r
-      float mine = 0.f;
-#pragma unroll
-      for (int r = 0; r < kRows; ++r) mine = (lane == r) ? acc[r] : mine;
-      const int t = t0 + g + lane;
-      float contrib = 0.f;
-      if (lane < kRows && t < T_tot) {
-        const float l = __ldg(lse + (long long)t * Hq + h);
-        float dl = mine;
-        if (sink) {
-          const float ps = __expf(a - l);  // p_sink
-          if (dss) {
-            const float g = __ldg(dss + (long long)t * Hq + h);
-            contrib = -ps * (mine + g * (1.f - ps));
-            dl = mine - g * ps;
-          } else {
-            contrib = -mine * ps;  // -Delta * p_sink
-          }
+    for (int s = 0; s < kPreSlots; ++s) dot = (li == s) ? acc[s] : dot;
+    if (mine_ok) {
+      const int t = t0 + my_r / Hq, h = my_r % Hq;
+      float dl = dot, contrib = 0.f;
+      if (sink) {
+        const float ps = __expf(__ldg(sink + h) - l);  // p_sink
+        if (dss) {
+          contrib = -ps * (dot + g * (1.f - ps));
+          dl = dot - g * ps;
+        } else {
+          contrib = -dot * ps;  // -Delta * p_sink
         }
-        delta[(long long)h * T_tot + t] = dl;
-        lse2[(long long)h * T_tot + t] = (l == -INFINITY) ? INFINITY : l * kLog2e;
       }
-      dsum += contrib;
+      delta[(long long)h * T_tot + t] = dl;
+      lse2[(long long)h * T_tot + t] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+      contrib_s[my_r] = contrib;
     }
-    if (sink) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
-      if (lane == 0) part[(long long)blockIdx.x * Hq + h] = dsum;
-    }
+  }
+  if (!sink) return;  // uniform over the CTA
+  __syncthreads();
+  // the CTA's partial of head h: its tokens in order; head-major partials
+  for (int h = threadIdx.x; h < Hq; h += kPreThreads) {
+    float s = 0.f;
+    for (int tt = 0; tt < nt; ++tt) s += contrib_s[tt * Hq + h];
+    part[(long long)h * gridDim.x + blockIdx.x] = s;
   }
 }
 
-// dsink[h] = sum of the per-CTA partials: one warp per head, lanes stride
-// over the partials in a fixed order, then a fixed butterfly.
-__global__ void dsink_reduce_kernel(const float* part, int n_blocks, int Hq, float* dsink) {
-  const int h = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (h >= Hq) return;
+// dsink[h] = sum of head h's partials [n_blocks]: one CTA per head, each
+// thread sums a fixed strided subset in order, then a fixed tree.
+__global__ void __launch_bounds__(kRedThreads) dsink_reduce_kernel(const float* part, int n_blocks,
+                                                                  float* dsink) {
+  __shared__ float red[kRedThreads];
+  const int h = blockIdx.x;
+  const float* p = part + (long long)h * n_blocks;
   float s = 0.f;
-  for (int b = lane; b < n_blocks; b += 32) s += part[(long long)b * Hq + h];
+  for (int b = threadIdx.x; b < n_blocks; b += kRedThreads) s += __ldg(p + b);
+  red[threadIdx.x] = s;
+  __syncthreads();
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) dsink[h] = s;
+  for (int w = kRedThreads / 2; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) dsink[h] = red[0];
 }
 
 }  // namespace
@@ -159,7 +171,7 @@ int launch_bwd_preprocess(const AttnProblem& p, const BwdBuffers& b, cudaStream_
       preprocess_kernel<float, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   }
   if (p.sink && b.dsink)
-    dsink_reduce_kernel<<<(p.Hq + 3) / 4, 128, 0, stream>>>(b.dsink_part, nb, p.Hq, b.dsink);
+    dsink_reduce_kernel<<<p.Hq, kRedThreads, 0, stream>>>(b.dsink_part, nb, b.dsink);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

@@ -669,41 +669,77 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
 // Key tiles whose reverse list was split into several work units: zero their
 // fp32 dK/dV accumulator rows before the backward kernel, and round them to
-// bf16 (dK scaled by alpha) after it.  One CTA per backward item; unsplit
-// items return at once.
-__global__ void split_tiles_kernel(const int* plan, float* dk_acc, float* dv_acc,
-                                   __nv_bfloat16* dk, __nv_bfloat16* dv, int Hkv, int D,
-                                   float alpha, int finish) {
-  // blockIdx.x = backward item, blockIdx.y = row of its key tile
+// bf16 (dK scaled by alpha) after it.  CTA (item, chunk of kSplitRows rows of
+// its key tile); unsplit items return at once.  A thread moves kSplitVec
+// float4 of each accumulator, all loads before the stores.
+constexpr int kSplitRows = 16;
+constexpr int kSplitVec = 4;
+__global__ void __launch_bounds__(256) split_tiles_kernel(const int* plan, float* dk_acc,
+                                                          float* dv_acc, __nv_bfloat16* dk,
+                                                          __nv_bfloat16* dv, int Hkv, int D,
+                                                          float alpha, int finish) {
   const PlanHdr* h = reinterpret_cast<const PlanHdr*>(plan);
   if ((int)blockIdx.x >= h->cap_items) return;
   const TileItem it = reinterpret_cast<const TileItem*>(plan + h->off_bwd_items)[blockIdx.x];
-  if (it.entry_len < 0 || bwd_units_of(it.entry_len) <= 1 || (int)blockIdx.y >= it.tile_len) return;
+  const int row0 = blockIdx.y * kSplitRows;
+  if (it.entry_len < 0 || bwd_units_of(it.entry_len) <= 1 || row0 >= it.tile_len) return;
   const int kv0 = it.kvh >= 0 ? it.kvh : 0, kv1 = it.kvh >= 0 ? it.kvh + 1 : Hkv;
-  const long long base = ((long long)(it.seq_start + it.tile_start + blockIdx.y) * Hkv + kv0) * D;
-  const int n4 = (kv1 - kv0) * D / 4;
-  float4* ka = reinterpret_cast<float4*>(dk_acc + base);
-  float4* va = reinterpret_cast<float4*>(dv_acc + base);
-  for (int e = threadIdx.x; e < n4; e += blockDim.x) {
+  const int n4 = (kv1 - kv0) * D / 4;  // float4 per token row of the item
+  const long long tok0 = it.seq_start + it.tile_start + row0;
+  const int total = min(kSplitRows, it.tile_len - row0) * n4;
+  for (int e0 = threadIdx.x; e0 < total; e0 += 256 * kSplitVec) {
+    long long off[kSplitVec];
+#pragma unroll
+    for (int u = 0; u < kSplitVec; ++u) {
+      const int e = min(e0 + u * 256, total - 1);
+      const int row = e / n4;
+      off[u] = ((tok0 + row) * Hkv + kv0) * D / 4 + (e - row * n4);
+    }
     if (finish) {
-      const float4 x = ka[e], y = va[e];
-      reinterpret_cast<uint2*>(dk + base)[e] =
-          make_uint2(pack_bf16x2(x.x * alpha, x.y * alpha), pack_bf16x2(x.z * alpha, x.w * alpha));
-      reinterpret_cast<uint2*>(dv + base)[e] =
-          make_uint2(pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
+      float4 x[kSplitVec], y[kSplitVec];
+#pragma unroll
+      for (int u = 0; u < kSplitVec; ++u) {
+        x[u] = __ldcs(reinterpret_cast<const float4*>(dk_acc) + off[u]);
+        y[u] = __ldcs(reinterpret_cast<const float4*>(dv_acc) + off[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kSplitVec; ++u) {
+        if (e0 + u * 256 >= total) break;
+        reinterpret_cast<uint2*>(dk)[off[u]] = make_uint2(
+            pack_bf16x2(x[u].x * alpha, x[u].y * alpha), pack_bf16x2(x[u].z * alpha, x[u].w * alpha));
+        reinterpret_cast<uint2*>(dv)[off[u]] =
+            make_uint2(pack_bf16x2(y[u].x, y[u].y), pack_bf16x2(y[u].z, y[u].w));
+      }
     } else {
-      ka[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-      va[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kSplitVec; ++u) {
+        if (e0 + u * 256 >= total) break;
+        reinterpret_cast<float4*>(dk_acc)[off[u]] = make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(dv_acc)[off[u]] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
 }
 
-// dQ = alpha * accumulated fp32, rounded to bf16.
-__global__ void dq_convert_kernel(const float4* acc, uint2* dq, long long n4, float alpha) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n4) return;
-  const float4 v = acc[i];
-  dq[i] = make_uint2(pack_bf16x2(v.x * alpha, v.y * alpha), pack_bf16x2(v.z * alpha, v.w * alpha));
+// dQ = alpha * accumulated fp32, rounded to bf16: kDqVec float4 a thread, all
+// loads issued before the stores.
+constexpr int kDqVec = 4;
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float4* acc, uint2* dq, long long n4,
+                                                         float alpha) {
+  const long long i0 = (long long)blockIdx.x * (256 * kDqVec) + threadIdx.x;
+  float4 v[kDqVec];
+#pragma unroll
+  for (int u = 0; u < kDqVec; ++u) {
+    const long long i = i0 + u * 256;
+    v[u] = i < n4 ? __ldcs(acc + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int u = 0; u < kDqVec; ++u) {
+    const long long i = i0 + u * 256;
+    if (i < n4)
+      dq[i] = make_uint2(pack_bf16x2(v[u].x * alpha, v[u].y * alpha),
+                         pack_bf16x2(v[u].z * alpha, v[u].w * alpha));
+  }
 }
 
 template <class C>
@@ -750,7 +786,7 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != C::LAUNCH_REGS)
       return SINKATTN_ERR_UNSUPPORTED;
   }
-  const dim3 split_grid(p.ps.cap_items, C::KT);
+  const dim3 split_grid(p.ps.cap_items, (C::KT + kSplitRows - 1) / kSplitRows);
   split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
                                                      p.Hkv, D, p.scale, 0);
   record_start(SINKATTN_KERNEL_BWD, stream);
@@ -759,7 +795,7 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
                                                      p.Hkv, D, p.scale, 1);
   const long long n4 = (long long)p.T_tot * p.Hq * D / 4;
-  dq_convert_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(
+  dq_convert_kernel<<<(unsigned)((n4 + 256 * kDqVec - 1) / (256 * kDqVec)), 256, 0, stream>>>(
       reinterpret_cast<const float4*>(b.dq_accum), reinterpret_cast<uint2*>(b.dq), n4, p.scale);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }

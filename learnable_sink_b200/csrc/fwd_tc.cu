@@ -59,9 +59,10 @@ struct FwdCfg {
   // With two softmax warpgroups and one CTA per SM, registers are moved to the
   // softmax warpgroups: the producer and MMA warps then share a warpgroup with
   // two idle warps (setmaxnreg works on whole warpgroups), 12 warps in all,
-  // 168 registers per thread at launch and 256 x 224 + 128 x 56 = 384 x 168.
+  // 168 registers per thread at launch and 256 x 208 + 128 x 80 = 384 x 168
+  // (with 56 the producer and MMA warps spill; 208 still holds a softmax row).
   static constexpr bool REBALANCE = (NQT == 2 && MIN_BLOCKS == 1);
-  static constexpr int SOFTMAX_REGS = 224, AUX_REGS = 56;
+  static constexpr int SOFTMAX_REGS = 208, AUX_REGS = 80;
   static constexpr int THREADS = (4 * NQT + (REBALANCE ? 4 : 2)) * 32;
   static constexpr int PRODUCER_WARP = 4 * NQT;
   static constexpr int MMA_WARP = 4 * NQT + 1;

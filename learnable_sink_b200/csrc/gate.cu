@@ -78,11 +78,15 @@ __global__ void gate_reduce_kernel(const double* part, int n_blocks, int Hq, int
 // that does not see k_0 gets 1, a row that sees no key (L = -inf) gets 0.
 // HBM-bound (reads Q once).  A warp streams one token's contiguous Q row
 // [Hq, D] as 16-byte chunks, kGvInFlight per lane in flight; the CPH chunks
-// of a head row sit in CPH adjacent lanes, which reduce its dot product.
-// CTA = kGvRows tokens of one sequence; the sequence's k_0 rows [Hkv, D] are
-// staged once in shared memory when they fit kGvK0Smem bytes (else read
-// through L1), so the loop's only global loads are Q's.
-constexpr int kGvRows = 64;
+// of a head row sit in CPH adjacent lanes.  Their partial dot products are
+// summed by a shuffle reduce-scatter, after which every lane holds whole
+// dot products of max(1, kGvInFlight / CPH) heads (each head once per warp,
+// or twice when CPH = 32) and finishes those heads alone: one expm1 per head,
+// not one per lane and chunk.  CTA = kGvRows tokens of one sequence; the
+// sequence's k_0 rows [Hkv, D] are staged once in shared memory when they fit
+// kGvK0Smem bytes (else read through L1), so the loop's only global loads
+// are Q's and the LSE.
+constexpr int kGvRows = 16;
 constexpr int kGvInFlight = 16;
 constexpr int kGvK0Smem = 32 * 1024;
 
@@ -105,9 +109,48 @@ __device__ __forceinline__ float dot16(const uint4& a, const uint4& b) {
   }
 }
 
+// Reduce-scatter over lane masks M, M/2, ..., 1 of N values a lane: while
+// N > 1 a step sends one half of the values to the partner lane (lane ^ M),
+// keeps the other half and adds what arrives; once N = 1 a step is a plain
+// butterfly add.  Afterwards v[0 .. N_end) are sums over the lane group of
+// the values u0 .. u0 + N_end - 1, where u0 adds H for every halving step
+// whose mask bit is set in the lane.
+template <int M, int N>
+struct ReduceScatter {
+  template <int U>
+  __device__ __forceinline__ static void run(float (&v)[U], int lane) {
+    if constexpr (M >= 1) {
+      if constexpr (N > 1) {
+        constexpr int H = N / 2;
+        const bool up = (lane & M) != 0;
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+          const float send = up ? v[k] : v[k + H];
+          const float keep = up ? v[k + H] : v[k];
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+        }
+        ReduceScatter<M / 2, H>::run(v, lane);
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], M);
+        ReduceScatter<M / 2, 1>::run(v, lane);
+      }
+    }
+  }
+  __device__ __forceinline__ static int first(int lane) {
+    if constexpr (M >= 1 && N > 1)
+      return ((lane & M) ? N / 2 : 0) + ReduceScatter<M / 2, N / 2>::first(lane);
+    else
+      return 0;
+  }
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
   constexpr int CPH = D * (int)sizeof(T) / 16;  // 16-byte chunks per head row: 8, 16 or 32
+  constexpr int U = kGvInFlight;
+  constexpr int NV = U / CPH > 0 ? U / CPH : 1;   // heads a lane finishes per batch
+  constexpr int DUP = CPH / U > 0 ? CPH / U : 1;  // lanes holding the same head
+  using RS = ReduceScatter<CPH / 2, U>;
   const int s = blockIdx.y;
   const int start = __ldg(a.cu + s), len = __ldg(a.cu + s + 1) - start;
   const int i0 = blockIdx.x * kGvRows;
@@ -140,55 +183,56 @@ __global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
     for (int j = threadIdx.x; j < a.Hkv * CPH; j += blockDim.x) k0s[j] = __ldg(k0 + j);
     __syncthreads();
   }
+  // this lane's heads after the reduce-scatter: values u0 .. u0 + NV - 1 of
+  // lane group g; the lane writes them when it is the group's first copy
+  const int u0 = RS::first(lane), g = lane / CPH;
+  const bool writer = (lane % DUP) == 0;
   for (int i = i0 + warp; i < min(len, i0 + kGvRows); i += 8) {
     const long long t = start + i;
     const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(a.q) + t * a.Hq * D);
     // is k_0 visible to query i (sequence-local)?  causal: always (0 <= i)
     const bool vis_band = a.window == 0 || a.n_sink > 0 || i < a.window;
-    for (int c0 = 0; c0 < n16; c0 += 32 * kGvInFlight) {
-      // the batch covers heads hb0 .. hb0 + 32 kGvInFlight / CPH - 1 (at most
-      // 32): lane j loads head hb0 + j's LSE together with the Q chunks
-      const int hb0 = c0 / CPH;
-      const int hj = min(hb0 + lane, a.Hq - 1);
-      const float lse_b = __ldg(a.lse + t * a.Hq + hj);
-      uint4 qv[kGvInFlight], kv[kGvInFlight];
+    for (int c0 = 0; c0 < n16; c0 += 32 * U) {
+      float lse_v[NV];
+      int hv[NV];
 #pragma unroll
-      for (int u = 0; u < kGvInFlight; ++u) {
-        const int c = min(c0 + u * 32 + lane, n16 - 1);
-        const int h = c / CPH;
-        qv[u] = __ldg(qrow + c);
-        const int kc = (h / G) * CPH + (c - h * CPH);
-        kv[u] = k0_in_smem ? k0s[kc] : __ldg(k0 + kc);
+      for (int k = 0; k < NV; ++k) {
+        hv[k] = (c0 + (u0 + k) * 32) / CPH + g;
+        lse_v[k] = __ldg(a.lse + t * a.Hq + min(hv[k], a.Hq - 1));
       }
-      float dot[kGvInFlight];
+      float dot[U];
+      {
+        uint4 qv[U];
 #pragma unroll
-      for (int u = 0; u < kGvInFlight; ++u) dot[u] = dot16<T>(qv[u], kv[u]);
+        for (int u = 0; u < U; ++u) qv[u] = __ldg(qrow + min(c0 + u * 32 + lane, n16 - 1));
 #pragma unroll
-      for (int o = CPH / 2; o > 0; o >>= 1)
-#pragma unroll
-        for (int u = 0; u < kGvInFlight; ++u) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
-      // the first lane of each head's group writes that head
-#pragma unroll
-      for (int u = 0; u < kGvInFlight; ++u) {
-        const int c = c0 + u * 32 + lane;
-        const float l = __shfl_sync(0xffffffffu, lse_b, (min(c, n16 - 1) / CPH - hb0) & 31);
-        if (c < n16 && (lane % CPH) == 0) {
+        for (int u = 0; u < U; ++u) {
+          const int c = min(c0 + u * 32 + lane, n16 - 1);
           const int h = c / CPH;
-          bool vis = vis_band;
-          if (a.bi && vis) {
-            const int qb = qb_base + i / a.block_q;
-            vis = false;
-            if (qb < a.n_qblk) {
-              const int32_t* lst = a.bi + ((long long)(h / G) * a.n_qblk + qb) * a.max_blocks;
-              for (int e = 0; e < a.max_blocks; ++e) vis |= __ldg(lst + e) == 0;
-            }
-          }
-          float gv;
-          if (l == -INFINITY) gv = 0.f;
-          else if (!vis) gv = 1.f;
-          else gv = fmaxf(0.f, -expm1f(dot[u] * a.scale - l));
-          a.gate[t * a.Hq + h] = gv;
+          const int kc = (h / G) * CPH + (c - h * CPH);
+          dot[u] = dot16<T>(qv[u], k0_in_smem ? k0s[kc] : __ldg(k0 + kc));
         }
+      }
+      RS::run(dot, lane);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int h = hv[k];
+        if (!writer || h >= a.Hq) continue;
+        bool vis = vis_band;
+        if (a.bi && vis) {
+          const int qb = qb_base + i / a.block_q;
+          vis = false;
+          if (qb < a.n_qblk) {
+            const int32_t* lst = a.bi + ((long long)(h / G) * a.n_qblk + qb) * a.max_blocks;
+            for (int e = 0; e < a.max_blocks; ++e) vis |= __ldg(lst + e) == 0;
+          }
+        }
+        const float l = lse_v[k];
+        float gv;
+        if (l == -INFINITY) gv = 0.f;
+        else if (!vis) gv = 1.f;
+        else gv = fmaxf(0.f, -expm1f(dot[k] * a.scale - l));
+        a.gate[t * a.Hq + h] = gv;
       }
     }
   }

@@ -75,7 +75,7 @@ struct BwdBuffers {
   const float* dss;     // [T_tot, Hq] upstream dL/d sink_s, or nullptr
   float* delta;         // [Hq, T_tot] workspace (head-major)
   float* lse2;          // [Hq, T_tot] workspace: LSE_new * log2(e), -inf -> +inf
-  float* dsink_part;    // [n_part_blocks, Hq] workspace
+  float* dsink_part;    // [Hq, n_part_blocks] workspace
   float* dq_accum;      // [T_tot, Hq, D] fp32 workspace (tensor path)
   float* dk_accum;      // [T_tot, Hkv, D] fp32 workspace: split key tiles only
   float* dv_accum;      // [T_tot, Hkv, D] fp32 workspace: split key tiles only

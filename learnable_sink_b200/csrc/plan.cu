@@ -369,33 +369,44 @@ __global__ void plan_units_order_kernel(PlanArgs a) {
     order[u] = u;
 }
 
-// G: sort every reverse list by query tile, latest first (insertion sort;
-// lists are short).
-__global__ void plan_bwd_sort_kernel(PlanArgs a) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= a.cap_items) return;
+// G: sort every reverse list by query tile, latest first.  One warp per
+// item: a list of at most kSortShared entries is staged in shared memory and
+// every entry goes straight to its rank (the entries it must follow: larger
+// values, and equal values earlier in the list); a longer list is sorted in
+// place by one lane (insertion sort).
+constexpr int kSortShared = 256;
+constexpr int kSortWarps = 8;
+__global__ void __launch_bounds__(kSortWarps * 32) plan_bwd_sort_kernel(PlanArgs a) {
+  __shared__ int buf[kSortWarps][kSortShared];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kSortWarps + warp;
+  if (i >= a.cap_items) return;  // uniform over the warp
   const TileItem it = reinterpret_cast<const TileItem*>(a.plan + a.off_bwd_items)[i];
   if (it.entry_len <= 1 || it.entry_off + it.entry_len > a.cap_entries) return;
   int* e = a.plan + a.off_bwd_entries + it.entry_off;
-  constexpr int kLocal = 64;
-  if (it.entry_len <= kLocal) {
-    // short list: sort a private copy (L1-resident), then write it back once
-    int w[kLocal];
-    for (int x = 0; x < it.entry_len; ++x) w[x] = e[x];
-    for (int x = 1; x < it.entry_len; ++x) {
+  const int n = it.entry_len;
+  if (n <= kSortShared) {
+    int* w = buf[warp];
+    for (int x = lane; x < n; x += 32) w[x] = e[x];
+    __syncwarp();
+    for (int x = lane; x < n; x += 32) {
       const int v = w[x];
-      int p = x;
-      while (p > 0 && w[p - 1] < v) { w[p] = w[p - 1]; --p; }
-      w[p] = v;
+      int rank = 0;
+      for (int y = 0; y < n; ++y) {
+        const int u = w[y];
+        rank += (u > v) || (u == v && y < x);
+      }
+      e[rank] = v;
     }
-    for (int x = 0; x < it.entry_len; ++x) e[x] = w[x];
     return;
   }
-  for (int x = 1; x < it.entry_len; ++x) {
-    const int v = e[x];
-    int p = x;
-    while (p > 0 && e[p - 1] < v) { e[p] = e[p - 1]; --p; }
-    e[p] = v;
+  if (lane == 0) {
+    for (int x = 1; x < n; ++x) {
+      const int v = e[x];
+      int p = x;
+      while (p > 0 && e[p - 1] < v) { e[p] = e[p - 1]; --p; }
+      e[p] = v;
+    }
   }
 }
 
@@ -466,7 +477,7 @@ int launch_plan(const PlanLaunch& L, cudaStream_t stream) {
   plan_offsets_kernel<<<1, kScanThreads, 0, stream>>>(a, 1);
   plan_zero_kernel<<<nb, 256, 0, stream>>>(a.plan + a.off_bwd_cursor, z.cap_items);
   plan_bwd_scatter_kernel<<<(unsigned)(((long long)z.cap_items * 32 + 255) / 256), 256, 0, stream>>>(a);
-  plan_bwd_sort_kernel<<<nb, 256, 0, stream>>>(a);
+  plan_bwd_sort_kernel<<<(z.cap_items + kSortWarps - 1) / kSortWarps, kSortWarps * 32, 0, stream>>>(a);
   plan_units_scan_kernel<<<1, kScanThreads, 0, stream>>>(a);
   plan_units_fill_kernel<<<nb, 256, 0, stream>>>(a);
   plan_units_order_kernel<<<(z.cap_units + 255) / 256, 256, 0, stream>>>(a);
