@@ -41,7 +41,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // them (consecutive entries of the list) as one 128-key tile, so the score MMA
 // has N = 128 (N = 64 runs at 2/3 of the tensor rate: its shared-memory
 // operand reads become the limit) and the softmax covers 128 columns per pass.
-template <int D_, int TQ_, int TK_, int NQT_, bool PAIR_ = false>
+template <int D_, int TQ_, int TK_, int NQT_, bool PAIR_ = false, int MB_ = 1>
 struct FwdCfg {
   static constexpr int D = D_, TQ = TQ_, TK = TK_, NQT = NQT_;
   static constexpr bool PAIR = PAIR_;
@@ -51,18 +51,24 @@ struct FwdCfg {
   static constexpr int DH = D / 64;              // 64-column halves of a row
   static constexpr int Q_BYTES = 128 * D * 2;    // one query tile
   static constexpr int KV_BYTES = TK * D * 2;    // one K (or V) tile
-  static constexpr int SMEM_BUDGET = 200 * 1024;
+  static constexpr int SMEM_BUDGET = MB_ == 1 ? 200 * 1024 : 108 * 1024;
   static constexpr int NS_RAW = (SMEM_BUDGET - NQT * Q_BYTES) / (2 * KV_BYTES);
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static_assert(NS >= 2, "not enough shared memory for a two-stage ring");
-  static constexpr int MIN_BLOCKS = 1;
-  // With two softmax warpgroups and one CTA per SM, registers are moved to the
-  // softmax warpgroups: the producer and MMA warps then share a warpgroup with
-  // two idle warps (setmaxnreg works on whole warpgroups), 12 warps in all,
-  // 168 registers per thread at launch and 256 x 208 + 128 x 80 = 384 x 168
-  // (with 56 the producer and MMA warps spill; 208 still holds a softmax row).
-  static constexpr bool REBALANCE = (NQT == 2 && MIN_BLOCKS == 1);
-  static constexpr int SOFTMAX_REGS = 208, AUX_REGS = 80;
+  static constexpr int MIN_BLOCKS = MB_;
+  // Registers move to the softmax warpgroups: the producer and MMA warps share
+  // a warpgroup with two idle warps (setmaxnreg works on whole warpgroups).
+  //   two softmax warpgroups, one CTA per SM: 12 warps, 168 registers a thread
+  //     at launch, 256 x 208 + 128 x 80 = 384 x 168 (with 56 the producer and
+  //     MMA warps spill; 208 still holds a softmax row);
+  //   one softmax warpgroup, two CTAs per SM (MB_ = 2, which also halves the
+  //     shared-memory budget and the tensor memory of a CTA): 8 warps, 128
+  //     registers at launch, 128 x 208 + 128 x 48 = 256 x 128.  Each CTA then
+  //     hides the other's prologue and epilogue, which short block-sparse
+  //     query tiles expose.
+  static constexpr bool REBALANCE = (NQT == 2 && MIN_BLOCKS == 1) || (NQT == 1 && MIN_BLOCKS == 2);
+  static constexpr int SOFTMAX_REGS = 208;
+  static constexpr int AUX_REGS = MIN_BLOCKS == 1 ? 80 : 48;
   static constexpr int THREADS = (4 * NQT + (REBALANCE ? 4 : 2)) * 32;
   static constexpr int PRODUCER_WARP = 4 * NQT;
   static constexpr int MMA_WARP = 4 * NQT + 1;
@@ -596,9 +602,9 @@ bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, i
 
 namespace {
 
-template <int D, int TQ, int TK, int NQT, bool PAIR = false>
+template <int D, int TQ, int TK, int NQT, bool PAIR = false, int MB = 1>
 int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
-  using C = FwdCfg<D, TQ, TK, NQT, PAIR>;
+  using C = FwdCfg<D, TQ, TK, NQT, PAIR, MB>;
   CUtensorMap mq, mk, mv;
   if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, TQ) ||
       !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::PT) ||
@@ -631,7 +637,7 @@ int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaS
     // the register split assumes the launch-bound count per thread; with
     // fewer, a setmaxnreg.inc would wait for registers that never come
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != 65536 / C::THREADS / 8 * 8)
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != 65536 / (C::THREADS * C::MIN_BLOCKS) / 8 * 8)
       return SINKATTN_ERR_UNSUPPORTED;
   }
   record_start(SINKATTN_KERNEL_FWD, stream);
@@ -654,13 +660,13 @@ int launch_fwd_tc(const AttnProblem& p, void* out, float* lse, float* sink_s, cu
                : launch_cfg<64, 128, 128, 1>(p, out, lse, sink_s, stream);
   }
   // 64-token tiles need two heads per query tile; key blocks are staged in
-  // pairs as 128-key tiles
+  // pairs as 128-key tiles.  At D = 64 a CTA holds one query tile and two
+  // CTAs share an SM.
   if (G % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;
   const bool two = (G % 4 == 0);
   if (p.D == 128) return two ? launch_cfg<128, 64, 128, 2, true>(p, out, lse, sink_s, stream)
                              : launch_cfg<128, 64, 128, 1, true>(p, out, lse, sink_s, stream);
-  return two ? launch_cfg<64, 64, 128, 2, true>(p, out, lse, sink_s, stream)
-             : launch_cfg<64, 64, 128, 1, true>(p, out, lse, sink_s, stream);
+  return launch_cfg<64, 64, 128, 1, true, 2>(p, out, lse, sink_s, stream);
 }
 
 }  // namespace sk

@@ -145,7 +145,7 @@ struct ReduceScatter {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256) gate_vanilla_kernel(GateVanillaArgs a) {
+__global__ void __launch_bounds__(256, 2) gate_vanilla_kernel(GateVanillaArgs a) {
   constexpr int CPH = D * (int)sizeof(T) / 16;  // 16-byte chunks per head row: 8, 16 or 32
   constexpr int U = kGvInFlight;
   constexpr int NV = U / CPH > 0 ? U / CPH : 1;   // heads a lane finishes per batch
