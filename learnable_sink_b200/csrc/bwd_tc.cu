@@ -15,14 +15,18 @@
 // Tensor memory (512 columns):
 //   S^T  [keys x QR] fp32, overwritten in place by P^T (bf16, packed two per
 //        column at the front of each compute warpgroup's slice)
-//   dP^T [keys x QR] fp32, overwritten by dS^T (bf16, same packing)
+//   dP^T [keys x QR] fp32, overwritten by dS^T (bf16, same packing) when dQ
+//        has columns of its own
 //   dK, dV [keys x D] fp32 accumulators for the whole CTA
 //   dQ   [QR x D] fp32 in its own columns when they fit, else over dP^T once
-//        dK has consumed dS^T
+//        the compute warps have read it
 // MMAs of iteration i, issued by one thread:
-//   dV += P^T dO (TS) | S^T(i+1) = K Q^T (SS) | dK += dS^T Q (TS) |
-//   dQ = dS K (SS; dS^T also staged in shared memory) | dP^T(i+1) = V dO^T (SS)
-// so the tensor cores run dK/dQ of tile i while the compute warps
+//   dV += P^T dO (TS) | S^T(i+1) = K Q^T (SS) | dK += dS^T Q | dQ = dS K (SS;
+//   dS^T staged in shared memory) | dP^T(i+1) = V dO^T (SS)
+// With dQ in its own columns dK reads dS^T from tensor memory (TS) and goes
+// first.  With dQ over dP^T, dQ goes first so that its readout overlaps dK
+// (dP^T(i+1) waits for that readout), and dK reads the staged tile (SS).
+// The tensor cores run dK/dQ of tile i while the compute warps
 // exponentiate tile i+1 (S^T(i+1) moves behind dQ(i) when its Q tile has not
 // landed yet).  Warps 0-7 compute (warpgroup c owns query columns
 // [c QR/2, (c + 1) QR/2), thread = key row); warps 8-11 move each dQ tile out
@@ -75,13 +79,14 @@ struct BwdCfg {
   // registers move to the compute warpgroups; with 64 the launch split fits.
   static constexpr int LAUNCH_REGS = 65536 / THREADS;
   static constexpr bool REBALANCE = QR == 128;
-  static constexpr int COMPUTE_REGS = REBALANCE ? 184 : LAUNCH_REGS;
-  static constexpr int EPI_REGS = REBALANCE ? 72 : LAUNCH_REGS;
-  static constexpr int AUX_REGS = REBALANCE ? 72 : LAUNCH_REGS;
+  static constexpr bool DQ_OWN = 2 * QR + 3 * D <= 512;   // dQ in columns of its own
+  // the dQ epilogue holds half a dQ row when dQ shares the dP^T columns
+  static constexpr int COMPUTE_REGS = REBALANCE ? (DQ_OWN ? 184 : 176) : LAUNCH_REGS;
+  static constexpr int EPI_REGS = REBALANCE ? (DQ_OWN ? 72 : 96) : LAUNCH_REGS;
+  static constexpr int AUX_REGS = REBALANCE ? (DQ_OWN ? 72 : 64) : LAUNCH_REGS;
   static_assert(256 * COMPUTE_REGS + 128 * EPI_REGS + 128 * AUX_REGS <= 65536,
                 "register split exceeds the block's allocation");
   static constexpr int S_COL = 0, DP_COL = QR, DK_COL = 2 * QR, DV_COL = 2 * QR + D;
-  static constexpr bool DQ_OWN = 2 * QR + 3 * D <= 512;   // dQ in columns of its own
   static constexpr int DQ_COL = DQ_OWN ? 2 * QR + 2 * D : DP_COL;
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_K = 0;
@@ -92,7 +97,7 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[QR]
   static constexpr int OFF_DL = OFF_LSE + 512;            // float[QR]
   static constexpr int OFF_BAR = OFF_DL + 512;
-  static constexpr int N_BARS = 1 + 6 * NS + 7;
+  static constexpr int N_BARS = 1 + 6 * NS + 8;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
@@ -181,6 +186,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* bar_dq = bar_ds + 1;
   uint64_t* bar_dqf = bar_dq + 1;
   uint64_t* bar_fin = bar_dqf + 1;
+  uint64_t* bar_dk = bar_fin + 1;    // dK of the iteration complete (Q stage read)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
@@ -223,6 +229,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(bar_dq, 1);
     mbar_init(bar_dqf, 128);
     mbar_init(bar_fin, 1);
+    mbar_init(bar_dk, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -296,31 +303,35 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         constexpr uint32_t id_s = idesc_bf16_f32(KT, QR, 0, 0);  // S^T, dP^T
         constexpr uint32_t id_kv = idesc_bf16_f32(KT, D, 0, 1);  // dV, dK (B MN-major)
         constexpr uint32_t id_q = idesc_bf16_f32(QR, D, 1, 1);   // dQ (A, B MN-major)
+        // operand descriptors at the start of each buffer, K-major (k*) and
+        // MN-major (m*); every operand is a fixed byte offset from one of them
         const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V),
                        sDS = smem_u32(smem + C::OFF_DS), sQ = smem_u32(smem + C::OFF_Q),
                        sDO = smem_u32(smem + C::OFF_DO);
+        const uint32_t kK = sdesc_lo(sK, 16), kV = sdesc_lo(sV, 16), kQ = sdesc_lo(sQ, 16),
+                       kDO = sdesc_lo(sDO, 16), kDS = sdesc_lo(sDS, 16);
+        const uint32_t mQ = sdesc_lo(sQ, C::Q_BYTES / DH), mDO = sdesc_lo(sDO, C::Q_BYTES / DH),
+                       mDS = sdesc_lo(sDS, KT * 128), mK = sdesc_lo(sK, C::KV_BYTES / DH);
         // S^T = K Q^T (both K-major) of iteration j; its Q/dO stage has landed
         auto issue_s = [&](int j) {
-          const uint32_t q_s = sQ + (j % NS) * C::Q_BYTES;
+          const uint32_t q_off = (j % NS) * C::Q_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk & 3) * 32;
-            mma_ss(tmem + C::S_COL,
-                   sdesc_sw128(sK + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
-                   sdesc_sw128(q_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
+            mma_ss(tmem + C::S_COL, sdesc_at(kK, (kk / 4) * (C::KV_BYTES / DH) + off),
+                   sdesc_at(kQ, q_off + (kk / 4) * (C::Q_BYTES / DH) + off), id_s,
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_s);
         };
         // dP^T = V dO^T of iteration j (its dO tile has landed)
         auto issue_dp = [&](int j) {
-          const uint32_t do_s = sDO + (j % NS) * C::Q_BYTES;
+          const uint32_t do_off = (j % NS) * C::Q_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk & 3) * 32;
-            mma_ss(tmem + C::DP_COL,
-                   sdesc_sw128(sV + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024),
-                   sdesc_sw128(do_s + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024), id_s,
+            mma_ss(tmem + C::DP_COL, sdesc_at(kV, (kk / 4) * (C::KV_BYTES / DH) + off),
+                   sdesc_at(kDO, do_off + (kk / 4) * (C::Q_BYTES / DH) + off), id_s,
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_dp);
@@ -336,7 +347,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         for (int i = 0; i < n_it && ok; ++i) {
           const int s = i % NS;
-          const uint32_t q_s = sQ + s * C::Q_BYTES, do_s = sDO + s * C::Q_BYTES;
+          const uint32_t st_off = s * C::Q_BYTES;  // this iteration's Q / dO stage
           const bool more = i + 1 < n_it;
           const int s1 = (i + 1) % NS;
           const uint32_t par1 = ((i + 1) / NS) & 1;
@@ -347,7 +358,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < QR / 16; ++kk)
             mma_ts(tmem + C::DV_COL, tmem + C::S_COL + a_col<CW>(kk),
-                   sdesc_sw128(do_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
+                   sdesc_at(mDO, st_off + kk * 2048), id_kv,
                    (i > 0 || kk > 0) ? 1u : 0u);
           // S^T of the next iteration right behind dV (which frees the S^T
           // columns), if its tiles are already in shared memory
@@ -357,27 +368,42 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             issue_s(i + 1);
             s_next = true;
           }
-          // dK += dS^T Q  (dS^T bf16 in tensor memory over dP^T)
           ok = mbar_wait(bar_ds, i & 1, abort_flag, p.status);
           if (!ok) break;
           tc_fence_after();
+          // dQ = dS K  (A = dS from the staged dS^T tile, both MN-major)
+          auto issue_dq = [&]() {
 #pragma unroll
-          for (int kk = 0; kk < QR / 16; ++kk)
-            mma_ts(tmem + C::DK_COL, tmem + C::DP_COL + a_col<CW>(kk),
-                   sdesc_sw128(q_s + kk * 2048, C::Q_BYTES / DH, 1024), id_kv,
-                   (i > 0 || kk > 0) ? 1u : 0u);
-          // dQ = dS K  (A = dS from the staged dS^T tile, both MN-major); in
-          // columns of its own it waits until the previous tile was read out
-          if (C::DQ_OWN && i > 0) {
-            ok = mbar_wait(bar_dqf, (i - 1) & 1, abort_flag, p.status);
-            if (!ok) break;
-            tc_fence_after();
+            for (int kk = 0; kk < KT / 16; ++kk)
+              mma_ss(tmem + C::DQ_COL, sdesc_at(mDS, kk * 2048), sdesc_at(mK, kk * 2048), id_q,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(bar_dq);  // the stage is released once its dQ tile has been flushed
+          };
+          if constexpr (C::DQ_OWN) {
+            // dK += dS^T Q  (dS^T bf16 in tensor memory over dP^T), then dQ
+            // once the previous tile was read out of its columns
+#pragma unroll
+            for (int kk = 0; kk < QR / 16; ++kk)
+              mma_ts(tmem + C::DK_COL, tmem + C::DP_COL + a_col<CW>(kk),
+                     sdesc_at(mQ, st_off + kk * 2048), id_kv, (i > 0 || kk > 0) ? 1u : 0u);
+            if (i > 0) {
+              ok = mbar_wait(bar_dqf, (i - 1) & 1, abort_flag, p.status);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_dq();
+          } else {
+            // dQ first, then dK += dS^T Q with A = the staged tile read K-major
+            // (keys are its rows, 64 queries per 128-byte row; Q MN-major)
+            issue_dq();
+#pragma unroll
+            for (int kk = 0; kk < QR / 16; ++kk)
+              mma_ss(tmem + C::DK_COL,
+                     sdesc_at(kDS, (kk / 4) * (KT * 128) + (kk & 3) * 32),
+                     sdesc_at(mQ, st_off + kk * 2048), id_kv,
+                     (i > 0 || kk > 0) ? 1u : 0u);
           }
-#pragma unroll
-          for (int kk = 0; kk < KT / 16; ++kk)
-            mma_ss(tmem + C::DQ_COL, sdesc_sw128(sDS + kk * 2048, KT * 128, 1024),
-                   sdesc_sw128(sK + kk * 2048, C::KV_BYTES / DH, 1024), id_q, kk > 0 ? 1u : 0u);
-          mma_commit(bar_dq);  // the stage is released once its dQ tile has been flushed
+          mma_commit(bar_dk);  // the Q tile of the stage may now take staged dQ
           if (more) {
             if (!s_next) {
               ok = mbar_wait(bar_qf + s1, par1, abort_flag, p.status);
@@ -434,9 +460,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   } else if (warp >= C::EPI_WARP0) {
     // ------------------------------------------------------------ dQ epilogue
     // Query row m of the dQ tile sits at lane m (QR = 128) or at lane
-    // m % 16 + 32 (m / 16) (QR = 64).  All MMAs of the iteration are complete,
-    // so the stage's Q buffer takes columns [0, D/2) and its dO buffer columns
-    // [D/2, D), as fp32 boxes of 32 columns with the 128-byte swizzle.  Query
+    // m % 16 + 32 (m / 16) (QR = 64).  The stage's Q buffer takes columns
+    // [0, D/2) and its dO buffer columns [D/2, D), as fp32 boxes of 32 columns
+    // with the 128-byte swizzle.  Query
     // rows past the sequence end carry exact zeros (their P is 0), so adding
     // them is harmless.
     regs_to<C::EPI_REGS, C::LAUNCH_REGS>();
@@ -448,28 +474,66 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int s = i % NS;
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dq, i & 1, abort_flag, p.status))) break;
       tc_fence_after();
+      if constexpr (C::DQ_OWN) {
+        // every MMA of the iteration is complete
 #pragma unroll
-      for (int c32 = 0; c32 < D / 32; ++c32) {
-        uint32_t a[32];
-        tmem_ld32(tmem + lane_off + C::DQ_COL + 32 * c32, a);
-        tmem_ld_wait();
-        if (c32 == D / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(bar_dqf);  // the dQ columns may be overwritten
-        }
-        const int half = c32 / (D / 64), c = c32 % (D / 64);
-        uint8_t* row = smem + (half == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES +
-                       c * (QR * 128) + qrow * 128;
-        if (lane_ok) {
+        for (int c32 = 0; c32 < D / 32; ++c32) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::DQ_COL + 32 * c32, a);
+          tmem_ld_wait();
+          if (c32 == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar_dqf);  // the dQ columns may be overwritten
+          }
+          const int half = c32 / (D / 64), c = c32 % (D / 64);
+          uint8_t* row = smem + (half == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES +
+                         c * (QR * 128) + qrow * 128;
+          if (lane_ok) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
-                make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
+                  make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+          }
+          if (c == D / 64 - 1) {  // a half is staged: the reducer warp takes it from here
+            fence_async_smem();
+            mbar_arrive((half == 0 ? bar_dqs : bar_dds) + s);
+          }
         }
-        if (c == D / 64 - 1) {  // a half is staged: the reducer warp takes it from here
+      } else {
+        // Half 1 (columns [D/2, D), into the dO buffer, which dV and dP^T read
+        // before dQ ran) first, then half 0 (into the Q buffer, which dK reads:
+        // staged only once dK is complete).  The dQ columns are released after
+        // both halves are in registers and dK is complete, so dK(i + 1) cannot
+        // complete before this wait for dK(i).
+        bool got_dk = true;
+#pragma unroll
+        for (int hf = 1; hf >= 0; --hf) {
+          uint32_t a[D / 64][32];
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tmem_ld32(tmem + lane_off + C::DQ_COL + hf * (D / 2) + 32 * c, a[c]);
+          tmem_ld_wait();
+          if (hf == 0) {
+            got_dk = __all_sync(0xffffffffu, mbar_wait(bar_dk, i & 1, abort_flag, p.status));
+            tc_fence_before();
+            mbar_arrive(bar_dqf);  // the dQ columns may be overwritten
+          }
+          if (lane_ok && got_dk) {
+            uint8_t* base = smem + (hf == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES + qrow * 128;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              uint8_t* row = base + c * (QR * 128);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
+                    make_uint4(a[c][4 * j], a[c][4 * j + 1], a[c][4 * j + 2], a[c][4 * j + 3]);
+            }
+          }
+          // the half is staged: the reducer warp takes it from here
           fence_async_smem();
-          mbar_arrive((half == 0 ? bar_dqs : bar_dds) + s);
+          mbar_arrive((hf == 0 ? bar_dqs : bar_dds) + s);
         }
+        if (!got_dk) break;
       }
     }
   } else {
@@ -570,13 +634,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                         P[x + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[x + 1]));
         }
       }
-      if constexpr (CW == 64)
-        tmem_st32(tmem + lane_off + C::DP_COL + CW * cw, ds);
-      else
-        tmem_st16(tmem + lane_off + C::DP_COL + CW * cw, ds);
+      if constexpr (C::DQ_OWN) {  // dK reads dS^T from tensor memory
+        if constexpr (CW == 64)
+          tmem_st32(tmem + lane_off + C::DP_COL + CW * cw, ds);
+        else
+          tmem_st16(tmem + lane_off + C::DP_COL + CW * cw, ds);
+      }
       // The staged dS tile is free: dP^T of this iteration was issued after
-      // the previous dQ MMA, and its completion covers that MMA.  Layout:
-      // [QR / 64 atoms][keys][64 queries] with the 128-byte swizzle.
+      // the previous dQ and dK MMAs, and its completion covers them.  Layout:
+      // [QR / 64 atoms][keys][64 queries] with the 128-byte swizzle; dQ reads
+      // it MN-major and (with dQ over dP^T) dK K-major.
       if (row_ok) {
         constexpr int CHUNKS = CW / 8;  // 16-byte chunks of this warpgroup's queries
         uint8_t* row = smem + C::OFF_DS + ((CW * cw) / 64) * (KT * 128) + r * 128;
@@ -587,7 +654,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               make_uint4(ds[4 * j], ds[4 * j + 1], ds[4 * j + 2], ds[4 * j + 3]);
       }
       fence_async_smem();
-      tmem_st_wait();
+      if constexpr (C::DQ_OWN) tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_ds);
     }

@@ -170,6 +170,23 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
          (uint64_t(2) << 61);
 }
 
+// A descriptor for the same layout `bytes` further on (a multiple of 16): the
+// start address is the low field, in 16-byte units, and shared-memory
+// addresses stay below 2^18, so the sum never carries out of it.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (bytes >> 4);
+}
+// The same descriptors split in two words: every one built here has the high
+// word kSdescHi (SBO = 1024 B, bit 46, 128-byte swizzle), so a kernel that
+// keeps many operand bases live holds only their low words (LBO, start).
+constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t smem_addr, uint32_t lbo_bytes) {
+  return (((lbo_bytes >> 4) & 0x3FFFu) << 16) | ((smem_addr >> 4) & 0x3FFFu);
+}
+__device__ __forceinline__ uint64_t sdesc_at(uint32_t lo, uint32_t bytes) {
+  return (uint64_t(kSdescHi) << 32) | uint64_t(lo + (bytes >> 4));
+}
+
 // Tensor-memory loads/stores: warp w of a warpgroup reaches lanes
 // [32 (w % 4), 32 (w % 4) + 32); thread t of the warp gets lane 32 (w % 4) + t,
 // `N` consecutive 32-bit columns starting at the address's column.

@@ -237,44 +237,50 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
                                           p.window);
       };
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t sq = smem_u32(smem + C::OFF_Q), sk = smem_u32(smem + C::OFF_K),
-                     sv = smem_u32(smem + C::OFF_V);
+      // descriptors of query tile 0, K stage 0 (both K-major) and V stage 0
+      // (B of PV, MN-major: 64-column atoms TK*128 B apart, 8-row groups 1 KB
+      // apart); every other operand is a fixed byte offset from these
+      const uint64_t dq0 = sdesc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(smem + C::OFF_V), TK * 128, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status);
+      bool narrow_prev = false;
       for (int j = 0; j <= nt && ok; ++j) {
+        const bool narrow_j = j < nt && narrow(j);
         if (j < nt) ok = mbar_wait(bar_kf + j % NS, (j / NS) & 1, abort_flag, p.status);
         if (ok && j > 0) ok = mbar_wait(bar_vf + (j - 1) % NS, ((j - 1) / NS) & 1, abort_flag, p.status);
         if (!ok) break;
         tc_fence_after();
+        const uint64_t dv = sdesc_add(dv0, ((j + NS - 1) % NS) * C::KV_BYTES);
+        const uint64_t dk = sdesc_add(dk0, (j % NS) * C::KV_BYTES);
+        const uint32_t idq = narrow_j ? idesc_qk16 : idesc_qk;
+        const int kk_end = narrow_prev ? 1 : TK / 16;
         for (int t = 0; t < NQT && ok; ++t) {
           if (j > 0) {
             ok = mbar_wait(bar_p + t, (j - 1) & 1, abort_flag, p.status);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vbase = sv + ((j - 1) % NS) * C::KV_BYTES;
-            const int kk_end = narrow(j - 1) ? 1 : TK / 16;
 #pragma unroll
             for (int kk = 0; kk < TK / 16; ++kk) {
               if (kk >= kk_end) break;
-              // B = V tile, MN-major: 64-column atoms TK*128 B apart, 8-row groups 1 KB apart
-              const uint64_t bdesc = sdesc_sw128(vbase + kk * 16 * 128, TK * 128, 1024);
-              mma_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * TK + kk * 8, bdesc, idesc_pv,
-                     (j > 1 || kk > 0) ? 1u : 0u);
+              mma_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * TK + kk * 8,
+                     sdesc_add(dv, kk * 16 * 128), idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
             }
           }
           if (j < nt) {
-            const uint32_t qbase = sq + t * C::Q_BYTES;
-            const uint32_t kbase = sk + (j % NS) * C::KV_BYTES;
-            const uint32_t idq = narrow(j) ? idesc_qk16 : idesc_qk;
+            const uint64_t dq = sdesc_add(dq0, t * C::Q_BYTES);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B inside the 128-B row
-              const uint64_t adesc = sdesc_sw128(qbase + (kk / 4) * (C::Q_BYTES / DH) + off, 16, 1024);
-              const uint64_t bdesc = sdesc_sw128(kbase + (kk / 4) * (C::KV_BYTES / DH) + off, 16, 1024);
-              mma_ss(tmem + C::S_COL + t * TK, adesc, bdesc, idq, kk > 0 ? 1u : 0u);
+              // 16 bf16 = 32 B inside the 128-B row; 64-column atoms
+              mma_ss(tmem + C::S_COL + t * TK,
+                     sdesc_add(dq, (kk / 4) * (C::Q_BYTES / DH) + (kk & 3) * 32),
+                     sdesc_add(dk, (kk / 4) * (C::KV_BYTES / DH) + (kk & 3) * 32), idq,
+                     kk > 0 ? 1u : 0u);
             }
             mma_commit(bar_s + t);
           }
         }
+        narrow_prev = narrow_j;
         if (!ok) break;
         if (j > 0) mma_commit(bar_ve + (j - 1) % NS);
         if (j < nt) mma_commit(bar_ke + j % NS);
