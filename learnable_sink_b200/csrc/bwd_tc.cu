@@ -64,6 +64,7 @@ struct BwdCfg {
   static constexpr int CW = QR / 2;             // query columns per compute warpgroup
   static constexpr int DH = D / 64;
   static_assert(QR == 64 || QR == 128, "query rows");
+  static_assert(KT != 64 || QR == 128, "64-key tiles take 128 query rows (two warpgroups of 64)");
   static constexpr int Q_BYTES = QR * D * 2;    // Q or dO tile
   static constexpr int KV_BYTES = KT * D * 2;   // K or V tile
   static constexpr int DS_BYTES = KT * QR * 2;  // dS^T tile
@@ -149,6 +150,25 @@ __device__ __forceinline__ void bulk_wait_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+
+// M = 64 accumulators put row m at lane m % 16 + 32 (m / 16): the lower 16
+// lanes of each warp's quadrant.  The 16x256b / 16x128b shapes spread those
+// 16 lanes over all 32 threads: with .x8, thread t gets register 4k + 2h + e
+// = (lane t/4 + 8h, column 8k + 2 (t % 4) + e) from a 64-column load, and
+// stores register 2k + h to (lane t/4 + 8h, column 4k + t % 4).
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -550,6 +570,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const float* lse_s = s_lse + CW * cw;
     const float* dl_s = s_dl + CW * cw;
+    // KT = 64 (M = 64 tiles): the two key rows and the column offset of this
+    // thread in the 16x256b layout
+    const int r2[2] = {wq * 16 + lane / 4, wq * 16 + lane / 4 + 8};
+    const int cq = 2 * (lane & 3);
     // The next iteration's entry and (for CW of the threads) its LSE2 / Delta
     // values are loaded one iteration ahead, so global-load latency stays off
     // the critical path.
@@ -587,33 +611,71 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s, i & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      float P[CW];
-#pragma unroll
-      for (int h2 = 0; h2 < CW / 32; ++h2) {
+      // KT = 64: every thread of the warp takes part (rows r2[h], columns
+      // 8k + cq + e); otherwise thread = key row, CW columns
+      constexpr int NP = KT == 64 ? 32 : CW;
+      float P[NP];
+      if constexpr (KT == 64) {
         uint32_t a[32];
-        tmem_ld32(tmem + lane_off + C::S_COL + CW * cw + 32 * h2, a);
+        tmem_ld_16x256b_x8(tmem + lane_off + C::S_COL + CW * cw, a);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          P[32 * h2 + c] = fast_exp2(__uint_as_float(a[c]) * p.scale_log2 - lse_s[32 * h2 + c]);
-      }
-      if (partial) {
-        const KeySpan ks = key_span(kj, q0, it.seq_len, p.causal, p.n_sink, p.window);
+        for (int k = 0; k < 8; ++k) {
+          const float2 l = *reinterpret_cast<const float2*>(lse_s + 8 * k + cq);
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
-          const int tok = (CW * cw + c) / HPT;
-          if (tok < ks.lo || tok > ks.hi) P[c] = 0.f;
+          for (int h = 0; h < 2; ++h) {
+            P[4 * k + 2 * h] = fast_exp2(__uint_as_float(a[4 * k + 2 * h]) * p.scale_log2 - l.x);
+            P[4 * k + 2 * h + 1] = fast_exp2(__uint_as_float(a[4 * k + 2 * h + 1]) * p.scale_log2 - l.y);
+          }
         }
-      }
-      {
-        uint32_t pk[CW / 2];
+        if (partial) {
 #pragma unroll
-        for (int c = 0; c < CW / 2; ++c) pk[c] = pack_bf16x2(P[2 * c], P[2 * c + 1]);
-        if constexpr (CW == 64)
-          tmem_st32(tmem + lane_off + C::S_COL + CW * cw, pk);
-        else
-          tmem_st16(tmem + lane_off + C::S_COL + CW * cw, pk);
+          for (int h = 0; h < 2; ++h) {
+            const KeySpan ks = key_span(k0 + r2[h], q0, it.seq_len, p.causal, p.n_sink, p.window);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+#pragma unroll
+              for (int e2 = 0; e2 < 2; ++e2) {
+                const int tok = (CW * cw + 8 * k + cq + e2) / HPT;
+                if (tok < ks.lo || tok > ks.hi) P[4 * k + 2 * h + e2] = 0.f;
+              }
+          }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) pk[2 * k + h] = pack_bf16x2(P[4 * k + 2 * h], P[4 * k + 2 * h + 1]);
+        tmem_st_16x128b_x8(tmem + lane_off + C::S_COL + CW * cw, pk);
         tmem_st_wait();
+      } else {
+#pragma unroll
+        for (int h2 = 0; h2 < CW / 32; ++h2) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::S_COL + CW * cw + 32 * h2, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            P[32 * h2 + c] = fast_exp2(__uint_as_float(a[c]) * p.scale_log2 - lse_s[32 * h2 + c]);
+        }
+        if (partial) {
+          const KeySpan ks = key_span(kj, q0, it.seq_len, p.causal, p.n_sink, p.window);
+#pragma unroll
+          for (int c = 0; c < CW; ++c) {
+            const int tok = (CW * cw + c) / HPT;
+            if (tok < ks.lo || tok > ks.hi) P[c] = 0.f;
+          }
+        }
+        {
+          uint32_t pk[CW / 2];
+#pragma unroll
+          for (int c = 0; c < CW / 2; ++c) pk[c] = pack_bf16x2(P[2 * c], P[2 * c + 1]);
+          if constexpr (CW == 64)
+            tmem_st32(tmem + lane_off + C::S_COL + CW * cw, pk);
+          else
+            tmem_st16(tmem + lane_off + C::S_COL + CW * cw, pk);
+          tmem_st_wait();
+        }
       }
       tc_fence_before();
       mbar_arrive(bar_p);
@@ -621,37 +683,63 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, i & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t ds[CW / 2];
-#pragma unroll
-      for (int h2 = 0; h2 < CW / 32; ++h2) {
+      if constexpr (KT == 64) {
         uint32_t a[32];
-        tmem_ld32(tmem + lane_off + C::DP_COL + CW * cw + 32 * h2, a);
+        tmem_ld_16x256b_x8(tmem + lane_off + C::DP_COL + CW * cw, a);
         tmem_ld_wait();
+        uint32_t dsk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int x = 32 * h2 + 2 * c;
-          ds[16 * h2 + c] = pack_bf16x2(P[x] * (__uint_as_float(a[2 * c]) - dl_s[x]),
-                                        P[x + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[x + 1]));
+        for (int k = 0; k < 8; ++k) {
+          const float2 d = *reinterpret_cast<const float2*>(dl_s + 8 * k + cq);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            dsk[2 * k + h] = pack_bf16x2(P[4 * k + 2 * h] * (__uint_as_float(a[4 * k + 2 * h]) - d.x),
+                                         P[4 * k + 2 * h + 1] * (__uint_as_float(a[4 * k + 2 * h + 1]) - d.y));
         }
-      }
-      if constexpr (C::DQ_OWN) {  // dK reads dS^T from tensor memory
-        if constexpr (CW == 64)
-          tmem_st32(tmem + lane_off + C::DP_COL + CW * cw, ds);
-        else
-          tmem_st16(tmem + lane_off + C::DP_COL + CW * cw, ds);
-      }
-      // The staged dS tile is free: dP^T of this iteration was issued after
-      // the previous dQ and dK MMAs, and its completion covers them.  Layout:
-      // [QR / 64 atoms][keys][64 queries] with the 128-byte swizzle; dQ reads
-      // it MN-major and (with dQ over dP^T) dK K-major.
-      if (row_ok) {
-        constexpr int CHUNKS = CW / 8;  // 16-byte chunks of this warpgroup's queries
-        uint8_t* row = smem + C::OFF_DS + ((CW * cw) / 64) * (KT * 128) + r * 128;
-        const int j0 = ((CW * cw) % 64) / 8;
+        if constexpr (C::DQ_OWN)  // dK reads dS^T from tensor memory
+          tmem_st_16x128b_x8(tmem + lane_off + C::DP_COL + CW * cw, dsk);
+        // staged tile (free as below): key row r2[h], queries CW cw + 8k + cq,
+        // + 1 as one 4-byte word of 16-byte chunk k
 #pragma unroll
-        for (int j = 0; j < CHUNKS; ++j)
-          *reinterpret_cast<uint4*>(row + (((j0 + j) ^ (r & 7)) * 16)) =
-              make_uint4(ds[4 * j], ds[4 * j + 1], ds[4 * j + 2], ds[4 * j + 3]);
+        for (int h = 0; h < 2; ++h) {
+          uint8_t* row = smem + C::OFF_DS + ((CW * cw) / 64) * (KT * 128) + r2[h] * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint32_t*>(row + ((k ^ (r2[h] & 7)) * 16) + 2 * cq) = dsk[2 * k + h];
+        }
+      } else {
+        uint32_t ds[CW / 2];
+#pragma unroll
+        for (int h2 = 0; h2 < CW / 32; ++h2) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::DP_COL + CW * cw + 32 * h2, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int x = 32 * h2 + 2 * c;
+            ds[16 * h2 + c] = pack_bf16x2(P[x] * (__uint_as_float(a[2 * c]) - dl_s[x]),
+                                          P[x + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[x + 1]));
+          }
+        }
+        if constexpr (C::DQ_OWN) {  // dK reads dS^T from tensor memory
+          if constexpr (CW == 64)
+            tmem_st32(tmem + lane_off + C::DP_COL + CW * cw, ds);
+          else
+            tmem_st16(tmem + lane_off + C::DP_COL + CW * cw, ds);
+        }
+        // The staged dS tile is free: dP^T of this iteration was issued after
+        // the previous dQ and dK MMAs, and its completion covers them.  Layout:
+        // [QR / 64 atoms][keys][64 queries] with the 128-byte swizzle; dQ reads
+        // it MN-major and (with dQ over dP^T) dK K-major.
+        if (row_ok) {
+          constexpr int CHUNKS = CW / 8;  // 16-byte chunks of this warpgroup's queries
+          uint8_t* row = smem + C::OFF_DS + ((CW * cw) / 64) * (KT * 128) + r * 128;
+          const int j0 = ((CW * cw) % 64) / 8;
+#pragma unroll
+          for (int j = 0; j < CHUNKS; ++j)
+            *reinterpret_cast<uint4*>(row + (((j0 + j) ^ (r & 7)) * 16)) =
+                make_uint4(ds[4 * j], ds[4 * j + 1], ds[4 * j + 2], ds[4 * j + 3]);
+        }
       }
       fence_async_smem();
       if constexpr (C::DQ_OWN) tmem_st_wait();
