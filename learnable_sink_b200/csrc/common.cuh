@@ -274,28 +274,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x for a pair of values on the FMA pipe, for kernels whose exponentials
-// would otherwise saturate the MUFU unit.  Cody-Waite style reduction
-// x = n + f with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to the
-// nearest integer, whose bits then give n), |f| <= 1/2; 2^f from a degree-4
-// polynomial fitted by iteratively reweighted least squares to the relative
-// error on [-1/2, 1/2] (Lawson's algorithm, near-minimax; max relative error
-// 2.6e-6); 2^n enters through the exponent field.  Valid for x in [-126, 64];
-// x below -126, -inf included, gives exactly 0.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
-  float2 p = make_float2(0.009570101276040077f, 0.009570101276040077f);
-  p = __ffma2_rn(p, f, make_float2(0.05591785907745361f, 0.05591785907745361f));
-  p = __ffma2_rn(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
-  p = __ffma2_rn(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
-  p = __ffma2_rn(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-  const int nx = __float_as_int(t.x) - 0x4B400000, ny = __float_as_int(t.y) - 0x4B400000;
-  const float rx = __int_as_float(__float_as_int(p.x) + (nx << 23));
-  const float ry = __int_as_float(__float_as_int(p.y) + (ny << 23));
-  return make_float2(x.x < -126.f ? 0.f : rx, x.y < -126.f ? 0.f : ry);
-}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

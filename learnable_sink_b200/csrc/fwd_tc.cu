@@ -101,6 +101,32 @@ struct FwdParams {
   float scale_log2;
 };
 
+// Named barrier over `count` threads that also returns the AND of every
+// participant's `in` (the same value in all of them).
+__device__ __forceinline__ bool bar_red_and(int id, int count, bool in) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(res)
+      : "r"(in ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return res != 0;
+}
+
+// Bulk tensor store of a shared-memory box (same box and swizzle as the map's
+// loads); the group is committed and waited for by the issuing thread.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 __device__ __forceinline__ bool wait_noabort(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity))
@@ -112,7 +138,8 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                   const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmap_v,
+                  const __grid_constant__ CUtensorMap tmap_o, const FwdParams p) {
   constexpr int D = C::D, TK = C::TK, NQT = C::NQT, HPT = C::HPT, NS = C::NS, DH = C::DH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -168,6 +195,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
     prefetch_tensormap(&tmap_q);
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
+    prefetch_tensormap(&tmap_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -518,6 +546,13 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
           o_scale = fr / den;
         }
       }
+      // A whole tile (every row stores) goes out through shared memory and a
+      // bulk tensor store: the warpgroup writes its rows into its Q buffer
+      // (every MMA that read Q is complete) in the layout the Q load used,
+      // and one thread stores the box.  A tile cut by the sequence end keeps
+      // per-row stores (the box would spill into the next sequence's rows).
+      const bool whole = ok && it.tile_len == C::TQ;  // uniform over the warp
+      uint8_t* qbuf = smem + C::OFF_Q + t * C::Q_BYTES;
       const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
       uint4* dst = reinterpret_cast<uint4*>(p.out + row * D);
 #pragma unroll
@@ -525,18 +560,38 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
         uint32_t rr[32];
         tmem_ld32(o_addr + c * 32, rr);
         tmem_ld_wait();
-        if (store) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * o_scale, __uint_as_float(rr[8 * v + 1]) * o_scale);
-            u.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * o_scale, __uint_as_float(rr[8 * v + 3]) * o_scale);
-            u.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * o_scale, __uint_as_float(rr[8 * v + 5]) * o_scale);
-            u.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * o_scale, __uint_as_float(rr[8 * v + 7]) * o_scale);
+        for (int v = 0; v < 4; ++v) {
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * o_scale, __uint_as_float(rr[8 * v + 1]) * o_scale);
+          u.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * o_scale, __uint_as_float(rr[8 * v + 3]) * o_scale);
+          u.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * o_scale, __uint_as_float(rr[8 * v + 5]) * o_scale);
+          u.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * o_scale, __uint_as_float(rr[8 * v + 7]) * o_scale);
+          if (whole) {
+            // columns 32c + 8v .. + 7: atom (32c) / 64, 16-byte chunk
+            // ((32c) % 64) / 8 + v, 128-byte swizzle over the row
+            const int col8 = (32 * c) % 64 / 8 + v;
+            *reinterpret_cast<uint4*>(qbuf + (32 * c / 64) * (C::Q_BYTES / DH) + r * 128 +
+                                      ((col8 ^ (r & 7)) * 16)) = u;
+          } else if (store) {
             dst[c * 4 + v] = u;
           }
         }
       }
+    }
+    // Every warp of the warpgroup passes this barrier exactly once; the box
+    // is stored only if all four staged their rows (a warp whose waits timed
+    // out did not, and the outputs of that call are undefined anyway).
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic -> async proxy
+    const bool staged = bar_red_and(1 + t, 128, have_o && ok && it.tile_len == C::TQ);
+    if (staged && wq == 0 && lane == 0) {
+      const int tok0 = it.seq_start + it.tile_start;
+      uint8_t* qbuf = smem + C::OFF_Q + t * C::Q_BYTES;
+#pragma unroll
+      for (int h = 0; h < DH; ++h)
+        tma_store_3d(&tmap_o, qbuf + h * (C::Q_BYTES / DH), h * 64, head0 + t * HPT, tok0);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -611,8 +666,9 @@ namespace {
 template <int D, int TQ, int TK, int NQT, bool PAIR = false, int MB = 1>
 int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
   using C = FwdCfg<D, TQ, TK, NQT, PAIR, MB>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, TQ) ||
+      !make_tmap_3d(&mo, out, p.T_tot, p.Hq, D, C::HPT, TQ) ||
       !make_tmap_3d(&mk, p.k, p.T_tot, p.Hkv, D, 1, C::PT) ||
       !make_tmap_3d(&mv, p.v, p.T_tot, p.Hkv, D, 1, C::PT))
     return SINKATTN_ERR_CUDA;
@@ -647,7 +703,7 @@ int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaS
       return SINKATTN_ERR_UNSUPPORTED;
   }
   record_start(SINKATTN_KERNEL_FWD, stream);
-  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, fp);
+  kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
   record_stop(SINKATTN_KERNEL_FWD, stream);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
