@@ -81,10 +81,9 @@ struct BwdCfg {
   static constexpr int LAUNCH_REGS = 65536 / THREADS;
   static constexpr bool REBALANCE = QR == 128;
   static constexpr bool DQ_OWN = 2 * QR + 3 * D <= 512;   // dQ in columns of its own
-  // the dQ epilogue holds half a dQ row when dQ shares the dP^T columns
-  static constexpr int COMPUTE_REGS = REBALANCE ? (DQ_OWN ? 184 : 176) : LAUNCH_REGS;
-  static constexpr int EPI_REGS = REBALANCE ? (DQ_OWN ? 72 : 96) : LAUNCH_REGS;
-  static constexpr int AUX_REGS = REBALANCE ? (DQ_OWN ? 72 : 64) : LAUNCH_REGS;
+  static constexpr int COMPUTE_REGS = REBALANCE ? 184 : LAUNCH_REGS;
+  static constexpr int EPI_REGS = REBALANCE ? 72 : LAUNCH_REGS;
+  static constexpr int AUX_REGS = REBALANCE ? 72 : LAUNCH_REGS;
   static_assert(256 * COMPUTE_REGS + 128 * EPI_REGS + 128 * AUX_REGS <= 65536,
                 "register split exceeds the block's allocation");
   static constexpr int S_COL = 0, DP_COL = QR, DK_COL = 2 * QR, DV_COL = 2 * QR + D;
@@ -521,37 +520,35 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       } else {
         // Half 1 (columns [D/2, D), into the dO buffer, which dV and dP^T read
-        // before dQ ran) first, then half 0 (into the Q buffer, which dK reads:
-        // staged only once dK is complete).  The dQ columns are released after
-        // both halves are in registers and dK is complete, so dK(i + 1) cannot
-        // complete before this wait for dK(i).
+        // before dQ ran) first, then, once dK is complete, half 0 (into the Q
+        // buffer, which dK reads); 32 columns at a time.  The dQ columns are
+        // released after the last load, so dK(i + 1) cannot complete before
+        // this wait for dK(i).
         bool got_dk = true;
 #pragma unroll
-        for (int hf = 1; hf >= 0; --hf) {
-          uint32_t a[D / 64][32];
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tmem_ld32(tmem + lane_off + C::DQ_COL + hf * (D / 2) + 32 * c, a[c]);
+        for (int q = 0; q < D / 32; ++q) {
+          const int hf = q < D / 64 ? 1 : 0;
+          const int c = q % (D / 64);  // 32-column box within the half
+          if (q == D / 64) got_dk = __all_sync(0xffffffffu, mbar_wait(bar_dk, i & 1, abort_flag, p.status));
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + C::DQ_COL + hf * (D / 2) + 32 * c, a);
           tmem_ld_wait();
-          if (hf == 0) {
-            got_dk = __all_sync(0xffffffffu, mbar_wait(bar_dk, i & 1, abort_flag, p.status));
+          if (q == D / 32 - 1) {
             tc_fence_before();
             mbar_arrive(bar_dqf);  // the dQ columns may be overwritten
           }
           if (lane_ok && got_dk) {
-            uint8_t* base = smem + (hf == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES + qrow * 128;
+            uint8_t* row = smem + (hf == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES +
+                           c * (QR * 128) + qrow * 128;
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              uint8_t* row = base + c * (QR * 128);
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
-                    make_uint4(a[c][4 * j], a[c][4 * j + 1], a[c][4 * j + 2], a[c][4 * j + 3]);
-            }
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(row + ((j ^ (qrow & 7)) * 16)) =
+                  make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
           }
-          // the half is staged: the reducer warp takes it from here
-          fence_async_smem();
-          mbar_arrive((hf == 0 ? bar_dqs : bar_dds) + s);
+          if (c == D / 64 - 1) {  // the half is staged: the reducer warp takes it from here
+            fence_async_smem();
+            mbar_arrive((hf == 0 ? bar_dqs : bar_dds) + s);
+          }
         }
         if (!got_dk) break;
       }
