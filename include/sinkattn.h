@@ -76,7 +76,8 @@ typedef struct CUstream_st *sinkattn_stream_t;
  * always float32 (page 1 section 9: sink_s is kept in FP32). */
 typedef enum {
     SINKATTN_BF16 = 0, /* tensor-core path (tcgen05), fp32 accumulation   */
-    SINKATTN_FP32 = 2  /* exact-fp32 CUDA-core path                        */
+    SINKATTN_FP16 = 1, /* the same path with f16 operands (kind::f16)     */
+    SINKATTN_FP32 = 2  /* fp32: 3xTF32 tensor-core forward, CUDA-core rest */
 } sinkattn_dtype;
 
 /* Mask descriptor (read on the host during the call; the arrays it points to
@@ -141,7 +142,8 @@ int sinkattn_plan(int T_tot, int Hq, int Hkv, const sinkattn_mask *mask,
 /* ---- forward --------------------------------------------------------------
  * Computes O, LSE_new and sink_s (page 1 section 4; page 4 section 5's gate
  * G = sigma(LSE - sink) equals sink_s).
- *   dt        SINKATTN_BF16 (D = 64 or 128) or SINKATTN_FP32 (D = 64 or 128).
+ *   dt        SINKATTN_BF16 or SINKATTN_FP16 (the tensor-core path; P and the
+ *             outputs rounded to dt) or SINKATTN_FP32; D = 64 or 128.
  *   T_tot     total packed tokens (>= 1).   Hq % Hkv == 0.
  *   scale     softmax scale alpha (typically 1/sqrt(D)).
  *   q, k, v   inputs of type dt, layouts above.
@@ -271,7 +273,7 @@ int sinkattn_gate_vanilla(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, 
  *   num_splits     partial results per (sequence, KV head) that the
  *                  workspace holds; 0 picks sinkattn_decode_num_splits.  A
  *                  count above ceil(S / 16) or above 128 is lowered to it
- *                  (same result).  bf16: the streaming kernel gives every warp
+ *                  (same result).  bf16 / f16: the streaming kernel gives every warp
  *                  an equal run of 16-row cache pieces and cuts no
  *                  (sequence, KV head) into more than num_splits runs (1 =
  *                  one warp per pair); fp32: num_splits equal key splits.
@@ -372,7 +374,7 @@ int sinkattn_cache_append_fp8(int B, int Hkv, int D, int n_sink, int window, con
  *   of the last `window` past them -- is written to its slot of sequence s;
  *   the other slots are left as they are.
  *   cache_seqlens_out  device int32 [n_seq] or NULL: receives each length.
- * Both: D in {64, 128}, dt BF16 or FP32, 16-byte aligned pointers (else
+ * Both: D in {64, 128}, dt BF16, FP16 or FP32, 16-byte aligned pointers (else
  * SINKATTN_ERR_INVALID_ARG); launch failures return SINKATTN_ERR_CUDA. */
 int sinkattn_cache_append(sinkattn_dtype dt, int B, int Hkv, int D, int n_sink, int window,
                           const void *k_new, const void *v_new, const int32_t *cache_seqlens,

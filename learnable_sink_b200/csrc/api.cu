@@ -104,7 +104,7 @@ BwdLayout bwd_layout(int dt, int T_tot, int Hq, int Hkv, int D) {
   L.lse2 = off; off += round_up(sizeof(float) * (size_t)T_tot * Hq);
   L.part = off; off += round_up(sizeof(float) * (size_t)preprocess_blocks(T_tot) * Hq);
   L.dq_accum = off;
-  if (dt == SINKATTN_BF16) off += round_up(bwd_tc_workspace_bytes(T_tot, Hq, Hkv, D));
+  if (dt != SINKATTN_FP32) off += round_up(bwd_tc_workspace_bytes(T_tot, Hq, Hkv, D));
   L.total = off;
   return L;
 }
@@ -158,7 +158,7 @@ static int attn_common(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D,
                        const void* q, const void* k, const void* v, const float* sink,
                        const sinkattn_mask* mask, const void* plan, size_t plan_bytes,
                        AttnProblem* p) {
-  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
+  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SINKATTN_ERR_INVALID_ARG;
   if (!mask_ok(T_tot, Hq, Hkv, mask)) return SINKATTN_ERR_INVALID_ARG;
   if (!q || !k || !v || !plan) return SINKATTN_ERR_INVALID_ARG;
@@ -215,7 +215,7 @@ int sinkattn_fwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float 
 size_t sinkattn_bwd_workspace_bytes(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D,
                                     const sinkattn_mask* mask) {
   if (!mask_ok(T_tot, Hq, Hkv, mask) || (D != 64 && D != 128)) return 0;
-  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP32) return 0;
+  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP16 && dt != SINKATTN_FP32) return 0;
   return bwd_layout(dt, T_tot, Hq, Hkv, D).total;
 }
 
@@ -274,7 +274,7 @@ int sinkattn_bwd_ex(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float 
 int sinkattn_gate_vanilla(sinkattn_dtype dt, int T_tot, int Hq, int Hkv, int D, float scale,
                           const void* q, const void* k, const float* lse,
                           const sinkattn_mask* mask, float* gate, sinkattn_stream_t stream) {
-  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
+  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SINKATTN_ERR_INVALID_ARG;
   if (!mask_ok(T_tot, Hq, Hkv, mask)) return SINKATTN_ERR_INVALID_ARG;
   if (!q || !k || !lse || !gate) return SINKATTN_ERR_INVALID_ARG;
@@ -330,7 +330,7 @@ int sinkattn_decode(sinkattn_dtype dt, int B, int Hq, int Hkv, int D, float scal
                     const float* learnable_sink, void* out, float* lse_new, float* sink_s,
                     int num_splits, void* workspace, size_t workspace_bytes,
                     sinkattn_stream_t stream) {
-  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
+  if (dt != SINKATTN_BF16 && dt != SINKATTN_FP16 && dt != SINKATTN_FP32) return SINKATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128)) return SINKATTN_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return SINKATTN_ERR_UNSUPPORTED;

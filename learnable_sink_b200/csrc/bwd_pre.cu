@@ -20,6 +20,8 @@
 // Each CTA owns a fixed range of tokens and writes one partial per head; a
 // second kernel sums the partials in a fixed order, so dsink is bitwise
 // deterministic.  HBM-bound: it streams O and dO once.
+#include <type_traits>
+
 #include "internal.h"
 
 namespace sk {
@@ -36,12 +38,13 @@ constexpr int kRedThreads = 256;
 template <typename T>
 __device__ __forceinline__ float chunk_dot(const uint4& a, const uint4& b) {
   if constexpr (sizeof(T) == 2) {
-    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+    using E = std::conditional_t<std::is_same_v<T, __half>, ElemF16, ElemBf16>;
+    const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+      const float2 u = E::widen(x[i]), v = E::widen(y[i]);
       s = fmaf(u.x, v.x, s);
       s = fmaf(u.y, v.y, s);
     }
@@ -162,6 +165,13 @@ int launch_bwd_preprocess(const AttnProblem& p, const BwdBuffers& b, cudaStream_
       preprocess_kernel<__nv_bfloat16, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
     else
       preprocess_kernel<__nv_bfloat16, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
+  } else if (p.dt == SINKATTN_FP16) {
+    const auto* o = static_cast<const __half*>(b.out);
+    const auto* d = static_cast<const __half*>(b.dout);
+    if (p.D == 64)
+      preprocess_kernel<__half, 64><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
+    else
+      preprocess_kernel<__half, 128><<<nb, kPreThreads, 0, stream>>>(o, d, b.lse, p.sink, b.dss, b.delta, b.lse2, b.dsink_part, p.T_tot, p.Hq);
   } else {
     const auto* o = static_cast<const float*>(b.out);
     const auto* d = static_cast<const float*>(b.dout);

@@ -56,8 +56,9 @@ namespace {
 //   <D, 64, 64, 2>:   64-key block selection: M = 64 for the key-side MMAs
 //                     (same lane layout), query tiles of 64 tokens x 2 heads
 //                     so the dQ MMA keeps M = 128.
-template <int D_, int KT_, int QT_, int HPT_>
+template <int D_, int KT_, int QT_, int HPT_, class E_ = ElemBf16>
 struct BwdCfg {
+  using E = E_;  // 16-bit element type of Q, K, V, dO, P^T, dS^T and the gradients
   static constexpr int D = D_, KT = KT_, QT = QT_, HPT = HPT_;
   static constexpr int QR = QT * HPT;           // query rows per iteration
   static constexpr int NSUB = KT / QT;          // sub-tiles per plan tile
@@ -319,9 +320,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else if (warp == C::MMA_WARP) {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0 && n_it > 0) {
-        constexpr uint32_t id_s = idesc_bf16_f32(KT, QR, 0, 0);  // S^T, dP^T
-        constexpr uint32_t id_kv = idesc_bf16_f32(KT, D, 0, 1);  // dV, dK (B MN-major)
-        constexpr uint32_t id_q = idesc_bf16_f32(QR, D, 1, 1);   // dQ (A, B MN-major)
+        constexpr uint32_t id_s = idesc_16_f32(C::E::kFmt, KT, QR, 0, 0);  // S^T, dP^T
+        constexpr uint32_t id_kv = idesc_16_f32(C::E::kFmt, KT, D, 0, 1);  // dV, dK (B MN-major)
+        constexpr uint32_t id_q = idesc_16_f32(C::E::kFmt, QR, D, 1, 1);   // dQ (A, B MN-major)
         // operand descriptors at the start of each buffer, K-major (k*) and
         // MN-major (m*); every operand is a fixed byte offset from one of them
         const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V),
@@ -642,7 +643,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 8; ++k)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) pk[2 * k + h] = pack_bf16x2(P[4 * k + 2 * h], P[4 * k + 2 * h + 1]);
+          for (int h = 0; h < 2; ++h) pk[2 * k + h] = C::E::pack(P[4 * k + 2 * h], P[4 * k + 2 * h + 1]);
         tmem_st_16x128b_x8(tmem + lane_off + C::S_COL + CW * cw, pk);
         tmem_st_wait();
       } else {
@@ -666,7 +667,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         {
           uint32_t pk[CW / 2];
 #pragma unroll
-          for (int c = 0; c < CW / 2; ++c) pk[c] = pack_bf16x2(P[2 * c], P[2 * c + 1]);
+          for (int c = 0; c < CW / 2; ++c) pk[c] = C::E::pack(P[2 * c], P[2 * c + 1]);
           if constexpr (CW == 64)
             tmem_st32(tmem + lane_off + C::S_COL + CW * cw, pk);
           else
@@ -690,7 +691,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const float2 d = *reinterpret_cast<const float2*>(dl_s + 8 * k + cq);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            dsk[2 * k + h] = pack_bf16x2(P[4 * k + 2 * h] * (__uint_as_float(a[4 * k + 2 * h]) - d.x),
+            dsk[2 * k + h] = C::E::pack(P[4 * k + 2 * h] * (__uint_as_float(a[4 * k + 2 * h]) - d.x),
                                          P[4 * k + 2 * h + 1] * (__uint_as_float(a[4 * k + 2 * h + 1]) - d.y));
         }
         if constexpr (C::DQ_OWN)  // dK reads dS^T from tensor memory
@@ -714,7 +715,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int x = 32 * h2 + 2 * c;
-            ds[16 * h2 + c] = pack_bf16x2(P[x] * (__uint_as_float(a[2 * c]) - dl_s[x]),
+            ds[16 * h2 + c] = C::E::pack(P[x] * (__uint_as_float(a[2 * c]) - dl_s[x]),
                                           P[x + 1] * (__uint_as_float(a[2 * c + 1]) - dl_s[x + 1]));
           }
         }
@@ -762,10 +763,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[4 * c + v] = make_uint4(
-                  pack_bf16x2(__uint_as_float(a[8 * v]) * f, __uint_as_float(a[8 * v + 1]) * f),
-                  pack_bf16x2(__uint_as_float(a[8 * v + 2]) * f, __uint_as_float(a[8 * v + 3]) * f),
-                  pack_bf16x2(__uint_as_float(a[8 * v + 4]) * f, __uint_as_float(a[8 * v + 5]) * f),
-                  pack_bf16x2(__uint_as_float(a[8 * v + 6]) * f, __uint_as_float(a[8 * v + 7]) * f));
+                  C::E::pack(__uint_as_float(a[8 * v]) * f, __uint_as_float(a[8 * v + 1]) * f),
+                  C::E::pack(__uint_as_float(a[8 * v + 2]) * f, __uint_as_float(a[8 * v + 3]) * f),
+                  C::E::pack(__uint_as_float(a[8 * v + 4]) * f, __uint_as_float(a[8 * v + 5]) * f),
+                  C::E::pack(__uint_as_float(a[8 * v + 6]) * f, __uint_as_float(a[8 * v + 7]) * f));
           }
         }
       } else if (store) {
@@ -826,6 +827,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // float4 of each accumulator, all loads before the stores.
 constexpr int kSplitRows = 16;
 constexpr int kSplitVec = 4;
+template <class E>
 __global__ void __launch_bounds__(256) split_tiles_kernel(const int* plan, float* dk_acc,
                                                           float* dv_acc, __nv_bfloat16* dk,
                                                           __nv_bfloat16* dv, int Hkv, int D,
@@ -858,9 +860,9 @@ __global__ void __launch_bounds__(256) split_tiles_kernel(const int* plan, float
       for (int u = 0; u < kSplitVec; ++u) {
         if (e0 + u * 256 >= total) break;
         reinterpret_cast<uint2*>(dk)[off[u]] = make_uint2(
-            pack_bf16x2(x[u].x * alpha, x[u].y * alpha), pack_bf16x2(x[u].z * alpha, x[u].w * alpha));
+            E::pack(x[u].x * alpha, x[u].y * alpha), E::pack(x[u].z * alpha, x[u].w * alpha));
         reinterpret_cast<uint2*>(dv)[off[u]] =
-            make_uint2(pack_bf16x2(y[u].x, y[u].y), pack_bf16x2(y[u].z, y[u].w));
+            make_uint2(E::pack(y[u].x, y[u].y), E::pack(y[u].z, y[u].w));
       }
     } else {
 #pragma unroll
@@ -876,6 +878,7 @@ __global__ void __launch_bounds__(256) split_tiles_kernel(const int* plan, float
 // dQ = alpha * accumulated fp32, rounded to bf16: kDqVec float4 a thread, all
 // loads issued before the stores.
 constexpr int kDqVec = 4;
+template <class E>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* acc, uint2* dq, long long n4,
                                                          float alpha) {
   const long long i0 = (long long)blockIdx.x * (256 * kDqVec) + threadIdx.x;
@@ -889,8 +892,8 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* acc, uint
   for (int u = 0; u < kDqVec; ++u) {
     const long long i = i0 + u * 256;
     if (i < n4)
-      dq[i] = make_uint2(pack_bf16x2(v[u].x * alpha, v[u].y * alpha),
-                         pack_bf16x2(v[u].z * alpha, v[u].w * alpha));
+      dq[i] = make_uint2(E::pack(v[u].x * alpha, v[u].y * alpha),
+                         E::pack(v[u].z * alpha, v[u].w * alpha));
   }
 }
 
@@ -939,15 +942,15 @@ int launch_cfg(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
       return SINKATTN_ERR_UNSUPPORTED;
   }
   const dim3 split_grid(p.ps.cap_items, (C::KT + kSplitRows - 1) / kSplitRows);
-  split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
-                                                     p.Hkv, D, p.scale, 0);
+  split_tiles_kernel<typename C::E><<<split_grid, 256, 0, stream>>>(
+      p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv, p.Hkv, D, p.scale, 0);
   record_start(SINKATTN_KERNEL_BWD, stream);
   kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, mdq, mdk, mdv, bp);
   record_stop(SINKATTN_KERNEL_BWD, stream);
-  split_tiles_kernel<<<split_grid, 256, 0, stream>>>(p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv,
-                                                     p.Hkv, D, p.scale, 1);
+  split_tiles_kernel<typename C::E><<<split_grid, 256, 0, stream>>>(
+      p.plan, b.dk_accum, b.dv_accum, bp.dk, bp.dv, p.Hkv, D, p.scale, 1);
   const long long n4 = (long long)p.T_tot * p.Hq * D / 4;
-  dq_convert_kernel<<<(unsigned)((n4 + 256 * kDqVec - 1) / (256 * kDqVec)), 256, 0, stream>>>(
+  dq_convert_kernel<typename C::E><<<(unsigned)((n4 + 256 * kDqVec - 1) / (256 * kDqVec)), 256, 0, stream>>>(
       reinterpret_cast<const float4*>(b.dq_accum), reinterpret_cast<uint2*>(b.dq), n4, p.scale);
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
@@ -958,13 +961,19 @@ size_t bwd_tc_workspace_bytes(int T_tot, int Hq, int Hkv, int D) {
   return sizeof(float) * (size_t)T_tot * D * (Hq + 2 * Hkv);  // dQ, dK, dV accumulators
 }
 
-int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
+template <class E>
+int launch_bwd_e(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
   if (p.ps.tile == 128)
-    return p.D == 128 ? launch_cfg<BwdCfg<128, 128, 128, 1>>(p, b, stream)
-                      : launch_cfg<BwdCfg<64, 128, 128, 1>>(p, b, stream);
+    return p.D == 128 ? launch_cfg<BwdCfg<128, 128, 128, 1, E>>(p, b, stream)
+                      : launch_cfg<BwdCfg<64, 128, 128, 1, E>>(p, b, stream);
   if ((p.Hq / p.Hkv) % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;  // 64-token tiles pair heads
-  return p.D == 128 ? launch_cfg<BwdCfg<128, 64, 64, 2>>(p, b, stream)
-                    : launch_cfg<BwdCfg<64, 64, 64, 2>>(p, b, stream);
+  return p.D == 128 ? launch_cfg<BwdCfg<128, 64, 64, 2, E>>(p, b, stream)
+                    : launch_cfg<BwdCfg<64, 64, 64, 2, E>>(p, b, stream);
+}
+
+int launch_bwd_tc(const AttnProblem& p, const BwdBuffers& b, cudaStream_t stream) {
+  return p.dt == SINKATTN_FP16 ? launch_bwd_e<ElemF16>(p, b, stream)
+                               : launch_bwd_e<ElemBf16>(p, b, stream);
 }
 
 }  // namespace sk

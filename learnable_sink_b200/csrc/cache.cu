@@ -117,7 +117,7 @@ __global__ void cache_append_fp8_kernel(const uint4* k_new, const uint4* v_new,
 }
 
 bool cache_args_ok(sinkattn_dtype dt, int Hkv, int D, int n_sink, int window) {
-  return (dt == SINKATTN_BF16 || dt == SINKATTN_FP32) && Hkv >= 1 && (D == 64 || D == 128) &&
+  return (dt == SINKATTN_BF16 || dt == SINKATTN_FP16 || dt == SINKATTN_FP32) && Hkv >= 1 && (D == 64 || D == 128) &&
          n_sink >= 0 && window >= 0 && n_sink + window >= 1;
 }
 
@@ -136,7 +136,7 @@ extern "C" int sinkattn_cache_append(sinkattn_dtype dt, int B, int Hkv, int D, i
   if (!cache_args_ok(dt, Hkv, D, n_sink, window) || B < 1) return SINKATTN_ERR_INVALID_ARG;
   if (!k_new || !v_new || !cache_seqlens || !k_cache || !v_cache) return SINKATTN_ERR_INVALID_ARG;
   if (!a16(k_new) || !a16(v_new) || !a16(k_cache) || !a16(v_cache)) return SINKATTN_ERR_INVALID_ARG;
-  const int row16 = Hkv * D * (dt == SINKATTN_BF16 ? 2 : 4) / 16;
+  const int row16 = Hkv * D * (dt == SINKATTN_FP32 ? 4 : 2) / 16;
   cache_append_kernel<<<B, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), cache_seqlens,
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), n_sink + window, n_sink, window,
@@ -154,7 +154,7 @@ extern "C" int sinkattn_cache_fill(sinkattn_dtype dt, int n_seq, int T_tot, int 
     return SINKATTN_ERR_INVALID_ARG;
   if (!a16(k_cache) || !a16(v_cache) || (k && !a16(k)) || (v && !a16(v)))
     return SINKATTN_ERR_INVALID_ARG;
-  const int row16 = Hkv * D * (dt == SINKATTN_BF16 ? 2 : 4) / 16;
+  const int row16 = Hkv * D * (dt == SINKATTN_FP32 ? 4 : 2) / 16;
   const long long warps = T_tot > 0 ? T_tot : 1;
   const long long blocks = (warps * 32 + 255) / 256;
   if (blocks > 0x7fffffffLL) return SINKATTN_ERR_INVALID_ARG;

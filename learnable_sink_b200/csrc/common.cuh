@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -160,6 +161,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
          (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
+// The same for a 16-bit operand format `fmt` (0 = f16, 1 = bf16; A and B of
+// one MMA always share it).
+__host__ __device__ constexpr uint32_t idesc_16_f32(uint32_t fmt, int M, int N, int a_mn_major,
+                                                    int b_mn_major) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (uint32_t(a_mn_major) << 15) |
+         (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2),
 // descriptor version 1 (sm_100).  Offsets in bytes.
@@ -278,6 +286,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The 16-bit element types of the tensor-core path: bf16 and f16 share every
+// layout (2 bytes an element); they differ in the MMA operand format, the
+// rounding of fp32 values to pairs, and the widening of a pair.
+struct ElemBf16 {
+  using T = __nv_bfloat16;
+  static constexpr uint32_t kFmt = 1;
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) { return pack_bf16x2(lo, hi); }
+  __device__ __forceinline__ static float2 widen(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  }
+};
+struct ElemF16 {
+  using T = __half;
+  static constexpr uint32_t kFmt = 0;
+  __device__ __forceinline__ static uint32_t pack(float lo, float hi) { return pack_f16x2(lo, hi); }
+  __device__ __forceinline__ static float2 widen(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+};
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

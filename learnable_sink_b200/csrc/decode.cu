@@ -18,6 +18,8 @@
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "internal.h"
 
 namespace sk {
@@ -270,6 +272,22 @@ __device__ __forceinline__ void mma_top_rows(float& c0, float& c1, uint32_t a_lo
       : "r"(a_lo), "r"(0u), "r"(a_hi), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
 }
 
+// The same with f16 operands.
+__device__ __forceinline__ void mma_top_rows_h(float& c0, float& c1, uint32_t a_lo, uint32_t a_hi,
+                                               uint32_t b0, uint32_t b1) {
+  float x2, x3;
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %10, %10};"
+      : "+f"(c0), "+f"(c1), "=f"(x2), "=f"(x3)
+      : "r"(a_lo), "r"(0u), "r"(a_hi), "r"(0u), "r"(b0), "r"(b1), "f"(0.f));
+}
+template <class E>
+__device__ __forceinline__ void mma_top_rows_e(float& c0, float& c1, uint32_t a_lo, uint32_t a_hi,
+                                               uint32_t b0, uint32_t b1) {
+  if constexpr (E::kFmt == 0) mma_top_rows_h(c0, c1, a_lo, a_hi, b0, b1);
+  else mma_top_rows(c0, c1, a_lo, a_hi, b0, b1);
+}
+
 // Where the partial results of one (sequence, KV head) pair are.  A pair
 // owns np_max units of cache rows; its units are numbered from F = pair
 // np_max in a space split into runs of ppw units, and the run of global unit
@@ -370,7 +388,10 @@ __device__ __forceinline__ void combine_head(const DecodeProblem& p, const DecSc
 #pragma unroll
   for (int k = 0; k < DPL; k += 2) {
     const float o0 = den > 0.f ? o[k] / den : 0.f, o1 = den > 0.f ? o[k + 1] / den : 0.f;
-    if constexpr (sizeof(T) == 2)
+    if constexpr (std::is_same_v<T, __half>)
+      *reinterpret_cast<uint32_t*>(static_cast<__half*>(p.out) + row * D + lane * DPL + k) =
+          pack_f16x2(o0, o1);
+    else if constexpr (sizeof(T) == 2)
       *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) + row * D + lane * DPL + k) =
           pack_bf16x2(o0, o1);
     else
@@ -395,7 +416,7 @@ __device__ __forceinline__ void wait_prerequisite_grids() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <int D, int G>
+template <int D, int G, class E = ElemBf16>
 __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     DecodeProblem p, DecSched sc, int n_warps) {
@@ -556,8 +577,8 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
         const int row = (mi >> 1) * 8 + mr, chunk = ((2 * kk) & 7) + (mi & 1);
         uint32_t r[4];
         ldsm_x4(kb + (kk >> 2) * Geo::HALF_BYTES + row * 128 + ((chunk ^ mr) << 4), r);
-        mma_top_rows(sa0, sa1, qa[kk][0], qa[kk][1], r[0], r[1]);
-        mma_top_rows(sb0, sb1, qa[kk][0], qa[kk][1], r[2], r[3]);
+        mma_top_rows_e<E>(sa0, sa1, qa[kk][0], qa[kk][1], r[0], r[1]);
+        mma_top_rows_e<E>(sb0, sb1, qa[kk][0], qa[kk][1], r[2], r[3]);
       }
       // scores of head g at rows 2t, 2t + 1, 8 + 2t, 9 + 2t (log2 units)
       const int ra = 2 * t;
@@ -585,7 +606,7 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
       const float p2 = x2 == -INFINITY ? 0.f : fast_exp2(x2 - m_run);
       const float p3 = x3 == -INFINITY ? 0.f : fast_exp2(x3 - m_run);
       l_run += (p0 + p1) + (p2 + p3);
-      const uint32_t pa_lo = pack_bf16x2(p0, p1), pa_hi = pack_bf16x2(p2, p3);
+      const uint32_t pa_lo = E::pack(p0, p1), pa_hi = E::pack(p2, p3);
       // O += P V, two n-tiles (16 columns) per ldmatrix
 #pragma unroll
       for (int jp = 0; jp < Geo::NT / 2; ++jp) {
@@ -593,8 +614,8 @@ __global__ void __launch_bounds__(kDecWarps * 32, 1) decode_warp_kernel(
         const int row = (mi & 1) * 8 + mr, chunk = ((2 * jp) & 7) + (mi >> 1);
         uint32_t r[4];
         ldsm_x4_trans(vb + (jp >> 2) * Geo::HALF_BYTES + row * 128 + ((chunk ^ mr) << 4), r);
-        mma_top_rows(oc[2 * jp][0], oc[2 * jp][1], pa_lo, pa_hi, r[0], r[1]);
-        mma_top_rows(oc[2 * jp + 1][0], oc[2 * jp + 1][1], pa_lo, pa_hi, r[2], r[3]);
+        mma_top_rows_e<E>(oc[2 * jp][0], oc[2 * jp][1], pa_lo, pa_hi, r[0], r[1]);
+        mma_top_rows_e<E>(oc[2 * jp + 1][0], oc[2 * jp + 1][1], pa_lo, pa_hi, r[2], r[3]);
       }
       __syncwarp();  // every lane is done with the stage
       ++pc_cons;
@@ -670,15 +691,16 @@ int launch_combine(const DecodeProblem& p, const DecSched& sc, cudaStream_t stre
   return cudaGetLastError() == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
-template <int D, int G>
+template <class T, int D, int G>
 int launch_tma(const DecodeProblem& p, cudaStream_t stream) {
+  using E = std::conditional_t<std::is_same_v<T, __half>, ElemF16, ElemBf16>;
   using Geo = WarpGeom<D, G>;
   const int S = p.n_sink + p.window;
   CUtensorMap mk, mv;
   if (!make_tmap_3d(&mk, p.k_cache, p.B * S, p.Hkv, D, 1, Geo::R) ||
       !make_tmap_3d(&mv, p.v_cache, p.B * S, p.Hkv, D, 1, Geo::R))
     return SINKATTN_ERR_CUDA;
-  auto kern = decode_warp_kernel<D, G>;
+  auto kern = decode_warp_kernel<D, G, E>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM) !=
       cudaSuccess)
     return SINKATTN_ERR_CUDA;
@@ -694,12 +716,14 @@ int launch_tma(const DecodeProblem& p, cudaStream_t stream) {
   kern<<<grid, kDecWarps * 32, Geo::SMEM, stream>>>(mk, mv, p, sc, ds.n_warps);
   record_stop(SINKATTN_KERNEL_DECODE, stream);
   if (cudaGetLastError() != cudaSuccess) return SINKATTN_ERR_CUDA;
-  return launch_combine<__nv_bfloat16, D>(p, sc, stream);
+  return launch_combine<T, D>(p, sc, stream);
 }
 
 template <typename T, int D, int G>
 int launch_split(const DecodeProblem& p, cudaStream_t stream) {
-  if constexpr (sizeof(T) == 2) return launch_tma<D, G>(p, stream);
+  if constexpr (sizeof(T) == 2) {
+    return launch_tma<T, D, G>(p, stream);
+  } else {
   using Geo = DecGeom<D>;
   const int S = p.n_sink + p.window;
   // fp32: one CTA per (split, KV head, sequence), splits of `chunk` slots
@@ -717,6 +741,7 @@ int launch_split(const DecodeProblem& p, cudaStream_t stream) {
   if (cudaGetLastError() != cudaSuccess) return SINKATTN_ERR_CUDA;
   // split i of a pair is unit i of a run of one unit
   return launch_combine<T, D>(p, DecSched{chunk, p.num_splits, 1, 0}, stream);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -772,10 +797,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
       static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu), __NV_E4M3);
   return uint32_t(h.x) | (uint32_t(h.y) << 16);
-}
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  const __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
 }
 // 16-byte chunk of a swizzled window row: 128-byte rows (D = 128) use the
 // 128-byte swizzle (chunk ^ row % 8), 64-byte rows the 64-byte swizzle
@@ -1202,6 +1223,8 @@ int launch_decode(const DecodeProblem& p, cudaStream_t stream) {
   if (p.dt == SINKATTN_BF16)
     return p.D == 64 ? dispatch_g<__nv_bfloat16, 64>(p, stream)
                      : dispatch_g<__nv_bfloat16, 128>(p, stream);
+  if (p.dt == SINKATTN_FP16)
+    return p.D == 64 ? dispatch_g<__half, 64>(p, stream) : dispatch_g<__half, 128>(p, stream);
   return p.D == 64 ? dispatch_g<float, 64>(p, stream) : dispatch_g<float, 128>(p, stream);
 }
 

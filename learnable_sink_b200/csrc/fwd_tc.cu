@@ -41,8 +41,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // them (consecutive entries of the list) as one 128-key tile, so the score MMA
 // has N = 128 (N = 64 runs at 2/3 of the tensor rate: its shared-memory
 // operand reads become the limit) and the softmax covers 128 columns per pass.
-template <int D_, int TQ_, int TK_, int NQT_, bool PAIR_ = false, int MB_ = 1>
+template <int D_, int TQ_, int TK_, int NQT_, bool PAIR_ = false, int MB_ = 1, class E_ = ElemBf16>
 struct FwdCfg {
+  using E = E_;  // 16-bit element type of Q, K, V, O (and of P)
   static constexpr int D = D_, TQ = TQ_, TK = TK_, NQT = NQT_;
   static constexpr bool PAIR = PAIR_;
   static constexpr int PT = PAIR ? TK / 2 : TK;  // the plan's key tile
@@ -256,15 +257,15 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, TK, 0, 0);
-      constexpr uint32_t idesc_qk16 = idesc_bf16_f32(128, 16, 0, 0);
+      constexpr uint32_t idesc_qk = idesc_16_f32(C::E::kFmt, 128, TK, 0, 0);
+      constexpr uint32_t idesc_qk16 = idesc_16_f32(C::E::kFmt, 128, 16, 0, 0);
       // staged tile j is a band's sink-only first tile: scores on its first
       // 16 keys only, values from those 16 rows only
       auto narrow = [&](int j) {
         return !C::PAIR && sink_only_tile(__ldg(ent + j) >> 1, it.tile_start, TK, p.n_sink,
                                           p.window);
       };
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idesc_pv = idesc_16_f32(C::E::kFmt, 128, D, 0, 1);
       // descriptors of query tile 0, K stage 0 (both K-major) and V stage 0
       // (B of PV, MN-major: 64-column atoms TK*128 B apart, 8-row groups 1 KB
       // apart); every other operand is a fixed byte offset from these
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
           const float p0 = fast_exp2(fmaf(x16[2 * i], p.scale_log2, -mu));
           const float p1 = fast_exp2(fmaf(x16[2 * i + 1], p.scale_log2, -mu));
           rs += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          pk[i] = C::E::pack(p0, p1);
         }
         tmem_st8(s_addr, pk);
         l += rs;
@@ -492,7 +493,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
           const float2 y = __ffma2_rn(make_float2(x[c * 64 + 2 * i], x[c * 64 + 2 * i + 1]), sc2, nm2);
           const float2 pp = make_float2(fast_exp2(y.x), fast_exp2(y.y));
           rs4[i & 3] = __fadd2_rn(rs4[i & 3], pp);
-          pk[i] = pack_bf16x2(pp.x, pp.y);
+          pk[i] = C::E::pack(pp.x, pp.y);
         }
         tmem_st32(s_addr + c * 32, pk);  // P over the first TK/2 columns of S_t
       }
@@ -563,10 +564,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * o_scale, __uint_as_float(rr[8 * v + 1]) * o_scale);
-          u.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * o_scale, __uint_as_float(rr[8 * v + 3]) * o_scale);
-          u.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * o_scale, __uint_as_float(rr[8 * v + 5]) * o_scale);
-          u.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * o_scale, __uint_as_float(rr[8 * v + 7]) * o_scale);
+          u.x = C::E::pack(__uint_as_float(rr[8 * v + 0]) * o_scale, __uint_as_float(rr[8 * v + 1]) * o_scale);
+          u.y = C::E::pack(__uint_as_float(rr[8 * v + 2]) * o_scale, __uint_as_float(rr[8 * v + 3]) * o_scale);
+          u.z = C::E::pack(__uint_as_float(rr[8 * v + 4]) * o_scale, __uint_as_float(rr[8 * v + 5]) * o_scale);
+          u.w = C::E::pack(__uint_as_float(rr[8 * v + 6]) * o_scale, __uint_as_float(rr[8 * v + 7]) * o_scale);
           if (whole) {
             // columns 32c + 8v .. + 7: atom (32c) / 64, 16-byte chunk
             // ((32c) % 64) / 8 + v, 128-byte swizzle over the row
@@ -663,9 +664,9 @@ bool make_tmap_3d_f32(CUtensorMap* map, const void* base, int T, int H, int D, i
 
 namespace {
 
-template <int D, int TQ, int TK, int NQT, bool PAIR = false, int MB = 1>
+template <class E, int D, int TQ, int TK, int NQT, bool PAIR = false, int MB = 1>
 int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
-  using C = FwdCfg<D, TQ, TK, NQT, PAIR, MB>;
+  using C = FwdCfg<D, TQ, TK, NQT, PAIR, MB, E>;
   CUtensorMap mq, mk, mv, mo;
   if (!make_tmap_3d(&mq, p.q, p.T_tot, p.Hq, D, C::HPT, TQ) ||
       !make_tmap_3d(&mo, out, p.T_tot, p.Hq, D, C::HPT, TQ) ||
@@ -710,25 +711,31 @@ int launch_cfg(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaS
 
 }  // namespace
 
-int launch_fwd_tc(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
+template <class E>
+int launch_fwd_e(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
   const int G = p.Hq / p.Hkv;
   const int tile = p.ps.tile;  // 128 (dense masks) or the block size (64/128)
   // a query tile is 128 rows: 128 tokens x 1 head, or 64 tokens x 2 heads
   if (tile == 128) {
     const bool two = (G % 2 == 0);
-    if (p.D == 128) return two ? launch_cfg<128, 128, 128, 2>(p, out, lse, sink_s, stream)
-                               : launch_cfg<128, 128, 128, 1>(p, out, lse, sink_s, stream);
-    return two ? launch_cfg<64, 128, 128, 2>(p, out, lse, sink_s, stream)
-               : launch_cfg<64, 128, 128, 1>(p, out, lse, sink_s, stream);
+    if (p.D == 128) return two ? launch_cfg<E, 128, 128, 128, 2>(p, out, lse, sink_s, stream)
+                               : launch_cfg<E, 128, 128, 128, 1>(p, out, lse, sink_s, stream);
+    return two ? launch_cfg<E, 64, 128, 128, 2>(p, out, lse, sink_s, stream)
+               : launch_cfg<E, 64, 128, 128, 1>(p, out, lse, sink_s, stream);
   }
   // 64-token tiles need two heads per query tile; key blocks are staged in
   // pairs as 128-key tiles.  At D = 64 a CTA holds one query tile and two
   // CTAs share an SM.
   if (G % 2 != 0) return SINKATTN_ERR_UNSUPPORTED;
   const bool two = (G % 4 == 0);
-  if (p.D == 128) return two ? launch_cfg<128, 64, 128, 2, true>(p, out, lse, sink_s, stream)
-                             : launch_cfg<128, 64, 128, 1, true>(p, out, lse, sink_s, stream);
-  return launch_cfg<64, 64, 128, 1, true, 2>(p, out, lse, sink_s, stream);
+  if (p.D == 128) return two ? launch_cfg<E, 128, 64, 128, 2, true>(p, out, lse, sink_s, stream)
+                             : launch_cfg<E, 128, 64, 128, 1, true>(p, out, lse, sink_s, stream);
+  return launch_cfg<E, 64, 64, 128, 1, true, 2>(p, out, lse, sink_s, stream);
+}
+
+int launch_fwd_tc(const AttnProblem& p, void* out, float* lse, float* sink_s, cudaStream_t stream) {
+  return p.dt == SINKATTN_FP16 ? launch_fwd_e<ElemF16>(p, out, lse, sink_s, stream)
+                               : launch_fwd_e<ElemBf16>(p, out, lse, sink_s, stream);
 }
 
 }  // namespace sk

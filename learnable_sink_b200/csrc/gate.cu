@@ -12,6 +12,8 @@
 // head i % Hq of rows i / Hq, i / Hq + R, ...); the second sums the partials
 // per head in a fixed order.  The partition depends only on (T_tot, Hq), so
 // the result is bitwise reproducible.  HBM-bound: sink_s is read once.
+#include <type_traits>
+
 #include "internal.h"
 
 namespace sk {
@@ -93,12 +95,13 @@ constexpr int kGvK0Smem = 32 * 1024;
 template <typename T>
 __device__ __forceinline__ float dot16(const uint4& a, const uint4& b) {
   if constexpr (sizeof(T) == 2) {
-    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+    using E = std::conditional_t<std::is_same_v<T, __half>, ElemF16, ElemBf16>;
+    const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+      const float2 u = E::widen(x[i]), v = E::widen(y[i]);
       s = fmaf(u.x, v.x, s);
       s = fmaf(u.y, v.y, s);
     }
@@ -243,12 +246,15 @@ __global__ void __launch_bounds__(256, 2) gate_vanilla_kernel(GateVanillaArgs a)
 int launch_gate_vanilla(const GateVanillaArgs& a, int dt, int D, int max_seqlen,
                         cudaStream_t stream) {
   const dim3 grid((max_seqlen + kGvRows - 1) / kGvRows, a.n_seq);
-  const size_t k0_bytes = (size_t)a.Hkv * D * (dt == SINKATTN_BF16 ? 2 : 4);
+  const size_t k0_bytes = (size_t)a.Hkv * D * (dt == SINKATTN_FP32 ? 4 : 2);
   const size_t smem = k0_bytes <= (size_t)kGvK0Smem ? k0_bytes : 0;
   record_start(SINKATTN_KERNEL_GATE, stream);
   if (dt == SINKATTN_BF16) {
     if (D == 64) gate_vanilla_kernel<__nv_bfloat16, 64><<<grid, 256, smem, stream>>>(a);
     else gate_vanilla_kernel<__nv_bfloat16, 128><<<grid, 256, smem, stream>>>(a);
+  } else if (dt == SINKATTN_FP16) {
+    if (D == 64) gate_vanilla_kernel<__half, 64><<<grid, 256, smem, stream>>>(a);
+    else gate_vanilla_kernel<__half, 128><<<grid, 256, smem, stream>>>(a);
   } else {
     if (D == 64) gate_vanilla_kernel<float, 64><<<grid, 256, smem, stream>>>(a);
     else gate_vanilla_kernel<float, 128><<<grid, 256, smem, stream>>>(a);

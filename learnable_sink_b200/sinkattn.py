@@ -19,7 +19,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsinkattn.so")
 
-BF16, FP32 = 0, 2
+BF16, FP16, FP32 = 0, 1, 2
 OK = 0
 ERR_NAMES = {1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "WORKSPACE", 5: "TIMEOUT",
              6: "BOUNDS", 7: "PLAN"}
@@ -121,9 +121,11 @@ def _stream(stream=None):
 def _dt(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return BF16
+    if t.dtype == torch.float16:
+        return FP16
     if t.dtype == torch.float32:
         return FP32
-    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16, float16 or float32")
 
 
 @dataclass

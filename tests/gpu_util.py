@@ -11,6 +11,10 @@ from learnable_sink_b200 import sinkattn as S
 TOL = {
     torch.float32: dict(o=1e-4, lse=1e-4, ss=1e-4, grad=1e-3),
     torch.bfloat16: dict(o=2e-2, lse=1e-3, ss=1e-3, grad=2e-2),
+    # f16 keeps 3 more mantissa bits than bf16 (P, dS and the outputs are
+    # rounded to it); the bounds are a quarter of bf16's for O and half for
+    # the gradients
+    torch.float16: dict(o=5e-3, lse=1e-3, ss=1e-3, grad=1e-2),
 }
 
 

@@ -95,7 +95,7 @@ def test_gate_vanilla_and_bwd_ex_host_validation(lib):
     a16 = 256  # stand-in 16-byte-aligned device addresses: never dereferenced here
     gv = lib.sinkattn_gate_vanilla
     assert gv(0, 128, 4, 2, 96, 0.1, a16, a16, a16, ctypes.byref(m), a16, None) == 1  # D
-    assert gv(1, 128, 4, 2, 64, 0.1, a16, a16, a16, ctypes.byref(m), a16, None) == 1  # fp16
+    assert gv(3, 128, 4, 2, 64, 0.1, a16, a16, a16, ctypes.byref(m), a16, None) == 1  # no such dtype
     assert gv(0, 128, 4, 2, 64, 0.1, None, a16, a16, ctypes.byref(m), a16, None) == 1  # q
     assert gv(0, 128, 4, 2, 64, 0.1, a16, a16, a16, ctypes.byref(m), None, None) == 1  # gate
     assert gv(0, 128, 4, 2, 64, 0.1, a16 + 8, a16, a16, ctypes.byref(m), a16, None) == 1
