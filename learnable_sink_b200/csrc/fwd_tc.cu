@@ -73,9 +73,16 @@ struct FwdCfg {
   static constexpr int THREADS = (4 * NQT + (REBALANCE ? 4 : 2)) * 32;
   static constexpr int PRODUCER_WARP = 4 * NQT;
   static constexpr int MMA_WARP = 4 * NQT + 1;
+  // SDB: one query tile, two CTAs per SM, and the score tiles of consecutive
+  // key tiles in two overlapping tensor-memory regions, [0, TK) for even j and
+  // [TK/2, 3TK/2) for odd j, with P(j) packed into the half the next region
+  // leaves free ([0, TK/2) or [TK, 3TK/2)).  S(j+1) is then issued as soon as
+  // the softmax has read S(j) into registers, and the softmax never waits for
+  // the PV and S MMAs of its own tile between two key tiles.
+  static constexpr bool SDB = PAIR_ && MB_ == 2 && NQT_ == 1;
   static constexpr int S_COL = 0;                // S_t at t * TK
-  static constexpr int O_COL = NQT * TK;         // O_t at O_COL + t * D
-  static constexpr int TMEM_NEED = NQT * (TK + D);
+  static constexpr int O_COL = SDB ? TK + TK / 2 : NQT * TK;  // O_t at O_COL + t * D
+  static constexpr int TMEM_NEED = SDB ? TK + TK / 2 + D : NQT * (TK + D);
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64
                                  : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   static_assert(TMEM_NEED <= 512, "tensor memory budget");
@@ -84,7 +91,7 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + NQT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-  static constexpr int N_BARS = 1 + 4 * NS + 3 * NQT + 1;
+  static constexpr int N_BARS = 1 + 4 * NS + 5 * NQT + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
 };
@@ -154,6 +161,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
   uint64_t* bar_p = bar_s + NQT;
   uint64_t* bar_o = bar_p + NQT;
   uint64_t* bar_fin = bar_o + NQT;
+  uint64_t* bar_sr = bar_fin + 1;  // SDB: the softmax has read S_t(j)
+  uint64_t* bar_pv = bar_sr + NQT;  // SDB: PV_t(j) complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -183,6 +192,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       mbar_init(bar_s + t, 1);
       mbar_init(bar_p + t, 128);
       mbar_init(bar_o + t, 1);
+      mbar_init(bar_sr + t, 128);
+      mbar_init(bar_pv + t, 1);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -273,6 +284,51 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       const uint64_t dk0 = sdesc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(smem + C::OFF_V), TK * 128, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status);
+      if constexpr (C::SDB) {
+        // S(j+1) into the other region as soon as the softmax has read S(j)
+        // (and after PV(j-1), whose P it overwrites: tcgen05 operations run
+        // in issue order); PV(j) once P(j) is written.
+        auto issue_s = [&](int j) {
+          const uint64_t dk = sdesc_add(dk0, (j % NS) * C::KV_BYTES);
+          const uint32_t s_col = (j & 1) ? TK / 2 : 0;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + s_col, sdesc_add(dq0, (kk / 4) * (C::Q_BYTES / DH) + (kk & 3) * 32),
+                   sdesc_add(dk, (kk / 4) * (C::KV_BYTES / DH) + (kk & 3) * 32), idesc_qk,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar_s);
+          mma_commit(bar_ke + j % NS);
+        };
+        if (ok) ok = mbar_wait(bar_kf, 0, abort_flag, p.status);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+        }
+        for (int j = 0; j < nt && ok; ++j) {
+          if (j + 1 < nt) {
+            ok = mbar_wait(bar_sr, j & 1, abort_flag, p.status) &&
+                 mbar_wait(bar_kf + (j + 1) % NS, ((j + 1) / NS) & 1, abort_flag, p.status);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(j + 1);
+          }
+          ok = mbar_wait(bar_p, j & 1, abort_flag, p.status) &&
+               mbar_wait(bar_vf + j % NS, (j / NS) & 1, abort_flag, p.status);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dv = sdesc_add(dv0, (j % NS) * C::KV_BYTES);
+          const uint32_t p_col = (j & 1) ? TK : 0;
+#pragma unroll
+          for (int kk = 0; kk < TK / 16; ++kk)
+            mma_ts(tmem + C::O_COL, tmem + p_col + kk * 8, sdesc_add(dv, kk * 16 * 128), idesc_pv,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_ve + j % NS);
+          mma_commit(bar_pv);
+        }
+        if (ok) mma_commit(bar_o);
+        mma_commit(bar_fin);
+        wait_noabort(bar_fin, 0);
+      } else {
       bool narrow_prev = false;
       for (int j = 0; j <= nt && ok; ++j) {
         const bool narrow_j = j < nt && narrow(j);
@@ -319,6 +375,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       // drain: every MMA issued by this thread has completed once bar_fin fires
       mma_commit(bar_fin);
       wait_noabort(bar_fin, 0);
+      }
     }
   } else if (warp < 4 * NQT) {
     // ------------------------------------------------------------ softmax
@@ -399,11 +456,12 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       }
       // raw scores x = Q.K (the scale is folded into the exponent below)
       // all TK / 32 loads in flight, one wait for them together
+      const uint32_t s_cur = C::SDB ? tmem + lane_off + ((j & 1) ? TK / 2 : 0) : s_addr;
       float x[TK];
       {
         uint32_t rr[TK / 32][32];
 #pragma unroll
-        for (int c = 0; c < TK / 32; ++c) tmem_ld32(s_addr + c * 32, rr[c]);
+        for (int c = 0; c < TK / 32; ++c) tmem_ld32(s_cur + c * 32, rr[c]);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < TK / 32; ++c)
@@ -412,6 +470,11 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
             asm volatile("" : "+r"(rr[c][i]));  // the values exist only after the wait
             x[c * 32 + i] = __uint_as_float(rr[c][i]);
           }
+      }
+      if constexpr (C::SDB) {
+        // S(j) is in registers: the next score tile may overwrite its columns
+        tc_fence_before();
+        mbar_arrive(bar_sr + t);
       }
       // partial tiles: element mask from the row's visible span
       if constexpr (C::PAIR) {
@@ -464,7 +527,16 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       const bool touch_o = need && j > 0 && m != -INFINITY;
       if (__any_sync(0xffffffffu, touch_o)) {
         // O_t row *= corr.  Safe: PV_t(j-1) completed before S_t(j) was
-        // signalled (tcgen05 operations complete in issue order).
+        // signalled (tcgen05 operations complete in issue order); with SDB
+        // S_t(j) was issued before PV_t(j-1), whose completion is awaited
+        // here (PV_t(j) waits for this tile's P, so the phase is unambiguous).
+        if constexpr (C::SDB) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_pv + t, (j - 1) & 1, abort_flag, p.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
         const float f = touch_o ? corr : 1.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -495,7 +567,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
           rs4[i & 3] = __fadd2_rn(rs4[i & 3], pp);
           pk[i] = C::E::pack(pp.x, pp.y);
         }
-        tmem_st32(s_addr + c * 32, pk);  // P over the first TK/2 columns of S_t
+        // P over the first TK/2 columns of S_t (with SDB, of the half the
+        // next score tile leaves free)
+        tmem_st32((C::SDB ? tmem + lane_off + ((j & 1) ? TK : 0) : s_addr) + c * 32, pk);
       }
       const float2 r01 = __fadd2_rn(rs4[0], rs4[1]), r23 = __fadd2_rn(rs4[2], rs4[3]);
       const float2 rsum = __fadd2_rn(r01, r23);
