@@ -100,7 +100,8 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_DL + 512;
   static constexpr int N_BARS = 1 + 6 * NS + 8;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int OFF_ENT = OFF_MISC + 16;           // int[kBwdChunk]: the unit's entries
+  static constexpr int SMEM_BYTES = OFF_ENT + 4 * kBwdChunk + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
   static_assert(NS * Q_BYTES >= KT * D * 4, "Q stages must hold an fp32 dK tile");
 };
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* bar_dk = bar_fin + 1;    // dK of the iteration complete (Q stage read)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int* s_ent = reinterpret_cast<int*>(smem + C::OFF_ENT);
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* s_dl = reinterpret_cast<float*>(smem + C::OFF_DL);
 
@@ -221,6 +223,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // work unit: a slice of one key tile's reverse list (long lists are split)
   const int4 unit = reinterpret_cast<const int4*>(p.plan + hdr->off_bwd_units)[
       p.plan[hdr->off_bwd_unit_order + rank]];
+  if (unit.z > kBwdChunk) {  // the plan never builds such a unit
+    if (threadIdx.x == 0) set_status(p.status, SINKATTN_ERR_PLAN);
+    return;
+  }
   const TileItem it = reinterpret_cast<const TileItem*>(p.plan + hdr->off_bwd_items)[unit.x];
   const bool split_tile = unit.w > 1;  // partial dK/dV go through fp32 reductions
   const int kvh = it.kvh >= 0 ? it.kvh : rem;
@@ -232,6 +238,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int k0 = it.tile_start;         // sequence-local first key
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the unit's reverse-list entries, read from shared memory by every role
+  // (a unit has at most kBwdChunk of them)
+  if ((int)threadIdx.x < unit.z) s_ent[threadIdx.x] = __ldg(ent + threadIdx.x);
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
     for (int s = 0; s < NS; ++s) {
@@ -290,7 +299,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         bool ok = true;
         for (int i = 0; i < n_it && ok; ++i) {
           const int s = i % NS;
-          const int e = __ldg(ent + i / PER_E);
+          const int e = s_ent[i / PER_E];
           const int q_tok = it.seq_start + q_first(i, e);
           const int h0 = h_first(i);
           const uint32_t par = ((i / NS) & 1) ^ 1;
@@ -452,7 +461,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (lane == 0 && n_it > 0) {
         for (int i = 0; i < n_it; ++i) {
           const int s = i % NS;
-          const int e = __ldg(ent + i / PER_E);
+          const int e = s_ent[i / PER_E];
           const int q_tok = it.seq_start + q_first(i, e);
           const int h0 = h_first(i);
           const uint32_t par = (i / NS) & 1;
@@ -576,7 +585,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // values are loaded one iteration ahead, so global-load latency stays off
     // the critical path.
     auto fetch = [&](int i, int& e, float& l2, float& dl) {
-      e = __ldg(ent + i / PER_E);
+      e = s_ent[i / PER_E];
       l2 = INFINITY;
       dl = 0.f;
       if (tw < CW) {

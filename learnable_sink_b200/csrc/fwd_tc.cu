@@ -389,6 +389,8 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + C::S_COL + t * TK;
     const uint32_t o_addr = tmem + lane_off + C::O_COL + t * D;
+    // the head's sink logit in log2 units, loaded before the key loop
+    const float sink_l2 = p.sink ? __ldg(p.sink + head) * kLog2e : -INFINITY;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -578,49 +580,40 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       tc_fence_before();
       mbar_arrive(bar_p + t);
     }
-    // epilogue: fold the sink into the denominator (log2 domain) and stream
-    // O out of tensor memory 32 columns at a time
-    const bool have_o =
-        __all_sync(0xffffffffu, n > 0 && ok && mbar_wait(bar_o + t, 0, abort_flag, p.status));
-    if (n > 0 && !have_o) ok = false;
+    // epilogue: fold the sink into the denominator (log2 domain), write LSE
+    // and sink_s while the last PV runs, then stream O out of tensor memory
+    // 32 columns at a time
+    const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
+    float o_scale = 0.f;
     if (ok && tok < it.tile_len) {
-      const float a2 = p.sink ? __ldg(p.sink + head) * kLog2e : -INFINITY;
-      const float mt = fmaxf(m, a2);
-      float o_scale = 0.f, lse_v = -INFINITY, ss = 0.f;
+      const float mt = fmaxf(m, sink_l2);
+      float lse_v = -INFINITY, ss = 0.f;
       if (mt != -INFINITY) {
         const float fr = (m == -INFINITY) ? 0.f : exp2f(m - mt);
         const float lr = l * fr;
-        const float den = lr + (p.sink ? exp2f(a2 - mt) : 0.f);
+        const float den = lr + (p.sink ? exp2f(sink_l2 - mt) : 0.f);
         o_scale = fr / den;
         lse_v = (mt + log2f(den)) * kLn2;
         ss = lr / den;
       }
-      const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
       p.lse[row] = lse_v;
       if (p.sink_s) p.sink_s[row] = ss;
       // the raw LSE over the visible keys (before the sink joins)
       if (p.lse_orig) p.lse_orig[row] = (m != -INFINITY && l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+    }
+    const bool have_o =
+        __all_sync(0xffffffffu, n > 0 && ok && mbar_wait(bar_o + t, 0, abort_flag, p.status));
+    if (n > 0 && !have_o) ok = false;
+    const bool store = ok && tok < it.tile_len;
+    if (store && !have_o) {  // no key tile: O is zero
       uint4* dst = reinterpret_cast<uint4*>(p.out + row * D);
-      if (!have_o) {
-        const uint4 z = make_uint4(0, 0, 0, 0);
+      const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) dst[c] = z;
-      }
+      for (int c = 0; c < D / 8; ++c) dst[c] = z;
     }
     if (have_o) {
       // all 32 lanes of the warp take part in the tcgen05.ld
       tc_fence_after();
-      const bool store = ok && tok < it.tile_len;
-      float o_scale = 0.f;
-      if (store) {
-        const float a2 = p.sink ? __ldg(p.sink + head) * kLog2e : -INFINITY;
-        const float mt = fmaxf(m, a2);
-        if (mt != -INFINITY) {
-          const float fr = (m == -INFINITY) ? 0.f : exp2f(m - mt);
-          const float den = l * fr + (p.sink ? exp2f(a2 - mt) : 0.f);
-          o_scale = fr / den;
-        }
-      }
       // A whole tile (every row stores) goes out through shared memory and a
       // bulk tensor store: the warpgroup writes its rows into its Q buffer
       // (every MMA that read Q is complete) in the layout the Q load used,
@@ -628,7 +621,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_BLOCKS)
       // per-row stores (the box would spill into the next sequence's rows).
       const bool whole = ok && it.tile_len == C::TQ;  // uniform over the warp
       uint8_t* qbuf = smem + C::OFF_Q + t * C::Q_BYTES;
-      const long long row = (long long)(it.seq_start + qi) * p.Hq + head;
       uint4* dst = reinterpret_cast<uint4*>(p.out + row * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
