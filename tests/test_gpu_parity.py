@@ -259,6 +259,55 @@ def test_decode_heads_and_many_splits(G, D, splits):
     _compare_decode(d, *_run_decode(d, splits), TOL[torch.bfloat16])
 
 
+def test_decode_workspace_contents_and_graph_replay():
+    # The workspace may hold anything before a call (all ones, random bytes,
+    # a previous call's partials): the merge reads only what the same call
+    # wrote.  A captured call replayed from a CUDA graph gives the same
+    # result every time.
+    d = W.decode(B=7, n_sink=4, window=200, Hq=8, Hkv=2, D=128, seqlen_range=(0, 260))
+    d.cache_seqlens[0] = 0
+    B, Hq, D = d.q.shape
+    Hkv = d.k_cache.shape[2]
+    ns = S.decode_num_splits(B, Hq, Hkv, D, d.n_sink, d.window)
+    nbytes = S.decode_workspace_bytes(B, Hq, D, ns)
+    q, kc, vc, cs, sk = (dev(d.q), dev(d.k_cache), dev(d.v_cache), dev(d.cache_seqlens),
+                         dev(d.sink))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device="cuda")
+    ss = torch.empty_like(lse)
+
+    def call():
+        S.decode(q, kc, vc, cs, d.n_sink, d.window, sk, scale=d.scale, num_splits=ns,
+                 workspace=ws, out=out, lse=lse, sink_s=ss)
+
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for fill in ("ones", "random", "leftover"):
+        if fill == "ones":
+            ws.fill_(255)
+        elif fill == "random":
+            ws.copy_(torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device="cuda", generator=g))
+        out.fill_(float("nan"))
+        call()
+        torch.cuda.synchronize()
+        _compare_decode(d, out.clone(), lse.clone(), ss.clone(), TOL[torch.bfloat16])
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()  # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        call()
+    for _ in range(3):
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        _compare_decode(d, out.clone(), lse.clone(), ss.clone(), TOL[torch.bfloat16])
+    del graph
+
+
 def test_decode_many_sequences():
     # more sequences than the streaming kernel stages cache lengths for in
     # shared memory (1024): the lengths are then read from global memory
