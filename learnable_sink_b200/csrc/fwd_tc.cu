@@ -1,4 +1,5 @@
-// Forward pass on the 5th-generation tensor cores (tcgen05) for bf16 inputs.
+// Forward pass on the 5th-generation tensor cores (tcgen05) for bf16 and f16
+// inputs (one template over the 16-bit element type).
 //
 // Page "Attention Sink, Learnable Sink and dsink": scores and GQA map
 // (section 1), the sink logit folded into the softmax denominator with a zero
@@ -19,7 +20,10 @@
 //                     softmax wrote it over S_t).
 // Tensor memory: S_t at columns [t TK, (t+1) TK), O_t after all S tiles.
 // The two query tiles ping-pong: while warpgroup 0 exponentiates S_0 the
-// tensor core runs tile 1's MMAs and vice versa.
+// tensor core runs tile 1's MMAs and vice versa.  With 64-key blocks at
+// D = 64 a CTA holds one query tile, two CTAs share an SM, and consecutive
+// score tiles sit in two overlapping regions (SDB below), so the next score
+// MMA runs while the softmax works on the current one.
 #include <cudaTypedefs.h>
 
 #include "internal.h"
