@@ -153,16 +153,10 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// Instruction descriptor for kind::f16: BF16 x BF16 -> FP32, dense.
-//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
-//   15 A major (0 = K), 16 B major, 17-22 N>>3, 24-28 M>>4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,
-                                                      int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
-         (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
-}
-// The same for a 16-bit operand format `fmt` (0 = f16, 1 = bf16; A and B of
-// one MMA always share it).
+// Instruction descriptor for kind::f16 with FP32 accumulation, dense:
+//   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (`fmt`: 0 =
+//   f16, 1 = bf16; A and B of one MMA always share it), 15 A major (0 = K),
+//   16 B major, 17-22 N>>3, 24-28 M>>4.
 __host__ __device__ constexpr uint32_t idesc_16_f32(uint32_t fmt, int M, int N, int a_mn_major,
                                                     int b_mn_major) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | (uint32_t(a_mn_major) << 15) |
