@@ -30,7 +30,9 @@
 // exponentiate tile i+1 (S^T(i+1) moves behind dQ(i) when its Q tile has not
 // landed yet).  Warps 0-7 compute (warpgroup c owns query columns
 // [c QR/2, (c + 1) QR/2), thread = key row); warps 8-11 move each dQ tile out
-// of tensor memory into the finished stage's shared memory; warp 12 is the TMA
+// of tensor memory into shared memory the iteration's MMAs have finished
+// reading (the stage's dO buffer, and the staged dS^T tile or the stage's Q
+// buffer); warp 12 is the TMA
 // producer, warp 13 issues MMAs and warp 14 adds the staged dQ tiles into an
 // fp32 buffer with bulk tensor reductions (a query row gets one contribution
 // per visible key tile); a small kernel converts it to bf16.
@@ -38,8 +40,11 @@
 // Two limits shape the schedule: the tensor cores read shared-memory operands
 // at about 128 bytes per cycle (a 128 x 128 x 16 SS MMA is already at that
 // rate, so every other shared-memory byte slows the MMAs), and an SM drains
-// about 20 bytes of dQ reductions per cycle, so a stage stays busy until its
-// fp32 dQ tile has left.  With 128-key tiles the query side uses 128 rows per
+// about 20 bytes of dQ reductions per cycle, so a buffer that holds a staged
+// fp32 dQ half stays busy until it has left.  Where the staged dS^T tile can
+// hold half of dQ it takes it, so the Q buffer, which the next S^T needs
+// first, goes back as soon as dK has read it (4 % on the D = 128 backward).
+// With 128-key tiles the query side uses 128 rows per
 // iteration: 64-row sub-tiles (supported by the template) halve the stage but
 // re-read K and V twice as often, which costs more shared-memory bandwidth
 // than the extra stages save.
@@ -82,6 +87,9 @@ struct BwdCfg {
   static constexpr int LAUNCH_REGS = 65536 / THREADS;
   static constexpr bool REBALANCE = QR == 128;
   static constexpr bool DQ_OWN = 2 * QR + 3 * D <= 512;   // dQ in columns of its own
+  // dQ over dP^T with a staged dS^T tile large enough for half a dQ tile:
+  // that half is staged there, not in the stage's Q buffer
+  static constexpr bool DQ_IN_DS = !DQ_OWN && KT * QR * 2 >= QR * D * 2;
   static constexpr int COMPUTE_REGS = REBALANCE ? 184 : LAUNCH_REGS;
   static constexpr int EPI_REGS = REBALANCE ? 72 : LAUNCH_REGS;
   static constexpr int AUX_REGS = REBALANCE ? 72 : LAUNCH_REGS;
@@ -98,7 +106,7 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DO + NS * Q_BYTES;   // float[QR]
   static constexpr int OFF_DL = OFF_LSE + 512;            // float[QR]
   static constexpr int OFF_BAR = OFF_DL + 512;
-  static constexpr int N_BARS = 1 + 6 * NS + 8;
+  static constexpr int N_BARS = 1 + 6 * NS + 9;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int OFF_ENT = OFF_MISC + 16;           // int[kBwdChunk]: the unit's entries
   static constexpr int SMEM_BYTES = OFF_ENT + 4 * kBwdChunk + 1024;
@@ -190,15 +198,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;
-  // Each stage is two buffers, Q and dO, with their own barriers: the dQ tile
-  // is staged as columns [0, D/2) in the Q buffer and [D/2, D) in the dO
-  // buffer, and each buffer goes back to the producer as soon as the bulk
+  // Each stage is two buffers, Q and dO, with their own barriers.  The dQ
+  // tile is staged as columns [D/2, D) in the dO buffer and columns [0, D/2)
+  // in the staged dS^T tile when that holds them (DQ_IN_DS: the Q buffer then
+  // goes back to the producer as soon as dK has read it), else in the Q
+  // buffer; each buffer that takes a half goes back as soon as the bulk
   // reduction has read its half.
   uint64_t* bar_qf = bars + 1;       // Q of stage s landed
   uint64_t* bar_df = bar_qf + NS;    // dO of stage s landed
   uint64_t* bar_qe = bar_df + NS;    // Q buffer of stage s free
   uint64_t* bar_de = bar_qe + NS;    // dO buffer of stage s free
-  uint64_t* bar_dqs = bar_de + NS;   // dQ half 0 of stage s staged in the Q buffer
+  uint64_t* bar_dqs = bar_de + NS;   // dQ half 0 of stage s staged
   uint64_t* bar_dds = bar_dqs + NS;  // dQ half 1 of stage s staged in the dO buffer
   uint64_t* bar_s = bar_dds + NS;
   uint64_t* bar_dp = bar_s + 1;
@@ -208,6 +218,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* bar_dqf = bar_dq + 1;
   uint64_t* bar_fin = bar_dqf + 1;
   uint64_t* bar_dk = bar_fin + 1;    // dK of the iteration complete (Q stage read)
+  // dQ over dP^T: the dQ half staged in the dS^T buffer has been read, so the
+  // next dS^T tile may be written there
+  uint64_t* bar_dsf = bar_dk + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* s_ent = reinterpret_cast<int*>(smem + C::OFF_ENT);
@@ -246,7 +259,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_qf + s, 1);
       mbar_init(bar_df + s, 1);
-      mbar_init(bar_qe + s, 1);    // released by the reducer warp
+      mbar_init(bar_qe + s, 1);    // released by the reducer or the MMA warp
       mbar_init(bar_de + s, 1);
       mbar_init(bar_dqs + s, 128); // every epilogue thread staged its part of the half
       mbar_init(bar_dds + s, 128);
@@ -259,6 +272,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(bar_dqf, 128);
     mbar_init(bar_fin, 1);
     mbar_init(bar_dk, 1);
+    mbar_init(bar_dsf, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -432,7 +446,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                      sdesc_at(mQ, st_off + kk * 2048), id_kv,
                      (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar_dk);  // the Q tile of the stage may now take staged dQ
+          mma_commit(bar_dk);  // what dK read may now take half of dQ
+          if constexpr (C::DQ_IN_DS) mma_commit(bar_qe + s);  // dK read the Q buffer last
           if (more) {
             if (!s_next) {
               ok = mbar_wait(bar_qf + s1, par1, abort_flag, p.status);
@@ -456,8 +471,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else if (warp == C::REDUCER_WARP) {
       // ---------------------------------------------------------- dQ reducer
       // Adds each staged fp32 dQ tile into the global accumulator with bulk
-      // tensor reductions, waits until they have read the stage, and hands
-      // the stage back to the producer; no other warp waits for this.
+      // tensor reductions, waits until they have read each half, and hands
+      // the dO buffer (and the Q buffer) back to the producer, or the staged
+      // dS^T tile back to the compute warps.
       if (lane == 0 && n_it > 0) {
         for (int i = 0; i < n_it; ++i) {
           const int s = i % NS;
@@ -470,7 +486,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int half = 0; half < 2 && got; ++half) {
             got = mbar_wait((half == 0 ? bar_dqs : bar_dds) + s, par, abort_flag, p.status);
             if (!got) break;
-            const uint8_t* stage = smem + (half == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES;
+            const uint8_t* stage =
+                half == 0 ? (C::DQ_IN_DS ? smem + C::OFF_DS : smem + C::OFF_Q + s * C::Q_BYTES)
+                          : smem + C::OFF_DO + s * C::Q_BYTES;
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
               tma_reduce_add_3d(&tmap_dq, stage + c * (QR * 128), (D / 2) * half + 32 * c, h0,
@@ -478,8 +496,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             bulk_commit();
           }
           if (!got) break;
-          bulk_wait_read1();         // the Q-buffer half has been read
-          mbar_arrive(bar_qe + s);
+          bulk_wait_read1();         // the first half has been read
+          mbar_arrive(C::DQ_IN_DS ? bar_dsf : bar_qe + s);
           bulk_wait_read0();         // the dO-buffer half too
           mbar_arrive(bar_de + s);
         }
@@ -489,9 +507,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   } else if (warp >= C::EPI_WARP0) {
     // ------------------------------------------------------------ dQ epilogue
     // Query row m of the dQ tile sits at lane m (QR = 128) or at lane
-    // m % 16 + 32 (m / 16) (QR = 64).  The stage's Q buffer takes columns
-    // [0, D/2) and its dO buffer columns [D/2, D), as fp32 boxes of 32 columns
-    // with the 128-byte swizzle.  Query
+    // m % 16 + 32 (m / 16) (QR = 64).  Columns [0, D/2) go to the staged dS^T
+    // tile (DQ_IN_DS) or the stage's Q buffer, columns [D/2, D) to its dO
+    // buffer, as fp32 boxes of 32 columns with the 128-byte swizzle.  Query
     // rows past the sequence end carry exact zeros (their P is 0), so adding
     // them is harmless.
     regs_to<C::EPI_REGS, C::LAUNCH_REGS>();
@@ -530,8 +548,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       } else {
         // Half 1 (columns [D/2, D), into the dO buffer, which dV and dP^T read
-        // before dQ ran) first, then, once dK is complete, half 0 (into the Q
-        // buffer, which dK reads); 32 columns at a time.  The dQ columns are
+        // before dQ ran) first, then, once dK is complete, half 0 (into the
+        // staged dS^T tile or the Q buffer, which dK reads); 32 columns at a
+        // time.  The dQ columns are
         // released after the last load, so dK(i + 1) cannot complete before
         // this wait for dK(i).
         bool got_dk = true;
@@ -548,7 +567,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             mbar_arrive(bar_dqf);  // the dQ columns may be overwritten
           }
           if (lane_ok && got_dk) {
-            uint8_t* row = smem + (hf == 0 ? C::OFF_Q : C::OFF_DO) + s * C::Q_BYTES +
+            uint8_t* row = (hf == 0 ? (C::DQ_IN_DS ? smem + C::OFF_DS : smem + C::OFF_Q + s * C::Q_BYTES)
+                                    : smem + C::OFF_DO + s * C::Q_BYTES) +
                            c * (QR * 128) + qrow * 128;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -734,10 +754,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           else
             tmem_st16(tmem + lane_off + C::DP_COL + CW * cw, ds);
         }
-        // The staged dS tile is free: dP^T of this iteration was issued after
-        // the previous dQ and dK MMAs, and its completion covers them.  Layout:
+        // The staged dS tile is free of MMA reads: dP^T of this iteration was
+        // issued after the previous dQ and dK MMAs, and its completion covers
+        // them (with DQ_IN_DS the wait above covers the dQ half staged there
+        // since).  Layout:
         // [QR / 64 atoms][keys][64 queries] with the 128-byte swizzle; dQ reads
         // it MN-major and (with dQ over dP^T) dK K-major.
+        if constexpr (C::DQ_IN_DS) {
+          if (i > 0) {  // the dQ half staged here in the previous iteration has been read
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_dsf, (i - 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+          }
+        }
         if (row_ok) {
           constexpr int CHUNKS = CW / 8;  // 16-byte chunks of this warpgroup's queries
           uint8_t* row = smem + C::OFF_DS + ((CW * cw) / 64) * (KT * 128) + r * 128;
